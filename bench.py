@@ -1,0 +1,454 @@
+"""Throughput of the ISD step on B200: committed tokens/s and roofline fractions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload qwen3_8b_b64|qwen3_8b_b1|tiny]
+
+One step = one isd_step over the whole batch: assemble the block, 36
+decoder layers (QKV / attention / O / MLP), LM head, verify-resample-
+propose and page bookkeeping, all in libisd.so's kernels. Weights are
+random-init (bf16 N(0, 0.02)) of the named shape, prompts uniform random
+tokens with seeded lengths, physical pages randomly permuted, KV filled by
+isd_prefill before timing. Accept-test uniforms are acceptance-controlled
+(each draft passes with probability 0.9, the pages' operating point) so the
+committed tokens per forward match a trained model's regime; the run with
+natural uniforms is reported beside it.
+
+Multi-GPU (torchrun): the method shards by request, so every rank runs an
+independent replica with its own batch (weak scaling, no collective in the
+step); time is the max over ranks, value the sum of all ranks' tokens.
+
+--impl reference times the CPU oracle (fp64 numpy) on a bounded sample of
+the same workload on rank 0 and extrapolates to the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOADS = {
+    # Qwen3-8B shape, batch 64, stride 4, prompt lengths U[512, 4096]
+    "qwen3_8b_b64": dict(shape=synth.QWEN3_8B, batch=64, stride=4, len_lo=512, len_hi=4096),
+    # Qwen3-8B shape, batch 1, stride 4, prompt 2048
+    "qwen3_8b_b1": dict(shape=synth.QWEN3_8B, batch=1, stride=4, len_lo=2048, len_hi=2048),
+    "tiny": dict(shape=synth.TINY, batch=1, stride=2, len_lo=32, len_hi=32),
+}
+ACCEPT_RATE = 0.9
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p.get("hbm_gbs", 6650.0), bf16=p.get("bf16_tflops", 1590.0),
+                    bf16_sus=p.get("bf16_tflops_sustained", 1400.0), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------ algorithmic ---
+
+def step_bytes_flops(shape, lens_now, B, N):
+    """Algorithmic bytes / flops of one step (weights once, KV once, logits once)."""
+    R = 2 * N - 1
+    w_params = shape.n_layers * shape.params_per_layer() + shape.vocab * shape.hidden
+    kv = sum(int(L) + R for L in lens_now) * shape.kv_bytes_per_token()
+    logits = B * R * shape.vocab * 4
+    flops = 2.0 * B * R * w_params
+    return 2 * w_params, kv, logits, flops
+
+
+# ---------------------------------------------------------------- CUDA arm ---
+
+def run_cuda(args, ws, rank, local):
+    import torch
+    import torch.distributed as dist
+    from strided_verify_propose_b200 import binding as Bd
+
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    wl = WORKLOADS[args.workload]
+    shape, B, N = wl["shape"], wl["batch"], wl["stride"]
+    R, P, V = 2 * N - 1, shape.page_size, shape.vocab
+    seed = 1000 + rank
+    total_steps = args.warmup + 3 * args.steps + 4
+    lens = synth.prompt_lengths(B, wl["len_lo"], wl["len_hi"], seed)
+    prompts = synth.prompts(shape, lens, seed)
+    maxp = -(-(int(lens.max()) + total_steps * N + R + 1) // P) + 1
+    need = [-(-(int(L) - 1 + R) // P) for L in lens]
+    num_pages = int(sum(need)) + B * (-(-total_steps * N // P) + 2)
+    table, free = synth.page_layout(need, num_pages, maxp, seed)
+
+    t0 = time.time()
+    weights = Bd.random_device_weights(shape, seed=seed)
+    G = shape.n_q_heads // shape.n_kv_heads
+    model = Bd.Model(shape, weights, max_batch=B, max_rows=max(B * R, B * (64 // G)),
+                     max_position=maxp * P)
+    kv = Bd.KVCache(shape, num_pages, table, free)
+    st = Bd.StepState(B, N, V, sample=False)
+    torch.cuda.synchronize()
+    t_setup = time.time() - t0
+    t0 = time.time()
+    Bd.prefill(model, kv, st, prompts)
+    torch.cuda.synchronize()
+    t_prefill = time.time() - t0
+    if int(st.status.item()) != 0:
+        raise RuntimeError(f"prefill status {int(st.status.item())}")
+
+    unif = np.stack([synth.controlled_uniforms(B, N, ACCEPT_RATE, seed, s) for s in range(total_steps)])
+    unif_nat = np.stack([synth.uniforms(B, R, seed + 77, s) for s in range(args.steps)])
+    unif_d = torch.from_numpy(unif).cuda()
+    unif_nat_d = torch.from_numpy(unif_nat).cuda()
+    hist = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
+    step_i = 0
+
+    def one(u, flags=0):
+        Bd.step(model, kv, st, u, flags)
+
+    for _ in range(args.warmup):
+        one(unif_d[step_i]); step_i += 1
+    torch.cuda.synchronize()
+    lens_before = st.seq_len.cpu().numpy().copy()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    # ---- timed region: K steps, inputs resident in HBM
+    stream = torch.cuda.current_stream()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e_start.record(stream)
+        for i in range(args.steps):
+            one(unif_d[step_i]); step_i += 1
+            hist[i].copy_(st.accepted)
+        e_stop.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = e_start.elapsed_time(e_stop)
+    launches_per_step = model.launches()
+    committed = int((hist.long() + 1).sum().item())
+    if int(st.status.item()) != 0:
+        raise RuntimeError(f"step status {int(st.status.item())}")
+
+    # ---- profiled region: same steps with per-kernel-class CUDA events
+    model.profile(True)
+    for i in range(args.steps):
+        one(unif_d[step_i]); step_i += 1
+    prof = model.profile_read()
+    model.profile(False)
+
+    # ---- natural uniforms (acceptance ~ 0 with random weights)
+    torch.cuda.synchronize()
+    n_start, n_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nat_hist = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
+    n_start.record(stream)
+    for i in range(args.steps):
+        one(unif_nat_d[i])
+        nat_hist[i].copy_(st.accepted)
+    n_stop.record(stream)
+    torch.cuda.synchronize()
+    nat_ms = n_start.elapsed_time(n_stop)
+    nat_committed = int((nat_hist.long() + 1).sum().item())
+
+    # ---- end to end through the C ABI with host buffers
+    pin_u = torch.from_numpy(unif[step_i:step_i + args.steps].copy()).pin_memory()
+    pin_acc = torch.zeros(args.steps, B, dtype=torch.int32).pin_memory()
+    pin_com = torch.zeros(args.steps, B, N, dtype=torch.int32).pin_memory()
+    u_dev = torch.empty(B, R, device="cuda", dtype=torch.float32)
+    torch.cuda.synchronize()
+    barrier()
+    x_start, x_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x_start.record(stream)
+    for i in range(args.steps):
+        u_dev.copy_(pin_u[i], non_blocking=True)
+        one(u_dev)
+        pin_acc[i].copy_(st.accepted, non_blocking=True)
+        pin_com[i].copy_(st.committed, non_blocking=True)
+        stream.synchronize()            # the host reads this step's committed tokens
+    x_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = x_start.elapsed_time(x_stop)
+    e2e_committed = int((pin_acc.long() + 1).sum().item())
+
+    # ---- reduce over ranks: max time, summed tokens
+    vals = torch.tensor([ms, e2e_ms, nat_ms], device="cuda", dtype=torch.float64)
+    toks = torch.tensor([committed, e2e_committed, nat_committed], device="cuda", dtype=torch.float64)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(toks, op=dist.ReduceOp.SUM)
+    ms, e2e_ms, nat_ms = vals.tolist()
+    committed, e2e_committed, nat_committed = toks.tolist()
+
+    result = None
+    if rank == 0:
+        peaks = load_peaks()
+        ms_step = ms / args.steps
+        wbytes, kvbytes, lbytes, flops = step_bytes_flops(shape, lens_before, B, N)
+        step_bytes = wbytes + kvbytes
+        hbm_frac_step = (step_bytes / (ms_step * 1e-3)) / (peaks["hbm"] * 1e9)
+        # ceiling: GEMMs at the tensor peak plus attention KV at HBM peak
+        t_floor = flops / (peaks["bf16"] * 1e12) + kvbytes / (peaks["hbm"] * 1e9)
+        ceiling = (step_bytes / (peaks["hbm"] * 1e9)) / t_floor
+        roof = roofline_entry(prof, shape, B, N, lens_before, args.steps, peaks)
+        result = {
+            "metric": "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
+            if args.workload == "qwen3_8b_b64" else f"committed tokens/s ({args.workload})",
+            "value": committed / (ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (random-init weights, uniform random prompts, seeded)",
+            "config": {"workload": args.workload, "model": "qwen3-8b-shape (random init)"
+                       if shape is synth.QWEN3_8B else "tiny", "batch_per_gpu": B,
+                       "global_batch": B * ws, "stride_n": N, "rows_per_step": B * R,
+                       "prompt_len": [wl["len_lo"], wl["len_hi"]], "page_size": P,
+                       "parallelism": f"replicas x{ws} (request-sharded, no collective)",
+                       "uniforms": f"acceptance-controlled a={ACCEPT_RATE}",
+                       "l2": "inputs larger than L2 (weights 16 GB + KV > 126 MB)"},
+            "tokens_per_forward": committed / (args.steps * B * ws),
+            "hbm_roofline_fraction_step": hbm_frac_step,
+            "hbm_roofline_ceiling_step": ceiling,
+            "step_algorithmic_bytes": step_bytes,
+            "natural_uniforms": {"value": nat_committed / (nat_ms * 1e-3), "unit": "tokens/s",
+                                 "tokens_per_forward": nat_committed / (args.steps * B * ws)},
+            "prefill_s": t_prefill, "setup_s": t_setup,
+            "gpu_launches": launches_per_step * args.steps,
+            "launches_per_step": launches_per_step,
+            "roofline": roof,
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in sorted(prof.items())},
+            "clocks": clk.summary(),
+            "e2e": {"value": e2e_committed / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": B * R * 4, "d2h_bytes_per_step": B * 4 + B * N * 4},
+            "peaks": peaks,
+        }
+    del model
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def roofline_entry(prof, shape, B, N, lens, steps, peaks):
+    """Roofline of the kernel class with the largest device time."""
+    if not prof:
+        return None
+    R = 2 * N - 1
+    top = max(prof, key=lambda k: prof[k][0])
+    tot_ms, cnt = prof[top]
+    avg_s = tot_ms / cnt * 1e-3
+    M = B * R
+    h, I, V = shape.hidden, shape.intermediate, shape.vocab
+    gemm_flops = {"gemm_qkv": 2 * M * h * shape.qkv_dim, "gemm_o": 2 * M * shape.q_dim * h,
+                  "gemm_gate_up_silu": 2 * M * h * 2 * I, "gemm_down": 2 * M * I * h,
+                  "gemm_lm_head": 2 * M * h * V}
+    if top in gemm_flops:
+        achieved = gemm_flops[top] / avg_s / 1e12
+        peak = peaks["bf16_sus"]
+        return {"kernel": top, "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_kind": f"{peaks['source']} sustained bf16",
+                "avg_launch_ms": avg_s * 1e3, "launches": cnt}
+    if top.startswith("attention"):
+        kv = sum(int(L) + R for L in lens) * shape.kv_dim * 2 * 2   # one layer's K+V
+        achieved = kv / avg_s / 1e9
+        peak = peaks["hbm"]
+        return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None, "peak_kind": f"{peaks['source']} HBM copy",
+                "avg_launch_ms": avg_s * 1e3, "launches": cnt}
+    return {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": None, "traffic": None, "avg_launch_ms": avg_s * 1e3, "launches": cnt}
+
+
+# ------------------------------------------------------------ oracle arm ---
+
+def oracle_sample(args, n_reps: int, workload: str):
+    """Time the oracle on a bounded sample of the workload and extrapolate.
+
+    Sample: one decoder layer at the workload's widths and one 1/16 slice of
+    the LM head, run by the oracle's own block forward for one request's
+    2N-1 rows against a random KV prefix of the batch's mean length, plus
+    the oracle's decide() on the full-vocabulary logits of that request.
+    Full step time = batch x (layers x t_layer + 16 x t_lm_slice + t_decide).
+    """
+    from oracle import isd as oi
+    from oracle import model as om
+    wl = WORKLOADS[workload]
+    shape, B, N = wl["shape"], wl["batch"], wl["stride"]
+    R = 2 * N - 1
+    slice_v = max(shape.vocab // 16, 128)
+    one = dataclasses.replace(shape, n_layers=1, vocab=slice_v)
+    w = synth.decoder_weights(one, seed=5)
+    dec = om.Decoder(one, w)
+    L = int(np.mean(synth.prompt_lengths(B, wl["len_lo"], wl["len_hi"], 1000)))
+    kv = om.DenseKV(one)
+    kv.k[0] = synth.normal((L, one.n_kv_heads, one.head_dim), 3, 1).astype(np.float64)
+    kv.v[0] = synth.normal((L, one.n_kv_heads, one.head_dim), 3, 2).astype(np.float64)
+    kv.n = L
+    z_full = synth.synthetic_logits(R, shape.vocab, 4, boost=7.5).astype(np.float64)
+    times, committed = [], 0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    for rep in range(n_reps):
+        u = synth.controlled_uniforms(1, N, ACCEPT_RATE, 9, rep)[0]
+        drafts = [int(np.argmax(z_full[j])) for j in range(N - 1)]
+        # the sliced model's vocabulary holds the block's tokens
+        toks = [1] + [t % slice_v for t in drafts] + [one.mask_token_id] * (R - N)
+        t0 = time.perf_counter()
+        om.block_forward(dec, kv, toks, L + np.arange(R))
+        t1 = time.perf_counter()
+        d = oi.decide(z_full, drafts, None, N, u)
+        t2 = time.perf_counter()
+        t_fwd = t1 - t0
+        # the forward above = 1 layer + embedding + LM-head slice; time the slice alone too
+        t3 = time.perf_counter()
+        x = np.ones((R, shape.hidden))
+        _ = om.rms_norm(x, dec.final_norm, shape.rms_eps) @ dec.lm_head.T
+        t_lm = time.perf_counter() - t3
+        t_layer = max(t_fwd - t_lm, 1e-9)
+        t_step = B * (shape.n_layers * t_layer + (shape.vocab / slice_v) * t_lm + (t2 - t1))
+        times.append(t_step)
+        committed += B * (d.accepted + 1)
+    per_step = float(np.mean(times))
+    value = (committed / n_reps) / per_step
+    sample = (f"{n_reps} reps of: 1 decoder layer at {workload} widths + 1/{shape.vocab // slice_v} "
+              f"LM-head slice for one request's {R} rows against a random KV prefix of {L} "
+              f"positions, plus decide() on full-vocab logits; extrapolated x{shape.n_layers} "
+              f"layers, full LM head, batch {B}")
+    return value, threads, sample, per_step
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return None
+    reps = max(1, args.steps)
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(args, 1, args.workload)
+    t0 = time.time()
+    value, threads, sample, per_step = oracle_sample(args, reps, args.workload)
+    wl = WORKLOADS[args.workload]
+    return {"metric": "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
+            if args.workload == "qwen3_8b_b64" else f"committed tokens/s ({args.workload})",
+            "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "batch_per_gpu": wl["batch"],
+                                             "stride_n": wl["stride"]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample, "wall_s": time.time() - t0},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="qwen3_8b_b64", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = setup_dist()
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res = run_cuda(args, ws, rank, local)
+    if res is not None:
+        if ws == 1 and not args.no_cpu_baseline:
+            v, threads, sample, _ = oracle_sample(args, 2, args.workload)
+            res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                   "sample": sample}
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+/*
+ * isd.h - C ABI of the B200 (sm_100a) Introspective Strided Decoding library.
+ *
+ * One ISD step: every request of a batch runs one strictly causal forward of
+ * a Qwen3-shaped decoder over a block [x* | N-1 pending drafts | N-1 MASK]
+ * against its paged KV prefix; the drafts are verified left to right with
+ * u < min(1, p/q) (p: this forward's anchor, q: the previous forward's
+ * proposal), the first rejected slot is refilled from norm(max(0, p - q)),
+ * and the MASK rows propose the next drafts.
+ *   Sources: Bud's Wiki "Introspective Diffusion Language Models" (TL;DR,
+ *   Key claims, Method); Agentic Commons blog of the same title ("How
+ *   Introspective Strided Decoding Works"); GeekNews (hi/pt) summaries
+ *   ("Inference & ISD", "Lossless R-ISD", "Speedup Factor Explorer").
+ *
+ * Block layout (rows r = 0..2N-2 at positions L..L+2N-2, L = committed length):
+ *   full step (n = N-1 drafts):  [x*, d_1..d_{N-1}, MASK x (N-1)]
+ *   restart step (n = 0):        [x*, MASK x (N-1), MASK padding x (N-1)]
+ * Row t scores the token at position t+1 (logit shift). Draft d_j is tested
+ * on row j-1; the new final token comes from row A (A = accepted drafts);
+ * rows n+1..n+N-1 propose the next drafts when no draft was rejected.
+ * Uniform slots per request (2N-1 floats in [0,1)): [0, N-1) accept tests,
+ * [N-1] the new token, [N, 2N-1) sampled proposals.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are device memory owned by the caller; the library
+ *    never frees or reallocates them. Host arrays of device pointers are
+ *    copied during the call that receives them.
+ *  - Matrices are row-major. "nn.Linear layout" means [out_features][in_features].
+ *  - bf16 means IEEE bfloat16 (torch.bfloat16).
+ *  - Functions return ISD_OK (0) or a negative ISD_E_* code; the text of the
+ *    last error of the calling thread is returned by isd_last_error().
+ *  - Work is enqueued on the given cudaStream_t (passed as void*); nothing
+ *    synchronises the stream. Faults found on the device (pool exhausted,
+ *    token or page id out of range, a bounded wait that ran out) are OR-ed
+ *    into the caller's int32 status word as ISD_DEV_* bits; read it after
+ *    synchronising. No kernel traps or asserts.
+ */
+#ifndef ISD_H_
+#define ISD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------ */
+#define ISD_OK             0
+#define ISD_E_INVALID     -1  /* null pointer, size or flag out of range            */
+#define ISD_E_UNSUPPORTED -2  /* a shape the kernels do not implement               */
+#define ISD_E_CUDA        -3  /* a CUDA runtime call failed                         */
+#define ISD_E_NOMEM       -4  /* workspace allocation failed (isd_init only)        */
+
+/* ---- device status bits (OR-ed into *status_dev) ----------------------- */
+#define ISD_DEV_POOL_EXHAUSTED 0x01 /* free list too short: no page handed out  */
+#define ISD_DEV_TABLE_FULL     0x02 /* a request outgrew max_pages_per_req      */
+#define ISD_DEV_BAD_TOKEN      0x04 /* token id outside [0, vocab)              */
+#define ISD_DEV_BAD_PAGE       0x08 /* page id outside [0, num_pages)           */
+#define ISD_DEV_TIMEOUT        0x10 /* a bounded device wait ran out            */
+#define ISD_DEV_BAD_STATE      0x20 /* n_draft not 0 or N-1, or length < 0      */
+
+/* ---- step mode flags ---------------------------------------------------- */
+#define ISD_PROPOSE_ARGMAX 0x0  /* MASK rows propose by argmax (lowest index on ties) */
+#define ISD_PROPOSE_SAMPLE 0x1  /* MASK rows sample; q rows stored in q_cache         */
+#define ISD_VERIFY_SAMPLE  0x0  /* u*q(d) < p(d) test, residual / bonus sampling      */
+#define ISD_VERIFY_GREEDY  0x2  /* temperature 0: accept iff d == argmax p            */
+#define ISD_USE_LORA       0x4  /* add the loaded gated LoRA on MASK rows only        */
+
+/* ---- model ------------------------------------------------------------- */
+typedef struct {
+  int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, intermediate, vocab;
+  float rope_theta;      /* NeoX rotate-half RoPE base (1e6 for Qwen3)            */
+  float rms_eps;         /* RMSNorm epsilon                                       */
+  int32_t mask_token_id; /* token fed to MASK rows                                */
+  int32_t page_size;     /* KV positions per page: 16, 32 or 64                   */
+  int32_t max_batch;     /* most requests one call may carry (workspace size)      */
+  int32_t max_rows;      /* most block rows one call may process (workspace size) */
+  int32_t max_position;  /* positions must stay below this (RoPE table size, and
+                            max_pages_per_req * page_size <= max_position)         */
+} isd_model_cfg;
+/* Supported: head_dim 64 or 128; hidden, n_q_heads*head_dim, intermediate
+ * multiples of 128 (intermediate of 64); n_q_heads/n_kv_heads in {1,2,4,8};
+ * vocab a multiple of 128. */
+
+typedef struct {
+  const void *embed_dev;        /* [vocab][hidden] bf16                                  */
+  const void *lm_head_dev;      /* [vocab][hidden] bf16 (nn.Linear layout, untied)       */
+  const float *final_norm_dev;  /* [hidden] fp32                                         */
+  /* host arrays of n_layers device pointers each:                                      */
+  const void *const *w_qkv;     /* [(nq+2nkv)*head_dim][hidden] bf16: q rows, k rows, v rows */
+  const void *const *w_o;       /* [hidden][nq*head_dim] bf16                            */
+  const void *const *w_gate_up; /* [2*intermediate][hidden] bf16; row block t of 128 holds
+                                   gate rows 64t..64t+63 then up rows 64t..64t+63       */
+  const void *const *w_down;    /* [hidden][intermediate] bf16                           */
+  const float *const *attn_norm;/* [hidden] fp32 (pre-attention RMSNorm weight)          */
+  const float *const *mlp_norm; /* [hidden] fp32 (pre-MLP RMSNorm weight)                */
+  const float *const *q_norm;   /* [head_dim] fp32 (per-head RMSNorm of q)               */
+  const float *const *k_norm;   /* [head_dim] fp32 (per-head RMSNorm of k)               */
+} isd_weights;
+
+/* Gated LoRA of R-ISD (Bud's Wiki, Key claims and Method: rank 128, active
+ * only at MASK positions, verify positions on base weights). Targets in
+ * order q, k, v, o, gate, up, down; each a host array of n_layers device
+ * pointers. A_t: [rank][in_t] bf16, B_t: [out_t][rank] bf16 (the two
+ * nn.Linear weights); delta = scale * (x A_t^T) B_t^T on MASK rows only. */
+typedef struct {
+  int32_t rank;     /* multiple of 64, at most 256 */
+  float scale;
+  const void *const *A[7];
+  const void *const *B[7];
+} isd_lora;
+
+/* ---- per-call state (all device memory, caller-owned) ------------------ */
+typedef struct {
+  int32_t batch;       /* B requests, 1..1024                                   */
+  int32_t stride_n;    /* N, 1..8                                               */
+  int32_t flags;       /* ISD_PROPOSE_* | ISD_VERIFY_* | ISD_USE_LORA            */
+  int32_t *seq_len_dev;/* [B] committed length L_b (updated: L_b += 1 + A_b)     */
+  int32_t *n_draft_dev;/* [B] pending drafts, 0 or N-1 (updated)                 */
+  float *logits_out_dev; /* optional [B*(2N-1)][vocab] fp32 block logits, or NULL */
+} isd_batch;
+
+typedef struct {
+  void *k_pool_dev;    /* [n_layers][num_pages][n_kv_heads][page_size][head_dim] bf16;
+                          must be initialised to finite values (e.g. zeros)       */
+  void *v_pool_dev;    /* same layout as k_pool_dev                              */
+  int32_t *page_table_dev; /* [B][max_pages_per_req] physical page ids (updated) */
+  const int32_t *free_list_dev; /* [free_count] page ids handed out in order     */
+  int32_t *free_head_dev;       /* [1] next unused free_list entry (updated)      */
+  int32_t num_pages, max_pages_per_req, free_count;
+} isd_kv;
+/* Invariant at entry of isd_step: request b holds valid pages for positions
+ * [0, seq_len[b] + 2N - 1). The step keeps it for the updated lengths. */
+
+typedef struct isd_ctx isd_ctx;
+
+/* Create a context: copies cfg and the weight pointer arrays (the weights
+ * stay caller-owned and must outlive the context), builds TMA descriptors,
+ * the RoPE table and the workspace (the library's only allocation).
+ * Returns ISD_E_UNSUPPORTED for shapes outside the list above. */
+int isd_init(const isd_model_cfg *cfg, const isd_weights *w, isd_ctx **out);
+
+/* Attach a gated LoRA (copies the pointer arrays; the tensors stay
+ * caller-owned). Steps use it when flags has ISD_USE_LORA. */
+int isd_load_gated_lora(isd_ctx *ctx, const isd_lora *lora);
+
+/* One ISD step for the whole batch (enqueue only; CUDA-graph capturable).
+ *  pending_dev   [B][N] int32: x* then the n drafts (in); next x* then the
+ *                next drafts (out).
+ *  q_cache_dev   [B][N-1][vocab] fp32 proposal distributions of the pending
+ *                drafts (read) and of the next drafts (written); used only
+ *                with ISD_PROPOSE_SAMPLE, may be NULL otherwise.
+ *  uniforms_dev  [B][2N-1] fp32 in [0,1), slot map above.
+ *  out_accepted_dev  [B] int32: A_b in [0, n_b].
+ *  out_committed_dev [B][N] int32: the A_b accepted drafts then the new
+ *                final token (A_b + 1 valid entries), or NULL.
+ *  status_dev    [1] int32 device status word (bits OR-ed in).
+ *  stream        cudaStream_t. */
+int isd_step(isd_ctx *ctx, const isd_batch *batch, const isd_kv *kv, int32_t *pending_dev,
+             float *q_cache_dev, const float *uniforms_dev, int32_t *out_accepted_dev,
+             int32_t *out_committed_dev, int32_t *status_dev, void *stream);
+
+/* Prefill prompts into the paged KV cache and set the starting state:
+ * KV of positions [0, len_b - 1), seq_len = len_b - 1, pending[b][0] =
+ * last prompt token, n_draft = 0 (so the first step is a restart step).
+ *  tokens_dev [B][max_len] int32; lens_host [B] host int32, 1 <= len <= max_len.
+ * Pages for positions [0, len_b - 1 + 2N - 1) must already be in the page
+ * table. Rows are processed in chunks through the same kernels as a step. */
+int isd_prefill(isd_ctx *ctx, const isd_kv *kv, const int32_t *tokens_dev, int32_t max_len,
+                const int32_t *lens_host, int32_t batch, int32_t stride_n,
+                int32_t *seq_len_dev, int32_t *n_draft_dev, int32_t *pending_dev,
+                int32_t *status_dev, void *stream);
+
+/* Number of kernel launches the last isd_step / isd_prefill enqueued. */
+int isd_last_launch_count(const isd_ctx *ctx);
+
+/* Per-kernel-class timing with CUDA events recorded around each launch on
+ * the step's stream (for measurement; off by default, not for use inside a
+ * CUDA graph capture). isd_profile_read synchronises on the last recorded
+ * event, writes the summed milliseconds and launch counts of each class
+ * (ISD_PROF_CLASSES entries) and clears the record. */
+#define ISD_PROF_CLASSES 16
+int isd_profile_enable(isd_ctx *ctx, int enable);
+int isd_profile_read(isd_ctx *ctx, double *total_ms, int32_t *counts);
+const char *isd_profile_class_name(int cls);
+
+const char *isd_last_error(void);
+void isd_destroy(isd_ctx *ctx);
+
+/* ---- component entry points (used by the tests; same kernels as a step) -- */
+
+/* Y = X W^T on the tcgen05 tensor cores, fp32 accumulate.
+ *  w_dev [n][k] bf16 (nn.Linear layout), x_dev [m][k] bf16,
+ *  y_dev [split_k][m][n] fp32: split s holds the partial sum over its share
+ *  of k (the caller adds the splits). n % 128 == 0, k % 64 == 0,
+ *  1 <= m <= 4096, 1 <= split_k <= 16. */
+int isd_gemm_bf16(const void *w_dev, const void *x_dev, float *y_dev, int32_t m, int32_t n,
+                  int32_t k, int32_t split_k, int32_t *status_dev, void *stream);
+
+/* Paged causal GQA attention for one layer.
+ *  q_dev [B*R][n_q_heads][head_dim] bf16 (already QK-normed and rotated)
+ *  row_pos_dev [B*R] int32: position of each row; a row sees keys t <= pos
+ *  (pos < 0: no keys, output 0). Keys live in the pools at layer `layer`.
+ *  out_dev [B*R][n_q_heads*head_dim] bf16.
+ *  workspace_dev: isd_attention_workspace_bytes(...) bytes of device memory. */
+size_t isd_attention_workspace_bytes(int32_t batch, int32_t rows_per_req, int32_t n_q_heads,
+                                     int32_t n_kv_heads, int32_t head_dim,
+                                     int32_t max_pages_per_req, int32_t page_size);
+int isd_paged_attention(const void *q_dev, const int32_t *row_pos_dev, const void *k_pool_dev,
+                        const void *v_pool_dev, const int32_t *page_table_dev, int32_t batch,
+                        int32_t rows_per_req, int32_t n_q_heads, int32_t n_kv_heads,
+                        int32_t head_dim, int32_t page_size, int32_t num_pages,
+                        int32_t max_pages_per_req, int32_t n_layers, int32_t layer,
+                        void *out_dev, void *workspace_dev, size_t workspace_bytes,
+                        int32_t *status_dev, void *stream);
+
+/* Verify / resample / propose from given block logits, then the length and
+ * page bookkeeping: the tail of isd_step without the forward.
+ *  logits_dev [B*(2N-1)][vocab] fp32; other arguments as in isd_step (kv
+ *  supplies page_table / free list / num_pages / max_pages_per_req / page_size).
+ *  workspace_dev: isd_accept_workspace_bytes(B, N, vocab) bytes. */
+size_t isd_accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab);
+int isd_accept_propose(const float *logits_dev, const isd_batch *batch, const isd_kv *kv,
+                       int32_t page_size, int32_t vocab, int32_t *pending_dev,
+                       float *q_cache_dev, const float *uniforms_dev,
+                       int32_t *out_accepted_dev, int32_t *out_committed_dev,
+                       void *workspace_dev, size_t workspace_bytes, int32_t *status_dev,
+                       void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ISD_H_ */

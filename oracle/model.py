@@ -69,22 +69,51 @@ class DenseKV:
     def __init__(self, shape):
         self.k = [np.zeros((0, shape.n_kv_heads, shape.head_dim)) for _ in range(shape.n_layers)]
         self.v = [np.zeros((0, shape.n_kv_heads, shape.head_dim)) for _ in range(shape.n_layers)]
+        self.n = 0           # committed positions (kept separately so 0 layers works)
 
     @property
     def length(self) -> int:
-        return self.k[0].shape[0]
+        return self.n
 
     def keep(self, n: int) -> None:
         """Truncate every layer's history to its first n positions."""
         for l in range(len(self.k)):
             self.k[l] = self.k[l][:n]
             self.v[l] = self.v[l][:n]
+        self.n = min(self.n, n)
 
     def copy(self) -> "DenseKV":
         c = DenseKV.__new__(DenseKV)
         c.k = [a.copy() for a in self.k]
         c.v = [a.copy() for a in self.v]
+        c.n = self.n
         return c
+
+
+def causal_gqa_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, q_pos: np.ndarray,
+                         k_pos: np.ndarray) -> np.ndarray:
+    """Grouped-query causal softmax attention.
+
+    q [R, n_q, d] at positions q_pos; K, V [T, n_kv, d] at positions k_pos.
+    Query head h reads KV head h // (n_q / n_kv); row r sees keys with
+    k_pos <= q_pos[r]; scores are scaled by 1/sqrt(d). Returns [R, n_q, d]
+    (a row with no visible key returns zeros).
+    """
+    R, n_q, d = q.shape
+    G = n_q // K.shape[1]
+    att = np.zeros((R, n_q, d))
+    scale = 1.0 / np.sqrt(d)
+    for r in range(R):
+        visible = k_pos <= q_pos[r]
+        if not visible.any():
+            continue
+        for hq in range(n_q):
+            g = hq // G
+            sc = (K[visible, g, :] @ q[r, hq]) * scale
+            w = np.exp(sc - sc.max())
+            w /= w.sum()
+            att[r, hq] = w @ V[visible, g, :]
+    return att
 
 
 def _proj(m: Decoder, l: int, name: str, wname: str, x: np.ndarray,
@@ -113,7 +142,6 @@ def block_forward(m: Decoder, kv: DenseKV, tokens: Sequence[int], positions: Seq
     tokens = np.asarray(tokens, dtype=np.int64)
     pos = np.asarray(positions, dtype=np.int64)
     R = len(tokens)
-    G = s.n_q_heads // s.n_kv_heads
     T = kv.length
     key_pos_prefix = np.arange(T, dtype=np.int64)
     x = m.embed[tokens].copy()
@@ -130,16 +158,7 @@ def block_forward(m: Decoder, kv: DenseKV, tokens: Sequence[int], positions: Seq
         K = np.concatenate([kv.k[l], k], axis=0)            # [T+R, n_kv, d]
         V = np.concatenate([kv.v[l], v], axis=0)
         kpos = np.concatenate([key_pos_prefix, pos])
-        att = np.zeros((R, s.n_q_heads, s.head_dim))
-        scale = 1.0 / np.sqrt(s.head_dim)
-        for r in range(R):
-            visible = kpos <= pos[r]
-            for hq in range(s.n_q_heads):
-                g = hq // G
-                sc = (K[visible, g, :] @ q[r, hq]) * scale
-                w = np.exp(sc - sc.max())
-                w /= w.sum()
-                att[r, hq] = w @ V[visible, g, :]
+        att = causal_gqa_attention(q, K, V, pos, kpos)
         x = x + _proj(m, l, "o", "wo", att.reshape(R, s.q_dim), lora_rows)
         h = rms_norm(x, lw["mlp_norm"], s.rms_eps)
         a = silu(_proj(m, l, "gate", "w_gate", h, lora_rows)) * _proj(m, l, "up", "w_up", h, lora_rows)
@@ -155,6 +174,7 @@ def commit_kv(kv: DenseKV, block_k, block_v, n_rows: int) -> None:
     for l in range(len(kv.k)):
         kv.k[l] = np.concatenate([kv.k[l], block_k[l][:n_rows]], axis=0)
         kv.v[l] = np.concatenate([kv.v[l], block_v[l][:n_rows]], axis=0)
+    kv.n += n_rows
 
 
 def prefill(m: Decoder, tokens: Sequence[int]) -> DenseKV:

@@ -1,0 +1,285 @@
+// Dense bf16 projection GEMMs on the tcgen05 tensor cores (sm_100a).
+//
+// Y[m][n_out] = X[m][k] * W[n_out][k]^T, with W a weight matrix in
+// nn.Linear layout and X the block's activations. Decode blocks are short
+// (m = B * (2N-1) rows, 7..448 at stride 4), so the kernel swaps the roles:
+// 128 weight rows form the UMMA M side and all of a CTA's token rows (up to
+// 512) form N, so every weight byte is read from HBM once and the fp32
+// accumulators of the whole token range sit in tensor memory (<= 512 columns).
+//
+// Per CTA: warp 0 (one lane) issues TMA loads of a 128x64 weight tile and an
+// n_pad x 64 activation tile per K-block into a ring of shared-memory
+// stages; warp 1 (one lane) issues tcgen05.mma and releases each stage with
+// tcgen05.commit; then all four warps read the accumulators back with
+// tcgen05.ld (one TMEM lane per thread = one output feature) and store.
+// Split-K CTAs write their partial sums to separate slices that a row-wise
+// kernel adds in a fixed order, so results are bitwise reproducible.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace isd {
+
+namespace {
+
+constexpr int kTileM = 128;                 // weight rows per CTA
+constexpr int kTileK = 64;                  // K elements per stage (128 bytes)
+constexpr int kStageA = kTileM * kTileK * 2;  // 16 KB
+constexpr size_t kMaxSmem = 232448;         // 227 KB dynamic shared memory
+
+struct GemmParams {
+  int32_t m, n_out, kb_total, kb_per_split;
+  int32_t n_pad, n_mma, mma_n, box_rows, n_boxes, stages;
+  uint32_t tmem_cols;
+  int32_t epi;
+  float* out;
+  __nv_bfloat16* out_act;
+  int64_t split_stride;
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(128, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_w,
+                      const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int mt = blockIdx.x;
+  const int tok0 = blockIdx.y * p.n_pad;
+  const int sp = blockIdx.z;
+  const int kb0 = sp * p.kb_per_split;
+  const int nkb = min(p.kb_total, kb0 + p.kb_per_split) - kb0;
+  const uint32_t stage_bytes = kStageA + static_cast<uint32_t>(p.n_pad) * 128u;
+
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
+  uint64_t* empty = full + p.stages;
+  uint64_t* accum = empty + p.stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmap_w);
+    prefetch_tensormap(&tmap_x);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_x = policy_evict_last();
+    const uint32_t tx = kStageA + static_cast<uint32_t>(p.n_boxes * p.box_rows) * 128u;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % p.stages;
+      const uint32_t ph = (i / p.stages) & 1;
+      if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
+        flag(p.status, ISD_DEV_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      uint8_t* sa = smem + s * stage_bytes;
+      uint8_t* sb = sa + kStageA;
+      const int kc = (kb0 + i) * kTileK;
+      mbar_arrive_expect_tx(&full[s], tx);
+      tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
+      for (int bx = 0; bx < p.n_boxes; ++bx)
+        tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc, tok0 + bx * p.box_rows,
+                         pol_x);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_m128(static_cast<uint32_t>(p.mma_n));
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % p.stages;
+      const uint32_t ph = (i / p.stages) & 1;
+      if (!mbar_wait(&full[s], ph) || *abort_flag) {
+        flag(p.status, ISD_DEV_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(smem + s * stage_bytes);
+      const uint32_t b_base = a_base + kStageA;
+#pragma unroll
+      for (int kk = 0; kk < kTileK / 16; ++kk) {
+        const uint64_t da = sw128_desc(a_base + kk * 32);
+        for (int j = 0; j < p.n_mma; ++j) {
+          const uint64_t db = sw128_desc(b_base + j * p.mma_n * 128 + kk * 32);
+          umma_bf16(tmem + j * p.mma_n, da, db, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      umma_commit(&empty[s]);
+    }
+    umma_commit(accum);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: TMEM -> registers -> global
+  const bool ok = __syncthreads_and(mbar_wait(accum, 0) && !*abort_flag);
+  tc_fence_after();
+  if (!ok) {
+    if (threadIdx.x == 0) flag(p.status, ISD_DEV_TIMEOUT);
+  } else {
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int nchunk = (p.n_pad + 31) / 32;  // tmem_cols >= 32 * nchunk
+    if (p.epi == kEpiF32) {
+      const int f = mt * kTileM + warp * 32 + lane;
+      float* outp = p.out + sp * p.split_stride + f;
+      for (int c = 0; c < nchunk; ++c) {
+        float v[32];
+        tmem_ld_32x32(lane_addr + c * 32, v);
+        const int t0 = tok0 + c * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j < p.n_pad && t0 + j < p.m)
+            outp[static_cast<int64_t>(t0 + j) * p.n_out] = v[j];
+      }
+    } else {
+      // rows 0..63 of the tile are gate features, rows 64..127 the matching up features
+      float* xch = reinterpret_cast<float*>(smem);  // stage 0 is free now: [64][33]
+      const int half_n = p.n_out / 2;
+      const int fo = mt * 64 + (warp & 1) * 32 + lane;
+      for (int c = 0; c < nchunk; ++c) {
+        float v[32];
+        tmem_ld_32x32(lane_addr + c * 32, v);
+        if (warp >= 2) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xch[((warp - 2) * 32 + lane) * 33 + j] = v[j];
+        }
+        __syncthreads();
+        if (warp < 2) {
+          const int t0 = tok0 + c * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (c * 32 + j < p.n_pad && t0 + j < p.m) {
+              const float g = v[j];
+              const float u = xch[(warp * 32 + lane) * 33 + j];
+              const float a = g / (1.0f + expf(-g)) * u;
+              p.out_act[static_cast<int64_t>(t0 + j) * half_n + fo] = __float2bfloat16_rn(a);
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+uint32_t pow2_at_least(uint32_t v) {
+  uint32_t r = 32;
+  while (r < v) r <<= 1;
+  return r;
+}
+
+}  // namespace
+
+GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, int32_t max_splits,
+                   int32_t num_sms) {
+  GemmPlan best;
+  const int kb_total = k / kTileK;
+  const int m_tiles = n_out / kTileM;
+  const int min_chunks = (m + 511) / 512;
+  double best_t = 1e30;
+  for (int nch = min_chunks; nch <= std::max(min_chunks * 4, 1); ++nch) {
+    const int tok = (m + nch - 1) / nch;
+    int n_pad = tok <= 256 ? ((tok + 15) / 16) * 16 : ((tok + 31) / 32) * 32;
+    if (n_pad > 512) continue;
+    if (nch > min_chunks && n_pad < 64) break;  // finer chunks only help big blocks
+    const int s_lo = force_splits > 0 ? force_splits : 1;
+    const int s_hi = force_splits > 0 ? force_splits : std::min(max_splits, kb_total);
+    for (int s = s_lo; s <= s_hi; ++s) {
+      const int kbs = (kb_total + s - 1) / s;
+      if ((s - 1) * kbs >= kb_total) continue;  // an empty split
+      const long units = static_cast<long>(m_tiles) * nch * s;
+      const long waves = (units + num_sms - 1) / num_sms;
+      const long active = std::min<long>(units, num_sms);
+      // cycles per K-block: tensor time vs weight streaming (HBM shared by active CTAs)
+      const double t_mma = 2.0 * n_pad;
+      const double t_hbm = 16384.0 / std::min(64.0, 3400.0 / active);
+      const double t_kb = std::max(t_mma, t_hbm) + 40.0;
+      const double t_epi = 4.0 * n_pad;                     // TMEM -> global stores
+      const double t_partial = s > 1 ? 1.5 * s * m * (double)n_out * 4.0 / 3400.0 : 0.0;
+      const double t = waves * (kbs * t_kb + t_epi + 600.0) + t_partial;
+      if (t < best_t * 0.999) {
+        best_t = t;
+        best.n_pad = n_pad;
+        best.n_chunks = nch;
+        best.splits = s;
+        best.kb_per_split = kbs;
+      }
+    }
+  }
+  if (best.n_pad == 0) return best;
+  best.n_mma = best.n_pad > 256 ? 2 : 1;
+  best.mma_n = best.n_pad / best.n_mma;
+  best.box_rows = best.n_pad > 256 ? best.n_pad / 2 : best.n_pad;
+  best.n_boxes = best.n_pad / best.box_rows;
+  const size_t stage = kStageA + static_cast<size_t>(best.n_pad) * 128;
+  const size_t extra = 1024 + 256;
+  int stages = static_cast<int>((kMaxSmem - extra) / stage);
+  stages = std::min(stages, 8);
+  stages = std::min(stages, std::max(best.kb_per_split, 2));
+  best.stages = std::max(stages, 2);
+  best.tmem_cols = pow2_at_least(static_cast<uint32_t>(best.n_pad));
+  best.smem_bytes = best.stages * stage + extra;
+  return best;
+}
+
+cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
+                        int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
+                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kMaxSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  GemmParams p;
+  p.m = m;
+  p.n_out = n_out;
+  p.kb_total = k / kTileK;
+  p.kb_per_split = plan.kb_per_split;
+  p.n_pad = plan.n_pad;
+  p.n_mma = plan.n_mma;
+  p.mma_n = plan.mma_n;
+  p.box_rows = plan.box_rows;
+  p.n_boxes = plan.n_boxes;
+  p.stages = plan.stages;
+  p.tmem_cols = plan.tmem_cols;
+  p.epi = epi;
+  p.out = out_f32;
+  p.out_act = out_act;
+  p.split_stride = static_cast<int64_t>(m) * n_out;
+  p.status = status;
+  dim3 grid(n_out / kTileM, plan.n_chunks, plan.splits);
+  gemm_bf16_tcgen05<<<grid, 128, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
+  return cudaGetLastError();
+}
+
+}  // namespace isd

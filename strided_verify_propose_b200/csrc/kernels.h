@@ -1,0 +1,121 @@
+// Host-side launchers of the ISD kernels (internal to libisd.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace isd {
+
+// --------------------------------------------------------------- tensor maps
+// 2-D bf16 tensor map over a row-major [rows][cols] matrix, box
+// {64 columns (128 B), box_rows}, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows, std::string* err);
+
+// ---------------------------------------------------------------------- GEMM
+enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
+
+struct GemmPlan {
+  int32_t n_pad = 0, n_mma = 0, mma_n = 0, box_rows = 0, n_boxes = 0;
+  int32_t n_chunks = 0, splits = 0, kb_per_split = 0, stages = 0;
+  uint32_t tmem_cols = 0;
+  size_t smem_bytes = 0;
+};
+
+// Tile plan for Y[m][n_out] = X[m][k] W[n_out][k]^T. force_splits > 0 pins
+// the split-K factor; max_splits bounds the automatic choice.
+GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, int32_t max_splits,
+                   int32_t num_sms);
+
+// tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
+// kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
+// with W's rows interleaved in blocks of 64 (gate rows then up rows).
+cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
+                        int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
+                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream);
+
+// ----------------------------------------------------------------- attention
+struct AttnShape {
+  int32_t batch, rows_per_req, n_q_heads, n_kv_heads, head_dim, page_size, num_pages,
+      max_pages_per_req, n_layers;
+};
+size_t attention_workspace_bytes(const AttnShape& s);
+// k_map / v_map: tensor maps over the pools as [n_layers*num_pages*n_kv*page_size][head_dim]
+// with box_rows = page_size.
+cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map, const AttnShape& s,
+                             int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,
+                             const int32_t* page_table, __nv_bfloat16* out, void* workspace,
+                             int32_t* status, cudaStream_t stream, int* launches,
+                             cudaEvent_t between = nullptr);
+
+// ------------------------------------------------------------------ row ops
+struct RowMeta {
+  int32_t* tok;     // [rows] input token
+  int32_t* pos;     // [rows] absolute position (-1: none)
+  int32_t* flags;   // [rows] bit0: write KV, bit1: MASK row (gated LoRA)
+};
+constexpr int32_t kRowWriteKV = 1;
+constexpr int32_t kRowMask = 2;
+
+cudaError_t launch_assemble_step(const int32_t* pending, const int32_t* n_draft,
+                                 const int32_t* seq_len, int32_t batch, int32_t stride_n,
+                                 int32_t mask_token, RowMeta meta, int32_t* status,
+                                 cudaStream_t stream);
+cudaError_t launch_assemble_prefill(const int32_t* tokens, int32_t max_len, const int32_t* lens,
+                                    int32_t batch, int32_t chunk, int32_t start, RowMeta meta,
+                                    cudaStream_t stream);
+cudaError_t launch_embed_norm(const __nv_bfloat16* embed, const float* norm_w, RowMeta meta,
+                              int32_t rows, int32_t hidden, int32_t vocab, float eps, float* x,
+                              __nv_bfloat16* hn, int32_t* status, cudaStream_t stream);
+
+struct QkvReduceArgs {
+  const float* part;        // [splits][rows][qkv_dim]
+  int32_t splits, rows, rows_per_req;
+  int32_t n_q, n_kv, head_dim;
+  const float* q_norm;      // [head_dim]
+  const float* k_norm;
+  float eps;
+  const float2* rope;       // [max_position][head_dim/2] (cos, sin)
+  int32_t max_position;
+  RowMeta meta;
+  const int32_t* page_table;
+  int32_t max_pages_per_req, page_size, num_pages, layer;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
+  __nv_bfloat16* q_out;     // [rows][n_q][head_dim]
+  int32_t* status;
+};
+cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream);
+
+// x[row] += sum_s part[s][row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w).
+cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
+                                 const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
+                                 cudaStream_t stream);
+
+// ---------------------------------------------------------- accept / propose
+struct AcceptArgs {
+  const float* logits;      // [B*R][V]
+  int32_t batch, stride_n, vocab, flags, page_size;
+  int32_t* pending;         // [B][N]
+  int32_t* n_draft;         // [B]
+  int32_t* seq_len;         // [B]
+  float* q_cache;           // [B][N-1][V] or null
+  const float* uniforms;    // [B][R]
+  int32_t* accepted;        // [B]
+  int32_t* committed;       // [B][N] or null
+  int32_t* page_table;      // [B][max_pages]
+  const int32_t* free_list;
+  int32_t* free_head;
+  int32_t num_pages, max_pages_per_req, free_count;
+  int32_t* status;
+};
+size_t accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab);
+// between[0] / between[1]: optional events recorded after the first and second kernel.
+cudaError_t launch_accept(const AcceptArgs& a, void* workspace, cudaStream_t stream, int* launches,
+                          cudaEvent_t between0 = nullptr, cudaEvent_t between1 = nullptr);
+
+}  // namespace isd

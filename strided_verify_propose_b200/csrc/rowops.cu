@@ -1,0 +1,267 @@
+// Row-wise kernels of the ISD forward (sm_100a): block assembly, embedding
+// + RMSNorm, the split-K reduction of the QKV projection fused with QK-norm,
+// rotary embedding and the KV page write, and residual add + RMSNorm.
+//
+// One CTA per block row; every row is computed independently of the others
+// (rows only meet inside causal attention), which keeps verify rows bitwise
+// independent of what happens on MASK rows.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace isd {
+
+namespace {
+
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (threadIdx.x < 32) {
+    t = threadIdx.x < NT / 32 ? red[threadIdx.x] : 0.f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  t = red[0];
+  __syncthreads();
+  return t;
+}
+
+// Block layout of one ISD step: rows [x*, d_1..d_n, MASK...] at positions
+// L..L+2N-2 (Bud's Wiki, Method: verify the previous drafts and propose at
+// MASK positions in the same forward).
+__global__ void assemble_step_kernel(const int32_t* pending, const int32_t* n_draft,
+                                     const int32_t* seq_len, int32_t stride_n, int32_t mask_token,
+                                     RowMeta meta, int32_t* status) {
+  const int b = blockIdx.x, r = threadIdx.x;
+  const int R = 2 * stride_n - 1;
+  if (r >= R) return;
+  int n = n_draft[b];
+  const int L = seq_len[b];
+  if (n != 0 && n != stride_n - 1) {
+    if (r == 0) flag(status, ISD_DEV_BAD_STATE);
+    n = 0;
+  }
+  if (L < 0 && r == 0) flag(status, ISD_DEV_BAD_STATE);
+  const int row = b * R + r;
+  int tok = mask_token;
+  if (r == 0) tok = pending[b * stride_n];
+  else if (r <= n) tok = pending[b * stride_n + r];
+  meta.tok[row] = tok;
+  meta.pos[row] = L < 0 ? -1 : L + r;
+  meta.flags[row] = (L < 0 ? 0 : kRowWriteKV) | (r > n ? kRowMask : 0);
+}
+
+// Prefill chunk: rows [start, start+chunk) of every prompt; positions past
+// len-2 are padding rows that see the prompt's keys but write nothing.
+__global__ void assemble_prefill_kernel(const int32_t* tokens, int32_t max_len, const int32_t* lens,
+                                        int32_t chunk, int32_t start, RowMeta meta) {
+  const int b = blockIdx.x, r = threadIdx.x;
+  if (r >= chunk) return;
+  const int row = b * chunk + r;
+  const int len = lens[b];
+  const int q = start + r;
+  if (q < len - 1) {
+    meta.tok[row] = tokens[static_cast<int64_t>(b) * max_len + q];
+    meta.pos[row] = q;
+    meta.flags[row] = kRowWriteKV;
+  } else {
+    meta.tok[row] = tokens[static_cast<int64_t>(b) * max_len];
+    meta.pos[row] = len >= 2 ? min(start, len - 2) : -1;
+    meta.flags[row] = 0;
+  }
+}
+
+// x = embed[tok] (fp32 residual stream); hn = bf16(RMSNorm(x) * w).
+__global__ void __launch_bounds__(256)
+    embed_norm_kernel(const __nv_bfloat16* embed, const float* norm_w, RowMeta meta, int32_t hidden,
+                      int32_t vocab, float eps, float* x, __nv_bfloat16* hn, int32_t* status) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  int tok = meta.tok[row];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) flag(status, ISD_DEV_BAD_TOKEN);
+    tok = 0;
+  }
+  const __nv_bfloat16* e = embed + static_cast<int64_t>(tok) * hidden;
+  float* xr = x + static_cast<int64_t>(row) * hidden;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 8; i < hidden; i += 256 * 8) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(e + i);
+    const __nv_bfloat16* h8 = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float v = __bfloat162float(h8[k]);
+      xr[i + k] = v;
+      ss += v * v;
+    }
+  }
+  const float tot = block_sum<256>(ss, red);
+  const float rstd = rsqrtf(tot / hidden + eps);
+  __nv_bfloat16* hr = hn + static_cast<int64_t>(row) * hidden;
+  for (int i = threadIdx.x * 8; i < hidden; i += 256 * 8) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(e + i);
+    const __nv_bfloat16* h8 = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    __align__(16) __nv_bfloat16 o8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o8[k] = __float2bfloat16_rn(__bfloat162float(h8[k]) * rstd * norm_w[i + k]);
+    *reinterpret_cast<uint4*>(hr + i) = *reinterpret_cast<const uint4*>(o8);
+  }
+}
+
+// x[row] += sum_s part[s][row] (fixed order); hn[row] = bf16(RMSNorm(x[row]) * w).
+__global__ void __launch_bounds__(256)
+    residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
+                         const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  float* xr = x + static_cast<int64_t>(row) * hidden;
+  const float* pr = part + static_cast<int64_t>(row) * hidden;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < hidden; i += 256 * 4) {
+    float4 v = *reinterpret_cast<const float4*>(xr + i);
+    for (int s = 0; s < splits; ++s) {
+      const float4 d = *reinterpret_cast<const float4*>(pr + s * split_stride + i);
+      v.x += d.x;
+      v.y += d.y;
+      v.z += d.z;
+      v.w += d.w;
+    }
+    *reinterpret_cast<float4*>(xr + i) = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  const float tot = block_sum<256>(ss, red);
+  const float rstd = rsqrtf(tot / hidden + eps);
+  __nv_bfloat16* hr = hn + static_cast<int64_t>(row) * hidden;
+  for (int i = threadIdx.x * 4; i < hidden; i += 256 * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + i);
+    __align__(8) __nv_bfloat16 o4[4] = {
+        __float2bfloat16_rn(v.x * rstd * norm_w[i]), __float2bfloat16_rn(v.y * rstd * norm_w[i + 1]),
+        __float2bfloat16_rn(v.z * rstd * norm_w[i + 2]),
+        __float2bfloat16_rn(v.w * rstd * norm_w[i + 3])};
+    *reinterpret_cast<uint2*>(hr + i) = *reinterpret_cast<const uint2*>(o4);
+  }
+}
+
+// QKV split-K reduction, then per head: RMSNorm over head_dim for q and k,
+// NeoX rotary embedding (pairs (i, i + d/2)) at the row's absolute position,
+// q to the attention input, k and v into the row's page slot.
+template <int HD>
+__global__ void __launch_bounds__(128) qkv_reduce_kernel(const QkvReduceArgs a) {
+  constexpr int J = HD / 32;       // values per lane
+  constexpr int JH = J / 2;        // partner offset (d + HD/2)
+  const int row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qkv_dim = (a.n_q + 2 * a.n_kv) * HD;
+  const int64_t split_stride = static_cast<int64_t>(a.rows) * qkv_dim;
+  const float* pr = a.part + static_cast<int64_t>(row) * qkv_dim;
+  const int flags = a.meta.flags[row];
+  int pos = a.meta.pos[row];
+  const bool write_kv = (flags & kRowWriteKV) && pos >= 0;
+  if (pos >= a.max_position) {
+    if (threadIdx.x == 0) flag(a.status, ISD_DEV_BAD_STATE);
+    pos = a.max_position - 1;
+  }
+  const int rpos = pos < 0 ? 0 : pos;
+  int64_t slot_base = -1;
+  if (write_kv) {
+    const int b = row / a.rows_per_req;
+    const int pidx = pos / a.page_size;
+    const int page = pidx < a.max_pages_per_req
+                         ? a.page_table[static_cast<int64_t>(b) * a.max_pages_per_req + pidx]
+                         : -1;
+    if (page < 0 || page >= a.num_pages) {
+      if (threadIdx.x == 0) flag(a.status, ISD_DEV_BAD_PAGE);
+    } else {
+      slot_base = (static_cast<int64_t>(a.layer) * a.num_pages + page) * a.n_kv;  // * P + slot below
+    }
+  }
+  const int n_heads = a.n_q + 2 * a.n_kv;
+  for (int hd = warp; hd < n_heads; hd += 4) {
+    float v[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int d = lane + 32 * j;
+      float s = 0.f;
+      for (int sp = 0; sp < a.splits; ++sp) s += pr[sp * split_stride + hd * HD + d];
+      v[j] = s;
+    }
+    if (hd < a.n_q + a.n_kv) {
+      const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < J; ++j) ss += v[j] * v[j];
+      ss = warp_sum(ss);
+      const float rstd = rsqrtf(ss / HD + a.eps);
+#pragma unroll
+      for (int j = 0; j < J; ++j) v[j] *= rstd * nw[lane + 32 * j];
+      const float2* cs = a.rope + static_cast<int64_t>(rpos) * (HD / 2);
+#pragma unroll
+      for (int j = 0; j < JH; ++j) {
+        const float2 c = cs[lane + 32 * j];
+        const float x1 = v[j], x2 = v[j + JH];
+        v[j] = x1 * c.x - x2 * c.y;
+        v[j + JH] = x2 * c.x + x1 * c.y;
+      }
+    }
+    if (hd < a.n_q) {
+      __nv_bfloat16* qo = a.q_out + (static_cast<int64_t>(row) * a.n_q + hd) * HD;
+#pragma unroll
+      for (int j = 0; j < J; ++j) qo[lane + 32 * j] = __float2bfloat16_rn(v[j]);
+    } else if (slot_base >= 0) {
+      const bool is_k = hd < a.n_q + a.n_kv;
+      const int g = is_k ? hd - a.n_q : hd - a.n_q - a.n_kv;
+      __nv_bfloat16* dst = (is_k ? a.k_pool : a.v_pool) +
+                           (((slot_base + g) * a.page_size) + pos % a.page_size) * HD;
+#pragma unroll
+      for (int j = 0; j < J; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_assemble_step(const int32_t* pending, const int32_t* n_draft,
+                                 const int32_t* seq_len, int32_t batch, int32_t stride_n,
+                                 int32_t mask_token, RowMeta meta, int32_t* status,
+                                 cudaStream_t stream) {
+  assemble_step_kernel<<<batch, 32, 0, stream>>>(pending, n_draft, seq_len, stride_n, mask_token,
+                                                 meta, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assemble_prefill(const int32_t* tokens, int32_t max_len, const int32_t* lens,
+                                    int32_t batch, int32_t chunk, int32_t start, RowMeta meta,
+                                    cudaStream_t stream) {
+  assemble_prefill_kernel<<<batch, 64, 0, stream>>>(tokens, max_len, lens, chunk, start, meta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed_norm(const __nv_bfloat16* embed, const float* norm_w, RowMeta meta,
+                              int32_t rows, int32_t hidden, int32_t vocab, float eps, float* x,
+                              __nv_bfloat16* hn, int32_t* status, cudaStream_t stream) {
+  embed_norm_kernel<<<rows, 256, 0, stream>>>(embed, norm_w, meta, hidden, vocab, eps, x, hn,
+                                              status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream) {
+  if (a.head_dim == 128)
+    qkv_reduce_kernel<128><<<a.rows, 128, 0, stream>>>(a);
+  else
+    qkv_reduce_kernel<64><<<a.rows, 128, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
+                                 const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
+                                 cudaStream_t stream) {
+  residual_norm_kernel<<<rows, 256, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
+                                                 hidden, norm_w, eps, x, hn);
+  return cudaGetLastError();
+}
+
+}  // namespace isd
