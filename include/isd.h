@@ -228,6 +228,25 @@ int isd_accept_propose(const float *logits_dev, const isd_batch *batch, const is
                        void *workspace_dev, size_t workspace_bytes, int32_t *status_dev,
                        void *stream);
 
+/* The same verify / resample / propose and bookkeeping as
+ * isd_accept_propose, for callers that cannot allocate device memory (a host
+ * program that hands out all GPU memory from its own fixed pool, a serving
+ * loop that must never enter the allocator, a plugin with no allocator of
+ * its own). The paper has no counterpart: this is a deployment variant.
+ * Scratch comes from a 4 MiB array compiled into the library, present on
+ * every GPU that loads it until the process exits; a call needs
+ * batch * (2N-1) * ceil(vocab/8192) * 16 bytes of it (at most 4 MiB, e.g.
+ * batch <= 1024 at N = 4 and vocab 151936) and returns ISD_E_UNSUPPORTED
+ * above that. The first call on each device looks up the array's device
+ * address with that device current; make that first call before any
+ * stream capture. All calls share the array: calls that overlap on the GPU
+ * race and must be serialised by the caller. No scratch needs clearing. */
+int isd_accept_propose_noalloc(const float *logits_dev, const isd_batch *batch, const isd_kv *kv,
+                               int32_t page_size, int32_t vocab, int32_t *pending_dev,
+                               float *q_cache_dev, const float *uniforms_dev,
+                               int32_t *out_accepted_dev, int32_t *out_committed_dev,
+                               int32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

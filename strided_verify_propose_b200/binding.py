@@ -32,7 +32,8 @@ USE_LORA = 0x4
 EXPORTS = ("isd_init", "isd_load_gated_lora", "isd_step", "isd_prefill", "isd_last_launch_count",
            "isd_last_error", "isd_destroy", "isd_gemm_bf16", "isd_attention_workspace_bytes",
            "isd_paged_attention", "isd_accept_workspace_bytes", "isd_accept_propose",
-           "isd_profile_enable", "isd_profile_read", "isd_profile_class_name")
+           "isd_profile_enable", "isd_profile_read", "isd_profile_class_name",
+           "isd_accept_propose_noalloc")
 PROF_CLASSES = 16
 
 
@@ -97,6 +98,8 @@ def lib():
     L.isd_accept_workspace_bytes.restype = sz
     L.isd_accept_propose.argtypes = [vp, C.POINTER(Batch), C.POINTER(KV), i32, i32, vp, vp, vp,
                                      vp, vp, vp, sz, vp, vp]
+    L.isd_accept_propose_noalloc.argtypes = [vp, C.POINTER(Batch), C.POINTER(KV), i32, i32, vp,
+                                             vp, vp, vp, vp, vp, vp]
     L.isd_profile_enable.argtypes = [vp, C.c_int]
     L.isd_profile_read.argtypes = [vp, C.POINTER(C.c_double), C.POINTER(i32)]
     L.isd_profile_class_name.argtypes = [C.c_int]
@@ -342,3 +345,15 @@ def accept_propose(logits, st: StepState, kv: KVCache, page_size: int, uniforms,
                                    _ptr(st.pending), _ptr(st.q_cache), _ptr(uniforms),
                                    _ptr(st.accepted), _ptr(st.committed), _ptr(ws), ws_bytes,
                                    _ptr(st.status), _stream()))
+
+
+def accept_propose_noalloc(logits, st: StepState, kv: KVCache, page_size: int, uniforms,
+                           flags: int = 0):
+    """accept_propose without any device allocation: the library's fixed
+    scratch array stands in for the workspace (for callers that cannot
+    allocate device memory)."""
+    b = Batch(st.B, st.N, flags, _ptr(st.seq_len), _ptr(st.n_draft), None)
+    check(lib().isd_accept_propose_noalloc(_ptr(logits), C.byref(b), C.byref(kv.c()), page_size,
+                                           logits.shape[1], _ptr(st.pending), _ptr(st.q_cache),
+                                           _ptr(uniforms), _ptr(st.accepted), _ptr(st.committed),
+                                           _ptr(st.status), _stream()))

@@ -63,6 +63,10 @@ int num_sms() {
 
 namespace isd {
 
+// Lets other translation units of the library report an error through
+// isd_last_error().
+int set_error(int code, const char* msg) { return fail(code, msg); }
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows, std::string* err) {
   if (!load_encode(err)) return false;

@@ -10,6 +10,9 @@
 
 namespace isd {
 
+// Record msg as the calling thread's last error (see isd_last_error); returns code.
+int set_error(int code, const char* msg);
+
 // --------------------------------------------------------------- tensor maps
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix, box
 // {64 columns (128 B), box_rows}, 128-byte swizzle, zero fill out of bounds.
