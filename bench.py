@@ -194,12 +194,14 @@ def run_cuda(args, ws, rank, local):
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        torch.cuda.nvtx.range_push("isd_timed")
         e_start.record(stream)
         for i in range(args.steps):
             one(unif_d[step_i]); step_i += 1
             hist[i].copy_(st.accepted)
         e_stop.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     barrier()
     ms = e_start.elapsed_time(e_stop)
     launches_per_step = model.launches()

@@ -64,6 +64,16 @@ def _weights(z, q_row, excluded):
     return p
 
 
+def draw_is_valid(w, u, token, eps_rel):
+    """token is a legal inverse-CDF draw of weights w at u, up to eps_rel * sum(w)."""
+    w = np.asarray(w, dtype=np.float64)
+    c = np.cumsum(w)
+    t = u * c[-1]
+    eps = eps_rel * c[-1]
+    lo = c[token - 1] if token > 0 else 0.0
+    return w[token] > 0 and lo - eps <= t < c[token] + eps
+
+
 def _argmax(z):
     z = np.asarray(z)
     return int(np.flatnonzero(z == z.max())[0])
@@ -71,7 +81,8 @@ def _argmax(z):
 
 class Outcome:
     def __init__(self):
-        self.clear = True        # every decision clear of the error band
+        self.clear = True          # every decision clear of the error band
+        self.accept_clear = True   # the accept tests were (A compared exactly)
         self.notes = []
 
     def near(self, what):
@@ -116,6 +127,7 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
         if not ok_o:
             break
     if not out.clear:
+        out.accept_clear = False
         return out
     assert gpu_A == dec.accepted, f"accepted {gpu_A} vs oracle {dec.accepted}"
     A = dec.accepted
@@ -136,6 +148,8 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
         assert t_o == dec.new_token
         if m_g >= FP32_REL:
             assert gpu_new == t_g, f"new token {gpu_new} is not the kernel logits' draw {t_g}"
+        else:
+            assert draw_is_valid(w_g, u[N - 1], gpu_new, FP32_REL), "new token outside the band"
         if t_o == t_g and m_g >= FP32_REL:
             assert gpu_new == dec.new_token
         else:
@@ -156,6 +170,8 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
                 t_g, m_g = _cdf_draw(_softmax(lg[r]), u[N + i - 1])
                 if m_g >= FP32_REL:
                     assert gpu_props[i - 1] == t_g
+                else:
+                    assert draw_is_valid(_softmax(lg[r]), u[N + i - 1], gpu_props[i - 1], FP32_REL)
                 if t_o == t_g and m_g >= FP32_REL:
                     assert gpu_props[i - 1] == dec.proposals[i - 1]
                 else:

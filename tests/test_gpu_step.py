@@ -146,6 +146,10 @@ def test_tiny_batch(N, propose, verify):
 
 def test_qwen3_8b_widths_two_layers():
     """Full Qwen3-8B widths (hidden 4096, 32/8 heads x 128, intermediate
-    12288, vocab 151936, page 64) with two layers, batch 3, stride 4."""
-    run_pair(synth.QWEN3_8B_2L, 3, 4, 3, oi.ARGMAX, oi.STOCHASTIC, seed=1, len_lo=20, len_hi=90,
-             min_exact=0.3)
+    12288, vocab 151936, page 64) with two layers, batch 3, stride 4, greedy
+    verification and argmax proposals: every decision is an argmax, so the
+    comparison is exact wherever the top-2 gap exceeds the logit error
+    (draws over 152k-token flat distributions would always sit inside the
+    fp32 rounding band of a CDF boundary)."""
+    run_pair(synth.QWEN3_8B_2L, 3, 4, 4, oi.ARGMAX, oi.GREEDY, seed=1, len_lo=20, len_hi=90,
+             min_exact=0.5)
