@@ -46,6 +46,9 @@ WORKLOADS = {
     # Qwen3-8B shape, batch 1, stride 4, prompt 2048
     "qwen3_8b_b1": dict(shape=synth.QWEN3_8B, batch=1, stride=4, len_lo=2048, len_hi=2048),
     "tiny": dict(shape=synth.TINY, batch=1, stride=2, len_lo=32, len_hi=32),
+    # R-ISD: Qwen3-8B shape + rank-128 gated LoRA on MASK rows, batch 32, N=4, prompts 2048
+    "risd_8b_b32": dict(shape=synth.QWEN3_8B, batch=32, stride=4, len_lo=2048, len_hi=2048,
+                        lora_rank=128),
 }
 ACCEPT_RATE = 0.9
 
@@ -145,7 +148,7 @@ def run_cuda(args, ws, rank, local):
     shape, B, N = wl["shape"], wl["batch"], wl["stride"]
     R, P, V = 2 * N - 1, shape.page_size, shape.vocab
     seed = 1000 + rank
-    total_steps = args.warmup + 3 * args.steps + 4
+    total_steps = args.warmup + 5 * args.steps + 4   # every step run below grows the sequences
     lens = synth.prompt_lengths(B, wl["len_lo"], wl["len_hi"], seed)
     prompts = synth.prompts(shape, lens, seed)
     maxp = -(-(int(lens.max()) + total_steps * N + R + 1) // P) + 1
@@ -158,6 +161,11 @@ def run_cuda(args, ws, rank, local):
     G = shape.n_q_heads // shape.n_kv_heads
     model = Bd.Model(shape, weights, max_batch=B, max_rows=max(B * R, B * (64 // G)),
                      max_position=maxp * P)
+    lora_rank = wl.get("lora_rank", 0)
+    flags = 0
+    if lora_rank:
+        model.load_lora(Bd.random_device_lora(shape, lora_rank, seed=seed, std=0.01), rank=lora_rank)
+        flags = Bd.USE_LORA
     kv = Bd.KVCache(shape, num_pages, table, free)
     st = Bd.StepState(B, N, V, sample=False)
     torch.cuda.synchronize()
@@ -176,8 +184,8 @@ def run_cuda(args, ws, rank, local):
     hist = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
     step_i = 0
 
-    def one(u, flags=0):
-        Bd.step(model, kv, st, u, flags)
+    def one(u, fl=None):
+        Bd.step(model, kv, st, u, flags if fl is None else fl)
 
     for _ in range(args.warmup):
         one(unif_d[step_i]); step_i += 1
@@ -215,6 +223,18 @@ def run_cuda(args, ws, rank, local):
         one(unif_d[step_i]); step_i += 1
     prof = model.profile_read()
     model.profile(False)
+
+    # ---- the same steps without the adapter: R-ISD overhead alpha
+    base_ms = None
+    if lora_rank:
+        torch.cuda.synchronize()
+        b_start, b_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b_start.record(stream)
+        for i in range(args.steps):
+            one(unif_d[step_i % total_steps], 0); step_i += 1
+        b_stop.record(stream)
+        torch.cuda.synchronize()
+        base_ms = b_start.elapsed_time(b_stop)
 
     # ---- natural uniforms (acceptance ~ 0 with random weights)
     torch.cuda.synchronize()
@@ -293,6 +313,7 @@ def run_cuda(args, ws, rank, local):
             "hbm_roofline_fraction_step": hbm_frac_step,
             "hbm_roofline_ceiling_step": ceiling,
             "step_algorithmic_bytes": step_bytes,
+            "risd_overhead_alpha": (ms / base_ms) if base_ms else None,
             "natural_uniforms": {"value": nat_committed / (nat_ms * 1e-3), "unit": "tokens/s",
                                  "tokens_per_forward": nat_committed / (args.steps * B * ws)},
             "prefill_s": t_prefill, "setup_s": t_setup,

@@ -90,8 +90,8 @@ typedef struct {
   /* host arrays of n_layers device pointers each:                                      */
   const void *const *w_qkv;     /* [(nq+2nkv)*head_dim][hidden] bf16: q rows, k rows, v rows */
   const void *const *w_o;       /* [hidden][nq*head_dim] bf16                            */
-  const void *const *w_gate_up; /* [2*intermediate][hidden] bf16; row block t of 128 holds
-                                   gate rows 64t..64t+63 then up rows 64t..64t+63       */
+  const void *const *w_gate_up; /* [2*intermediate][hidden] bf16; row block b of 32 holds
+                                   gate rows 16b..16b+15 then up rows 16b..16b+15       */
   const void *const *w_down;    /* [hidden][intermediate] bf16                           */
   const float *const *attn_norm;/* [hidden] fp32 (pre-attention RMSNorm weight)          */
   const float *const *mlp_norm; /* [hidden] fp32 (pre-MLP RMSNorm weight)                */

@@ -131,7 +131,7 @@ def _ptr_array(ts: Sequence) -> C.Array:
 
 def pack_weights(shape, w: Dict[str, object], device="cuda") -> Dict[str, object]:
     """Device tensors in the ABI layout from per-matrix weights (numpy or torch):
-    fused QKV rows [q | k | v], gate/up interleaved in blocks of 64 rows."""
+    fused QKV rows [q | k | v], gate/up interleaved in blocks of 16 rows."""
     import torch
 
     def bf(a):
@@ -147,8 +147,8 @@ def pack_weights(shape, w: Dict[str, object], device="cuda") -> Dict[str, object
     I = shape.intermediate
     for lw in w["layers"]:
         qkv = torch.cat([bf(lw["wq"]), bf(lw["wk"]), bf(lw["wv"])], 0).contiguous()
-        g = bf(lw["w_gate"]).view(I // 64, 64, shape.hidden)
-        u = bf(lw["w_up"]).view(I // 64, 64, shape.hidden)
+        g = bf(lw["w_gate"]).view(I // 16, 16, shape.hidden)
+        u = bf(lw["w_up"]).view(I // 16, 16, shape.hidden)
         gu = torch.stack([g, u], 1).reshape(2 * I, shape.hidden).contiguous()
         out["layers"].append({"w_qkv": qkv, "w_o": bf(lw["wo"]), "w_gate_up": gu,
                               "w_down": bf(lw["w_down"]), "attn_norm": f32(lw["attn_norm"]),
@@ -179,6 +179,24 @@ def random_device_weights(shape, seed: int = 0, std: float = 0.02, device="cuda"
                               "attn_norm": ones(h), "mlp_norm": ones(h),
                               "q_norm": ones(shape.head_dim), "k_norm": ones(shape.head_dim)})
     return out
+
+
+def random_device_lora(shape, rank: int = 128, seed: int = 0, std: float = 0.01, device="cuda"):
+    """Random gated-LoRA adapters on the device, per layer {target: (A [in, r], B [r, out])}
+    (for throughput runs; the oracle never sees these)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 7919)
+    h, i = shape.hidden, shape.intermediate
+    dims = {"q": (h, shape.q_dim), "k": (h, shape.kv_dim), "v": (h, shape.kv_dim),
+            "o": (shape.q_dim, h), "gate": (h, i), "up": (h, i), "down": (i, h)}
+
+    def rnd(*s):
+        t = torch.empty(*s, device=device, dtype=torch.bfloat16)
+        t.normal_(0.0, std, generator=gen)
+        return t
+    return [{t: (rnd(dims[t][0], rank), rnd(rank, dims[t][1])) for t in dims}
+            for _ in range(shape.n_layers)]
 
 
 class Model:
@@ -219,6 +237,30 @@ class Model:
 
     def launches(self) -> int:
         return int(lib().isd_last_launch_count(self.ctx))
+
+    def load_lora(self, lora_layers, rank: int = 128, scale: float = 1.0, device="cuda"):
+        """Attach a gated LoRA. lora_layers: per layer {target: (A [in, r], B [r, out])}
+        (numpy or torch, as synth.lora_weights returns them); passed to the library
+        as the nn.Linear weights A^T [r][in] and B^T [out][r] in bf16."""
+        import torch
+        targets = ("q", "k", "v", "o", "gate", "up", "down")
+
+        def bf(a):
+            t = a if isinstance(a, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(a))
+            return t.to(device=device, dtype=torch.bfloat16).t().contiguous()
+
+        self._lora = [{t: (bf(ll[t][0]), bf(ll[t][1])) for t in targets} for ll in lora_layers]
+        self._lora_arrays = []
+        lo = Lora()
+        lo.rank = rank
+        lo.scale = scale
+        for i, t in enumerate(targets):
+            a = _ptr_array([ll[t][0] for ll in self._lora])
+            b = _ptr_array([ll[t][1] for ll in self._lora])
+            self._lora_arrays += [a, b]
+            lo.A[i] = C.cast(a, _PP)
+            lo.B[i] = C.cast(b, _PP)
+        check(lib().isd_load_gated_lora(self.ctx, C.byref(lo)))
 
     def profile(self, enable: bool) -> None:
         check(lib().isd_profile_enable(self.ctx, 1 if enable else 0))

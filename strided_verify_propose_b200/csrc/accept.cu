@@ -448,8 +448,12 @@ cudaError_t launch_accept(const AcceptArgs& a, void* workspace, cudaStream_t str
   ChunkStat* stats = static_cast<ChunkStat*>(workspace);
   accept_stats_kernel<<<dim3(n_chunks, a.batch * R), kThreads, 0, stream>>>(a.logits, a.vocab,
                                                                            n_chunks, stats);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;   // each kernel reads what the previous one wrote
   if (between0) cudaEventRecord(between0, stream);
   accept_decide_kernel<<<a.batch, kThreads, 0, stream>>>(a, stats, n_chunks);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   if (between1) cudaEventRecord(between1, stream);
   bookkeep_kernel<<<1, 1024, 0, stream>>>(a);
   if (launches) *launches += 3;

@@ -89,6 +89,28 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return true;
 }
 
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t b0, uint32_t b1, uint32_t b2, std::string* err) {
+  if (!load_encode(err)) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (d0 * 2) % 16 != 0) {
+    if (err) *err = "tensor map base or row pitch not 16-byte aligned";
+    return false;
+  }
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (err) *err = "cuTensorMapEncodeTiled (3-D) failed (" + std::to_string(static_cast<int>(r)) + ")";
+    return false;
+  }
+  return true;
+}
+
 }  // namespace isd
 
 using isd::GemmPlan;
@@ -129,6 +151,21 @@ struct isd_ctx {
   std::map<std::tuple<int, int, int>, GemmPlan> plans;
   int launches = 0;
 
+  // gated LoRA (R-ISD): packed adapters per layer + their workspace
+  bool has_lora = false;
+  int32_t lora_rank = 0;
+  float lora_scale = 1.f;
+  void* lora_mem = nullptr;
+  struct LoraLayer {
+    __nv_bfloat16 *a_qkv, *b_qkv, *a_o, *b_o, *a_gu, *b_gu, *a_d, *b_d;
+    CUtensorMap ta_qkv, tb_qkv, ta_o, tb_o, ta_gu, tb_gu, ta_d, tb_d;
+  };
+  std::vector<LoraLayer> lora;
+  float* lora_xa_part = nullptr;         // [max_splits][max_rows][3r]
+  __nv_bfloat16* lora_xa = nullptr;      // [max_rows][3r]
+  float* lora_delta = nullptr;           // [max_rows][max(qkv_dim, hidden, 2 I)]
+  float* lora_gu = nullptr;              // [max_rows][2 I] base gate/up in fp32
+
   // per-kernel-class event timing (isd_profile_enable)
   bool prof_on = false;
   std::vector<cudaEvent_t> prof_pool;
@@ -146,7 +183,7 @@ enum ProfClass {
 const char* kProfNames[ISD_PROF_CLASSES] = {
     "assemble", "embed_norm", "gemm_qkv", "qkv_reduce_rope_kvwrite", "attention_split",
     "attention_combine", "gemm_o", "residual_norm", "gemm_gate_up_silu", "gemm_down",
-    "gemm_lm_head", "accept_stats", "accept_decide", "bookkeep", "other", "unused"};
+    "gemm_lm_head", "accept_stats", "accept_decide", "bookkeep", "lora_delta", "unused"};
 
 cudaEvent_t prof_event(isd_ctx* c) {
   if (!c->prof_on) return nullptr;
@@ -270,8 +307,27 @@ isd::AttnShape attn_shape(const isd_ctx* c, const isd_kv* kv, int batch, int row
 
 // The decoder layers over the rows described by the row metadata; leaves
 // bf16(final RMSNorm(x)) in c->hn.
+// Gated-LoRA delta of one projection for every row: delta = (x A^T) B^T,
+// with x A^T summed over its K splits in fixed order and cast to bf16.
+// Consumers add scale * delta on MASK rows only.
+int lora_delta(isd_ctx* c, const CUtensorMap& ta, const CUtensorMap& tb, const __nv_bfloat16* x,
+               int M, int in, int n_a, int out, int32_t* status, cudaStream_t st) {
+  int s = 1;
+  int rc = gemm(c, kPOther, ta, x, M, n_a, in, isd::kEpiF32, c->lora_xa_part,
+                static_cast<size_t>(c->max_splits) * c->cfg.max_rows * 3 * c->lora_rank,
+                c->max_splits, nullptr, &s, status, st);
+  if (rc) return rc;
+  cudaEvent_t e0 = prof_mark(c, st);
+  ISD_CUDA(isd::launch_sum_cast(c->lora_xa_part, s, M, n_a, c->lora_xa, st));
+  prof_add(c, kPOther, e0, prof_mark(c, st));
+  c->launches += 1;
+  const size_t wide = std::max(std::max(c->qkv_dim, c->cfg.hidden), 2 * c->cfg.intermediate);
+  return gemm(c, kPOther, tb, c->lora_xa, M, out, n_a, isd::kEpiF32, c->lora_delta,
+              static_cast<size_t>(c->cfg.max_rows) * wide, 1, nullptr, nullptr, status, st);
+}
+
 int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, int32_t* status,
-                   cudaStream_t st) {
+                   cudaStream_t st, bool use_lora = false) {
   const isd_model_cfg& g = c->cfg;
   const int M = batch * rows_per_req;
   const int H = g.hidden;
@@ -299,6 +355,12 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     int rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
                   c->part_elems, c->max_splits, nullptr, &s, status, st);
     if (rc) return rc;
+    const int r = c->lora_rank;
+    const isd_ctx::LoraLayer* ll = use_lora ? &c->lora[l] : nullptr;
+    if (ll) {
+      rc = lora_delta(c, ll->ta_qkv, ll->tb_qkv, c->hn, M, H, 3 * r, c->qkv_dim, status, st);
+      if (rc) return rc;
+    }
     isd::QkvReduceArgs qa;
     qa.part = c->part;
     qa.splits = s;
@@ -321,6 +383,8 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.k_pool = static_cast<__nv_bfloat16*>(kv->k_pool_dev);
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
+    qa.delta = ll ? c->lora_delta : nullptr;
+    qa.delta_scale = c->lora_scale;
     qa.status = status;
     cudaEvent_t a0 = prof_mark(c, st);
     ISD_CUDA(isd::launch_qkv_reduce(qa, st));
@@ -336,19 +400,45 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
               c->max_splits, nullptr, &s, status, st);
     if (rc) return rc;
+    if (ll) {
+      rc = lora_delta(c, ll->ta_o, ll->tb_o, c->attn, M, c->q_dim, r, H, status, st);
+      if (rc) return rc;
+    }
     cudaEvent_t r0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st,
+                                       ll ? c->lora_delta : nullptr, c->lora_scale, c->meta_flags));
     prof_add(c, kPResNorm, r0, prof_mark(c, st));
     c->launches += 1;
-    rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiSiluMul, nullptr,
-              0, 1, c->act, nullptr, status, st);
-    if (rc) return rc;
+    if (!ll) {
+      rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiSiluMul,
+                nullptr, 0, 1, c->act, nullptr, status, st);
+      if (rc) return rc;
+    } else {
+      // base gate/up in fp32 (one split, the same sums the fused epilogue sees),
+      // the delta, then SwiGLU with the delta on MASK rows only
+      rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiF32,
+                c->lora_gu, static_cast<size_t>(g.max_rows) * 2 * g.intermediate, 1, nullptr,
+                nullptr, status, st);
+      if (rc) return rc;
+      rc = lora_delta(c, ll->ta_gu, ll->tb_gu, c->hn, M, H, 2 * r, 2 * g.intermediate, status, st);
+      if (rc) return rc;
+      cudaEvent_t s0 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_lora_silu(c->lora_gu, c->lora_delta, c->lora_scale, c->meta_flags, M,
+                                     g.intermediate, c->act, st));
+      prof_add(c, kPOther, s0, prof_mark(c, st));
+      c->launches += 1;
+    }
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
               c->part_elems, c->max_splits, nullptr, &s, status, st);
     if (rc) return rc;
+    if (ll) {
+      rc = lora_delta(c, ll->ta_d, ll->tb_d, c->act, M, g.intermediate, r, H, status, st);
+      if (rc) return rc;
+    }
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
     cudaEvent_t r1 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st,
+                                       ll ? c->lora_delta : nullptr, c->lora_scale, c->meta_flags));
     prof_add(c, kPResNorm, r1, prof_mark(c, st));
     c->launches += 1;
   }
@@ -501,13 +591,112 @@ int isd_init(const isd_model_cfg* cfg, const isd_weights* w, isd_ctx** out) {
 void isd_destroy(isd_ctx* ctx) {
   if (!ctx) return;
   for (cudaEvent_t e : ctx->prof_pool) cudaEventDestroy(e);
+  if (ctx->lora_mem) cudaFree(ctx->lora_mem);
   if (ctx->ws) cudaFree(ctx->ws);
   delete ctx;
 }
 
 int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
   if (!ctx || !lora) return fail(ISD_E_INVALID, "ctx and lora are required");
-  return fail(ISD_E_UNSUPPORTED, "gated LoRA is not implemented in this build");
+  const isd_model_cfg& g = ctx->cfg;
+  const int r = lora->rank, L = g.n_layers;
+  if (r != 128 && r != 256) return fail(ISD_E_UNSUPPORTED, "gated LoRA rank must be 128 or 256");
+  if (L < 1) return fail(ISD_E_INVALID, "the model has no layers");
+  for (int t = 0; t < 7; ++t) {
+    if (!lora->A[t] || !lora->B[t]) return fail(ISD_E_INVALID, "missing LoRA pointer array");
+    for (int l = 0; l < L; ++l)
+      if (!lora->A[t][l] || !lora->B[t][l]) return fail(ISD_E_INVALID, "missing LoRA weight");
+  }
+  const int H = g.hidden, I = g.intermediate, Q = ctx->q_dim, KV = g.n_kv_heads * g.head_dim;
+  // packed per layer: A_qkv [3r][H], B_qkv [qkv][3r] (block diagonal), A_o [r][Q], B_o [H][r],
+  // A_gu [2r][H], B_gu [2I][2r] (block diagonal, 16-row gate/up interleave), A_d [r][I], B_d [H][r]
+  const size_t e_aqkv = 3ull * r * H, e_bqkv = 3ull * r * ctx->qkv_dim, e_ao = 1ull * r * Q,
+               e_bo = 1ull * H * r, e_agu = 2ull * r * H, e_bgu = 2ull * I * 2 * r, e_ad = 1ull * r * I,
+               e_bd = 1ull * H * r;
+  const size_t per_layer = e_aqkv + e_bqkv + e_ao + e_bo + e_agu + e_bgu + e_ad + e_bd;
+  const size_t R = g.max_rows;
+  const size_t wide = std::max(std::max<size_t>(ctx->qkv_dim, H), static_cast<size_t>(2) * I);
+  const size_t ws_bytes = ctx->max_splits * R * 3 * r * 4 + R * 3 * r * 2 + R * wide * 4 + R * 2 * I * 4;
+  if (ctx->lora_mem) {
+    cudaFree(ctx->lora_mem);
+    ctx->lora_mem = nullptr;
+    ctx->has_lora = false;
+  }
+  char* mem = nullptr;
+  const size_t w_bytes = per_layer * L * 2;
+  if (cudaMalloc(&mem, w_bytes + ws_bytes + 4096) != cudaSuccess)
+    return fail(ISD_E_NOMEM, "gated LoRA allocation failed");
+  ctx->lora_mem = mem;
+  ISD_CUDA(cudaMemset(mem, 0, w_bytes));   // block-diagonal zeros
+  cudaStream_t st;
+  ISD_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  ctx->lora.assign(L, isd_ctx::LoraLayer{});
+  auto bf = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
+  std::string err;
+  __nv_bfloat16* cur = reinterpret_cast<__nv_bfloat16*>(mem);
+  int rc = ISD_OK;
+  for (int l = 0; l < L && rc == ISD_OK; ++l) {
+    isd_ctx::LoraLayer& x = ctx->lora[l];
+    x.a_qkv = cur; cur += e_aqkv;
+    x.b_qkv = cur; cur += e_bqkv;
+    x.a_o = cur; cur += e_ao;
+    x.b_o = cur; cur += e_bo;
+    x.a_gu = cur; cur += e_agu;
+    x.b_gu = cur; cur += e_bgu;
+    x.a_d = cur; cur += e_ad;
+    x.b_d = cur; cur += e_bd;
+    // targets: 0 q, 1 k, 2 v, 3 o, 4 gate, 5 up, 6 down
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t v) { if (e == cudaSuccess) e = v; };
+    chk(isd::launch_pack_rows(bf(lora->A[0][l]), r, H, x.a_qkv, H, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->A[1][l]), r, H, x.a_qkv, H, r, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->A[2][l]), r, H, x.a_qkv, H, 2 * r, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[0][l]), Q, r, x.b_qkv, 3 * r, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[1][l]), KV, r, x.b_qkv, 3 * r, Q, r, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[2][l]), KV, r, x.b_qkv, 3 * r, Q + KV, 2 * r, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->A[3][l]), r, Q, x.a_o, Q, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[3][l]), H, r, x.b_o, r, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->A[4][l]), r, H, x.a_gu, H, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->A[5][l]), r, H, x.a_gu, H, r, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[4][l]), I, r, x.b_gu, 2 * r, 0, 0, 0, st));
+    chk(isd::launch_pack_rows(bf(lora->B[5][l]), I, r, x.b_gu, 2 * r, 0, r, 16, st));
+    chk(isd::launch_pack_rows(bf(lora->A[6][l]), r, I, x.a_d, I, 0, 0, -1, st));
+    chk(isd::launch_pack_rows(bf(lora->B[6][l]), H, r, x.b_d, r, 0, 0, -1, st));
+    if (e != cudaSuccess) {
+      rc = fail(ISD_E_CUDA, std::string("LoRA packing: ") + cudaGetErrorString(e));
+      break;
+    }
+    if (!isd::make_tmap_bf16(&x.ta_qkv, x.a_qkv, 3 * r, H, 128, &err) ||
+        !isd::make_tmap_bf16(&x.tb_qkv, x.b_qkv, ctx->qkv_dim, 3 * r, 128, &err) ||
+        !isd::make_tmap_bf16(&x.ta_o, x.a_o, r, Q, 128, &err) ||
+        !isd::make_tmap_bf16(&x.tb_o, x.b_o, H, r, 128, &err) ||
+        !isd::make_tmap_bf16(&x.ta_gu, x.a_gu, 2 * r, H, 128, &err) ||
+        !isd::make_tmap_bf16(&x.tb_gu, x.b_gu, 2 * I, 2 * r, 128, &err) ||
+        !isd::make_tmap_bf16(&x.ta_d, x.a_d, r, I, 128, &err) ||
+        !isd::make_tmap_bf16(&x.tb_d, x.b_d, H, r, 128, &err))
+      rc = fail(ISD_E_INVALID, "LoRA tensor map: " + err);
+  }
+  const cudaError_t se = cudaStreamSynchronize(st);
+  cudaStreamDestroy(st);
+  if (rc == ISD_OK && se != cudaSuccess) rc = fail(ISD_E_CUDA, cudaGetErrorString(se));
+  if (rc != ISD_OK) {
+    cudaFree(ctx->lora_mem);
+    ctx->lora_mem = nullptr;
+    ctx->lora.clear();
+    return rc;
+  }
+  char* w = mem + ((w_bytes + 1023) & ~static_cast<size_t>(1023));
+  ctx->lora_xa_part = reinterpret_cast<float*>(w);
+  w += ctx->max_splits * R * 3 * r * 4;
+  ctx->lora_xa = reinterpret_cast<__nv_bfloat16*>(w);
+  w += ((R * 3 * r * 2 + 255) / 256) * 256;
+  ctx->lora_delta = reinterpret_cast<float*>(w);
+  w += R * wide * 4;
+  ctx->lora_gu = reinterpret_cast<float*>(w);
+  ctx->lora_rank = r;
+  ctx->lora_scale = lora->scale;
+  ctx->has_lora = true;
+  return ISD_OK;
 }
 
 int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pending_dev,
@@ -524,7 +713,8 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
     return fail(ISD_E_INVALID, "seq_len and n_draft are required");
   if (batch->flags & ~(ISD_PROPOSE_SAMPLE | ISD_VERIFY_GREEDY | ISD_USE_LORA))
     return fail(ISD_E_INVALID, "unknown flag bits");
-  if (batch->flags & ISD_USE_LORA) return fail(ISD_E_UNSUPPORTED, "no gated LoRA loaded");
+  const bool use_lora = (batch->flags & ISD_USE_LORA) != 0;
+  if (use_lora && !ctx->has_lora) return fail(ISD_E_INVALID, "ISD_USE_LORA without a loaded gated LoRA");
   if ((batch->flags & ISD_PROPOSE_SAMPLE) && N > 1 && !q_cache_dev)
     return fail(ISD_E_INVALID, "SAMPLE proposals need q_cache");
   const int R = 2 * N - 1;
@@ -542,7 +732,7 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
                                      g.mask_token_id, meta, status_dev, st));
   prof_add(ctx, kPAssemble, e0, prof_mark(ctx, st));
   ctx->launches += 1;
-  rc = forward_layers(ctx, kv, B, R, status_dev, st);
+  rc = forward_layers(ctx, kv, B, R, status_dev, st, use_lora);
   if (rc) return rc;
   const int M = B * R;
   float* logits = batch->logits_out_dev ? batch->logits_out_dev : ctx->logits;

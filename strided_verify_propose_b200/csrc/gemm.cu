@@ -153,31 +153,28 @@ __global__ void __launch_bounds__(128, 1)
             outp[static_cast<int64_t>(t0 + j) * p.n_out] = v[j];
       }
     } else {
-      // rows 0..63 of the tile are gate features, rows 64..127 the matching up features
-      float* xch = reinterpret_cast<float*>(smem);  // stage 0 is free now: [64][33]
+      // Each warp's 32 TMEM lanes hold 16 gate rows then the 16 up rows of
+      // the same features (see the gate/up layout in isd.h). A lane pairs
+      // with lane ^ 16: low lanes finish even tokens, high lanes odd ones.
       const int half_n = p.n_out / 2;
-      const int fo = mt * 64 + (warp & 1) * 32 + lane;
+      const bool hi = lane >= 16;
+      const int f = mt * 64 + warp * 16 + (lane & 15);
       for (int c = 0; c < nchunk; ++c) {
         float v[32];
         tmem_ld_32x32(lane_addr + c * 32, v);
-        if (warp >= 2) {
+        const int t0 = tok0 + c * 32;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) xch[((warp - 2) * 32 + lane) * 33 + j] = v[j];
-        }
-        __syncthreads();
-        if (warp < 2) {
-          const int t0 = tok0 + c * 32;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (c * 32 + j < p.n_pad && t0 + j < p.m) {
-              const float g = v[j];
-              const float u = xch[(warp * 32 + lane) * 33 + j];
-              const float a = g / (1.0f + expf(-g)) * u;
-              p.out_act[static_cast<int64_t>(t0 + j) * half_n + fo] = __float2bfloat16_rn(a);
-            }
+        for (int j = 0; j < 32; j += 2) {
+          const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
+          const float x_j1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 16);
+          const float g = hi ? x_j1 : v[j];
+          const float u = hi ? v[j + 1] : x_j;
+          const int jj = j + (hi ? 1 : 0);
+          if (c * 32 + jj < p.n_pad && t0 + jj < p.m) {
+            const float a = g / (1.0f + expf(-g)) * u;
+            p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] = __float2bfloat16_rn(a);
           }
         }
-        __syncthreads();
       }
     }
   }
@@ -200,30 +197,32 @@ uint32_t pow2_at_least(uint32_t v) {
 GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, int32_t max_splits,
                    int32_t num_sms) {
   GemmPlan best;
+  const int force_chunks = 0;
   const int kb_total = k / kTileK;
   const int m_tiles = n_out / kTileM;
   const int min_chunks = (m + 511) / 512;
   double best_t = 1e30;
-  for (int nch = min_chunks; nch <= std::max(min_chunks * 4, 1); ++nch) {
+  // Measured on B200 (m = 448): one token chunk (all tokens of a CTA in
+  // TMEM, two N = 224 MMAs per k-step) beats finer chunks for every
+  // projection, and split-K that fills the SMs in one wave beats two waves.
+  // So: the fewest chunks that fit TMEM, then the split count whose waves
+  // cost least, counting each split's partial-sum traffic.
+  const int nch = force_chunks ? force_chunks : min_chunks;
+  {
     const int tok = (m + nch - 1) / nch;
-    int n_pad = tok <= 256 ? ((tok + 15) / 16) * 16 : ((tok + 31) / 32) * 32;
-    if (n_pad > 512) continue;
-    if (nch > min_chunks && n_pad < 64) break;  // finer chunks only help big blocks
+    const int n_pad = tok <= 256 ? ((tok + 15) / 16) * 16 : ((tok + 31) / 32) * 32;
     const int s_lo = force_splits > 0 ? force_splits : 1;
     const int s_hi = force_splits > 0 ? force_splits : std::min(max_splits, kb_total);
-    for (int s = s_lo; s <= s_hi; ++s) {
+    for (int s = s_lo; s <= s_hi && n_pad <= 512; ++s) {
       const int kbs = (kb_total + s - 1) / s;
       if ((s - 1) * kbs >= kb_total) continue;  // an empty split
       const long units = static_cast<long>(m_tiles) * nch * s;
       const long waves = (units + num_sms - 1) / num_sms;
-      const long active = std::min<long>(units, num_sms);
-      // cycles per K-block: tensor time vs weight streaming (HBM shared by active CTAs)
-      const double t_mma = 2.0 * n_pad;
-      const double t_hbm = 16384.0 / std::min(64.0, 3400.0 / active);
-      const double t_kb = std::max(t_mma, t_hbm) + 40.0;
-      const double t_epi = 4.0 * n_pad;                     // TMEM -> global stores
-      const double t_partial = s > 1 ? 1.5 * s * m * (double)n_out * 4.0 / 3400.0 : 0.0;
-      const double t = waves * (kbs * t_kb + t_epi + 600.0) + t_partial;
+      // per K-block: ~2 cycles per token column of MMA, or weight streaming
+      // when the token count is small
+      const double t_kb = std::max(2.0 * n_pad, 700.0) + 250.0;
+      const double t_partial = s > 1 ? 0.5 * s * m * (double)n_out * 4.0 / 3400.0 : 0.0;
+      const double t = waves * (kbs * t_kb + 5.0 * n_pad + 2000.0) + t_partial;
       if (t < best_t * 0.999) {
         best_t = t;
         best.n_pad = n_pad;

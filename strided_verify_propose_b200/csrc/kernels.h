@@ -18,6 +18,10 @@ int set_error(int code, const char* msg);
 // {64 columns (128 B), box_rows}, 128-byte swizzle, zero fill out of bounds.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows, std::string* err);
+// 3-D bf16 tensor map over a dense [d2][d1][d0] array (d0 innermost), box
+// {b0, b1, b2}, 128-byte swizzle (b0 * 2 must be 128), zero fill out of bounds.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t b0, uint32_t b1, uint32_t b2, std::string* err);
 
 // ---------------------------------------------------------------------- GEMM
 enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
@@ -36,7 +40,7 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
 
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
-// with W's rows interleaved in blocks of 64 (gate rows then up rows).
+// with W's rows interleaved in blocks of 16 (gate rows then up rows).
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream);
@@ -90,14 +94,28 @@ struct QkvReduceArgs {
   __nv_bfloat16* k_pool;
   __nv_bfloat16* v_pool;
   __nv_bfloat16* q_out;     // [rows][n_q][head_dim]
+  const float* delta;       // optional [rows][qkv_dim] gated-LoRA delta (MASK rows only)
+  float delta_scale;
   int32_t* status;
 };
 cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream);
 
-// x[row] += sum_s part[s][row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w).
+// x[row] += sum_s part[s][row] (+ delta_scale * delta[row] on MASK rows when
+// delta is given); hn[row] = bf16(RMSNorm(x[row]) * norm_w).
 cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
                                  const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, const float* delta = nullptr,
+                                 float delta_scale = 0.f, const int32_t* row_flags = nullptr);
+
+// ---------------------------------------------------------------- gated LoRA
+cudaError_t launch_pack_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst,
+                             int dst_ld, int row0, int col0, int interleave_off,
+                             cudaStream_t stream);
+cudaError_t launch_sum_cast(const float* part, int splits, int rows, int n, __nv_bfloat16* out,
+                            cudaStream_t stream);
+cudaError_t launch_lora_silu(const float* gu, const float* delta, float scale,
+                             const int32_t* row_flags, int rows, int inter, __nv_bfloat16* act,
+                             cudaStream_t stream);
 
 // ---------------------------------------------------------- accept / propose
 struct AcceptArgs {

@@ -115,11 +115,14 @@ __global__ void __launch_bounds__(256)
 // x[row] += sum_s part[s][row] (fixed order); hn[row] = bf16(RMSNorm(x[row]) * w).
 __global__ void __launch_bounds__(256)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
-                         const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
+                         const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
+                         const float* delta, float delta_scale, const int32_t* row_flags) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   float* xr = x + static_cast<int64_t>(row) * hidden;
   const float* pr = part + static_cast<int64_t>(row) * hidden;
+  const float* dr = (delta && (row_flags[row] & kRowMask)) ? delta + static_cast<int64_t>(row) * hidden
+                                                          : nullptr;
   float ss = 0.f;
   for (int i = threadIdx.x * 4; i < hidden; i += 256 * 4) {
     float4 v = *reinterpret_cast<const float4*>(xr + i);
@@ -129,6 +132,13 @@ __global__ void __launch_bounds__(256)
       v.y += d.y;
       v.z += d.z;
       v.w += d.w;
+    }
+    if (dr) {   // gated-LoRA delta: MASK rows only
+      const float4 d = *reinterpret_cast<const float4*>(dr + i);
+      v.x += delta_scale * d.x;
+      v.y += delta_scale * d.y;
+      v.z += delta_scale * d.z;
+      v.w += delta_scale * d.w;
     }
     *reinterpret_cast<float4*>(xr + i) = v;
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
@@ -149,8 +159,10 @@ __global__ void __launch_bounds__(256)
 // QKV split-K reduction, then per head: RMSNorm over head_dim for q and k,
 // NeoX rotary embedding (pairs (i, i + d/2)) at the row's absolute position,
 // q to the attention input, k and v into the row's page slot.
+constexpr int kQkvWarps = 16;
+
 template <int HD>
-__global__ void __launch_bounds__(128) qkv_reduce_kernel(const QkvReduceArgs a) {
+__global__ void __launch_bounds__(kQkvWarps * 32) qkv_reduce_kernel(const QkvReduceArgs a) {
   constexpr int J = HD / 32;       // values per lane
   constexpr int JH = J / 2;        // partner offset (d + HD/2)
   const int row = blockIdx.x;
@@ -180,7 +192,7 @@ __global__ void __launch_bounds__(128) qkv_reduce_kernel(const QkvReduceArgs a) 
     }
   }
   const int n_heads = a.n_q + 2 * a.n_kv;
-  for (int hd = warp; hd < n_heads; hd += 4) {
+  for (int hd = warp; hd < n_heads; hd += kQkvWarps) {
     float v[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
@@ -188,6 +200,11 @@ __global__ void __launch_bounds__(128) qkv_reduce_kernel(const QkvReduceArgs a) 
       float s = 0.f;
       for (int sp = 0; sp < a.splits; ++sp) s += pr[sp * split_stride + hd * HD + d];
       v[j] = s;
+    }
+    if (a.delta && (flags & kRowMask)) {   // gated-LoRA delta: MASK rows only
+      const float* dr = a.delta + static_cast<int64_t>(row) * qkv_dim + hd * HD;
+#pragma unroll
+      for (int j = 0; j < J; ++j) v[j] += a.delta_scale * dr[lane + 32 * j];
     }
     if (hd < a.n_q + a.n_kv) {
       const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
@@ -250,17 +267,19 @@ cudaError_t launch_embed_norm(const __nv_bfloat16* embed, const float* norm_w, R
 
 cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream) {
   if (a.head_dim == 128)
-    qkv_reduce_kernel<128><<<a.rows, 128, 0, stream>>>(a);
+    qkv_reduce_kernel<128><<<a.rows, kQkvWarps * 32, 0, stream>>>(a);
   else
-    qkv_reduce_kernel<64><<<a.rows, 128, 0, stream>>>(a);
+    qkv_reduce_kernel<64><<<a.rows, kQkvWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
                                  const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, const float* delta, float delta_scale,
+                                 const int32_t* row_flags) {
   residual_norm_kernel<<<rows, 256, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
-                                                 hidden, norm_w, eps, x, hn);
+                                                 hidden, norm_w, eps, x, hn, delta, delta_scale,
+                                                 row_flags);
   return cudaGetLastError();
 }
 

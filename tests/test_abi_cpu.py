@@ -44,7 +44,7 @@ def test_last_error_is_callable_without_gpu():
     assert binding.lib().isd_last_error() is not None
 
 
-def test_gate_up_packing_interleaves_blocks_of_64():
+def test_gate_up_packing_interleaves_blocks_of_16():
     torch = pytest.importorskip("torch")
     shape = synth.ModelShape(n_layers=1, hidden=128, n_q_heads=2, n_kv_heads=1, head_dim=64,
                              intermediate=192, vocab=256, page_size=16)
@@ -52,9 +52,9 @@ def test_gate_up_packing_interleaves_blocks_of_64():
     packed = binding.pack_weights(shape, w, device="cpu")
     gu = packed["layers"][0]["w_gate_up"].float().numpy()
     g, u = w["layers"][0]["w_gate"], w["layers"][0]["w_up"]
-    for t in range(shape.intermediate // 64):
-        assert np.array_equal(gu[128 * t:128 * t + 64], g[64 * t:64 * t + 64])
-        assert np.array_equal(gu[128 * t + 64:128 * t + 128], u[64 * t:64 * t + 64])
+    for t in range(shape.intermediate // 16):
+        assert np.array_equal(gu[32 * t:32 * t + 16], g[16 * t:16 * t + 16])
+        assert np.array_equal(gu[32 * t + 16:32 * t + 32], u[16 * t:16 * t + 16])
     qkv = packed["layers"][0]["w_qkv"].float().numpy()
     assert np.array_equal(qkv[:shape.q_dim], w["layers"][0]["wq"])
     assert np.array_equal(qkv[shape.q_dim + shape.kv_dim:], w["layers"][0]["wv"])

@@ -26,13 +26,14 @@ torch = pytest.importorskip("torch")
 
 
 def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exact=0.7,
-             useed=None):
+             useed=None, lora=False):
     from strided_verify_propose_b200 import binding as B
     R = 2 * N - 1
     P = shape.page_size
     V = shape.vocab
     w = synth.decoder_weights(shape, seed=seed)
-    dec = om.Decoder(shape, w)
+    lw = synth.lora_weights(shape, rank=128, seed=seed, std=0.05) if lora else None
+    dec = om.Decoder(shape, w, lora=lw)
     lens = synth.prompt_lengths(Bn, len_lo, len_hi, seed)
     prompts = synth.prompts(shape, lens, seed)
     maxp = op.pages_covering(int(lens.max()) + steps * N + R + 1, P) + 1
@@ -42,6 +43,8 @@ def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exa
     G = shape.n_q_heads // shape.n_kv_heads
     model = B.Model(shape, B.pack_weights(shape, w), max_batch=Bn,
                     max_rows=max(Bn * R, Bn * (64 // G)), max_position=maxp * P)
+    if lora:
+        model.load_lora(lw, rank=128)
     kv = B.KVCache(shape, num_pages, table, free)
     st = B.StepState(Bn, N, V, sample=propose == oi.SAMPLE)
     B.prefill(model, kv, st, prompts)
@@ -51,7 +54,7 @@ def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exa
     assert np.array_equal(st.seq_len.cpu().numpy(), [s.seq_len for s in states])
     assert np.array_equal(st.pending[:, 0].cpu().numpy(), [s.x_star for s in states])
     flags = (B.PROPOSE_SAMPLE if propose == oi.SAMPLE else 0) | \
-            (B.VERIFY_GREEDY if verify == oi.GREEDY else 0)
+            (B.VERIFY_GREEDY if verify == oi.GREEDY else 0) | (B.USE_LORA if lora else 0)
     in_sync = [True] * Bn
     all_sync = True
     o_table, o_head = table.copy(), 0
@@ -80,7 +83,7 @@ def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exa
             drafts = list(ost.drafts)
             q_o = None if ost.q_rows is None else [q.copy() for q in ost.q_rows]
             q_g = None if q_before is None else [q_before[b, j] for j in range(len(drafts))]
-            logits, _, _ = oi.step_logits(dec, ost, N)
+            logits, _, _ = oi.step_logits(dec, ost, N, lora=lora)
             rows = g_logits[b * R:(b + 1) * R]
             n = len(drafts)
             # the rows whose outputs the method reads (restart padding is ignored)
@@ -90,7 +93,7 @@ def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exa
             for r in used:
                 assert dz[r] <= tol, (s, b, r, dz[r], tol)
             max_dz = max(max_dz, float(max(dz[r] for r in used)))
-            res = oi.isd_step(dec, ost, N, u[b], propose, verify)
+            res = oi.isd_step(dec, ost, N, u[b], propose, verify, lora=lora)
             out = _parity.compare_decision(res, int(gA[b]), int(gp[b, 0]),
                                            [int(t) for t in gp[b, 1:]], logits, rows, drafts,
                                            q_o, q_g, u[b], N, propose, verify)
