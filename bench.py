@@ -19,6 +19,13 @@ step); time is the max over ranks, value the sum of all ranks' tokens.
 
 --impl reference times the CPU oracle (fp64 numpy) on a bounded sample of
 the same workload on rank 0 and extrapolates to the same metric.
+
+--component gemm:MxNxKxS | attention:WORKLOAD times one kernel of the step
+through its C-ABI component entry (isd_gemm_bf16: Y = X W^T with M tokens,
+N outputs, K inputs, S K-splits; isd_paged_attention on the workload's
+block rows and KV lengths), one launch per step with an L2 flush between,
+and prints its duration and throughput. It is the command the kernel
+profiles are taken with.
 """
 from __future__ import annotations
 
@@ -447,6 +454,69 @@ def run_reference(args, ws, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_component(args):
+    """Average device time of one component kernel over args.steps launches."""
+    import torch
+    from strided_verify_propose_b200 import binding as Bd
+
+    torch.cuda.set_device(0)
+    torch.manual_seed(0)
+    kind, _, spec = args.component.partition(":")
+    st = torch.zeros(1, device="cuda", dtype=torch.int32)
+    if kind == "gemm":
+        m, n, k, split = (int(v) for v in spec.split("x"))
+        w = (torch.randn(n, k, device="cuda") * 0.02).to(torch.bfloat16)
+        x = torch.randn(m, k, device="cuda").to(torch.bfloat16)
+
+        def fn():
+            Bd.gemm_bf16(w, x, split, status=st)
+        work = {"flops": 2.0 * m * n * k,
+                "bytes": 2.0 * n * k + 2.0 * m * k + 4.0 * split * m * n}
+    elif kind == "attention":
+        wl = WORKLOADS[spec]
+        shape, Bn, N = wl["shape"], wl["batch"], wl["stride"]
+        R, P, hd = 2 * N - 1, shape.page_size, shape.head_dim
+        lens = synth.prompt_lengths(Bn, wl["len_lo"], wl["len_hi"], 7)
+        need = [-(-(int(L) + R) // P) for L in lens]
+        maxp = max(need) + 1
+        num_pages = int(sum(need)) + 4
+        table, _ = synth.page_layout(need, num_pages, maxp, 7)
+        pool = (1, num_pages, shape.n_kv_heads, P, hd)
+        kp = torch.randn(pool, device="cuda").to(torch.bfloat16)
+        vp = torch.randn(pool, device="cuda").to(torch.bfloat16)
+        q = torch.randn(Bn * R, shape.n_q_heads, hd, device="cuda").to(torch.bfloat16)
+        pos = torch.tensor([int(L) + r for L in lens for r in range(R)], dtype=torch.int32,
+                           device="cuda")
+        tab = torch.from_numpy(table).cuda()
+
+        def fn():
+            Bd.paged_attention(q, pos, kp, vp, tab, R, 0, status=st)
+        keys = float(sum(int(L) + R for L in lens))
+        work = {"flops": 4.0 * keys * R * shape.n_q_heads * hd,
+                "bytes": keys * shape.n_kv_heads * hd * 2 * 2 + 2.0 * q.numel() * 2}
+    else:
+        raise SystemExit(f"unknown component {args.component!r}")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+    us = total / args.steps * 1e3
+    return {"component": args.component, "avg_us": us, "launches": args.steps,
+            "tflops": work["flops"] / us * 1e-6, "gbs": work["bytes"] / us * 1e-3,
+            "l2": "256 MB flush between launches"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,9 +525,14 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="qwen3_8b_b64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--component", default=None,
+                    help="gemm:MxNxKxS or attention:WORKLOAD (one kernel, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.component:
+        print(json.dumps(run_component(args)), flush=True)
+        return
     ws, rank, local = setup_dist()
     if args.impl == "reference":
         res = run_reference(args, ws, rank)

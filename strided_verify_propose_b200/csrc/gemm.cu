@@ -41,6 +41,16 @@ struct GemmParams {
   int32_t* status;
 };
 
+// kPair: a cluster of two CTAs (adjacent 128-row weight tiles) runs as one
+// 2-SM MMA group (tcgen05 cta_group::2, M = 256). Each CTA stages its own
+// 128 weight rows and half of every MMA's token columns, so a pair reads
+// the token tile once per 256 weight rows instead of once per 128 and each
+// SM fills 16 KB + n_pad * 64 B per K-block instead of 16 KB + n_pad * 128 B.
+// The leader CTA (rank 0) issues the MMAs; both CTAs' loads complete on the
+// leader's full barrier; each commit arrives on the barrier of both CTAs.
+// Each CTA's tensor memory ends up holding its own 128 rows x all tokens, so
+// the epilogue is the same as for a single CTA.
+template <bool kPair, int kNmma>
 __global__ void __launch_bounds__(128, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
@@ -54,7 +64,11 @@ __global__ void __launch_bounds__(128, 1)
   const int sp = blockIdx.z;
   const int kb0 = sp * p.kb_per_split;
   const int nkb = min(p.kb_total, kb0 + p.kb_per_split) - kb0;
-  const uint32_t stage_bytes = kStageA + static_cast<uint32_t>(p.n_pad) * 128u;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  // token rows this CTA stages per K-block
+  const uint32_t b_rows = static_cast<uint32_t>(p.n_boxes * p.box_rows);
+  const uint32_t stage_bytes = kStageA + b_rows * 128u;
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
   uint64_t* empty = full + p.stages;
@@ -74,20 +88,29 @@ __global__ void __launch_bounds__(128, 1)
     prefetch_tensormap(&tmap_x);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(tmem_slot, p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // the peer's barriers are initialised and its tensor memory allocated
+  // before any load or MMA of the pair touches them
+  if (kPair) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (both CTAs of a pair)
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_x = policy_evict_last();
-    const uint32_t tx = kStageA + static_cast<uint32_t>(p.n_boxes * p.box_rows) * 128u;
-    for (int i = 0; i < nkb; ++i) {
+    const uint32_t tx = (kPair ? 2u : 1u) * stage_bytes;
+    int i = 0;
+    for (; i < nkb; ++i) {
       const int s = i % p.stages;
       const uint32_t ph = (i / p.stages) & 1;
       if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
@@ -98,37 +121,81 @@ __global__ void __launch_bounds__(128, 1)
       uint8_t* sa = smem + s * stage_bytes;
       uint8_t* sb = sa + kStageA;
       const int kc = (kb0 + i) * kTileK;
-      mbar_arrive_expect_tx(&full[s], tx);
-      tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
-      for (int bx = 0; bx < p.n_boxes; ++bx)
-        tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc, tok0 + bx * p.box_rows,
-                         pol_x);
+      if (kPair) {
+        const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
+        if (leader) mbar_arrive_expect_tx(&full[s], tx);
+        tma_load_2d_pair(sa, &tmap_w, bar, kc, mt * kTileM, pol_w);
+        for (int bx = 0; bx < p.n_boxes; ++bx)
+          tma_load_2d_pair(sb + bx * p.box_rows * 128, &tmap_x, bar, kc,
+                           tok0 + bx * p.mma_n + static_cast<int>(rank) * p.box_rows, pol_x);
+      } else {
+        mbar_arrive_expect_tx(&full[s], tx);
+        tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
+        for (int bx = 0; bx < p.n_boxes; ++bx)
+          tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc,
+                           tok0 + bx * p.box_rows, pol_x);
+      }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    const uint32_t idesc = idesc_bf16_m128(static_cast<uint32_t>(p.mma_n));
+    if (kPair && i == nkb) {
+      // Drain: the leader's last commits still arrive on this CTA's empty
+      // barriers; wait for them so none lands after the CTA has exited.
+      for (int j = max(0, nkb - p.stages); j < nkb; ++j) {
+        if (!mbar_wait(&empty[j % p.stages], (j / p.stages) & 1)) {
+          flag(p.status, ISD_DEV_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------- MMA issuer (the leader of a pair)
+    // One thread issues every MMA, so its loop is kept to the bare
+    // instructions: descriptors advance by adding the byte offset >> 4 to
+    // precomputed bases (smem addresses stay below 2^18, inside the 14-bit
+    // address field), and the k-steps and MMAs of a stage are unrolled.
+    const uint32_t idesc = idesc_bf16(kPair ? 256u : 128u, static_cast<uint32_t>(p.mma_n));
+    const uint32_t base = smem_u32(smem);
+    const uint64_t da0 = sw128_desc(base);
+    const uint64_t db0 = sw128_desc(base + kStageA);
+    const uint64_t d_stage = stage_bytes >> 4;
+    // offset between consecutive MMAs' token tiles in this CTA, >> 4
+    const uint64_t d_mma = (static_cast<uint64_t>(kPair ? p.box_rows : p.mma_n) * 128u) >> 4;
+    const uint32_t tmem1 = tmem + static_cast<uint32_t>(p.mma_n);
+    int s = 0;
+    uint32_t ph = 0;
     for (int i = 0; i < nkb; ++i) {
-      const int s = i % p.stages;
-      const uint32_t ph = (i / p.stages) & 1;
-      if (!mbar_wait(&full[s], ph) || *abort_flag) {
+      if (!mbar_wait(&full[s], ph)) {
         flag(p.status, ISD_DEV_TIMEOUT);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t a_base = smem_u32(smem + s * stage_bytes);
-      const uint32_t b_base = a_base + kStageA;
+      const uint64_t da = da0 + static_cast<uint64_t>(s) * d_stage;
+      const uint64_t db = db0 + static_cast<uint64_t>(s) * d_stage;
 #pragma unroll
       for (int kk = 0; kk < kTileK / 16; ++kk) {
-        const uint64_t da = sw128_desc(a_base + kk * 32);
-        for (int j = 0; j < p.n_mma; ++j) {
-          const uint64_t db = sw128_desc(b_base + j * p.mma_n * 128 + kk * 32);
-          umma_bf16(tmem + j * p.mma_n, da, db, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        if (kPair) {
+          umma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
+          if (kNmma == 2) umma_bf16_pair(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
+        } else {
+          umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
+          if (kNmma == 2) umma_bf16(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
         }
       }
-      umma_commit(&empty[s]);
+      if (kPair)
+        umma_commit_pair(&empty[s]);
+      else
+        umma_commit(&empty[s]);
+      if (++s == p.stages) {
+        s = 0;
+        ph ^= 1;
+      }
     }
-    umma_commit(accum);
+    if (kPair)
+      umma_commit_pair(accum);
+    else
+      umma_commit(accum);
   }
   __syncwarp();
 
@@ -180,9 +247,15 @@ __global__ void __launch_bounds__(128, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair frees its tensor memory or exits while the other
+  // may still read it or signal its barriers
+  if (kPair) cluster_sync();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, p.tmem_cols);
+    if (kPair)
+      tmem_dealloc_pair(tmem, p.tmem_cols);
+    else
+      tmem_dealloc(tmem, p.tmem_cols);
   }
 }
 
@@ -235,9 +308,19 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
   if (best.n_pad == 0) return best;
   best.n_mma = best.n_pad > 256 ? 2 : 1;
   best.mma_n = best.n_pad / best.n_mma;
-  best.box_rows = best.n_pad > 256 ? best.n_pad / 2 : best.n_pad;
-  best.n_boxes = best.n_pad / best.box_rows;
-  const size_t stage = kStageA + static_cast<size_t>(best.n_pad) * 128;
+  // 2-SM pairs need an even number of 128-row tiles; mma_n is a multiple of
+  // 16 (n_pad is padded to 16, or to 32 when split over two MMAs), so each
+  // CTA's half of an MMA's tokens is a whole number of 8-row swizzle atoms.
+  best.pair = (m_tiles % 2 == 0 && best.mma_n % 16 == 0) ? 1 : 0;
+  if (best.pair) {
+    best.box_rows = best.mma_n / 2;
+    best.n_boxes = best.n_mma;
+  } else {
+    best.box_rows = best.n_pad > 256 ? best.n_pad / 2 : best.n_pad;
+    best.n_boxes = best.n_pad / best.box_rows;
+  }
+  const size_t stage =
+      kStageA + static_cast<size_t>(best.n_boxes) * static_cast<size_t>(best.box_rows) * 128;
   const size_t extra = 1024 + 256;
   int stages = static_cast<int>((kMaxSmem - extra) / stage);
   stages = std::min(stages, 8);
@@ -251,14 +334,19 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream) {
+  auto kernel = plan.pair ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
+                         : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kMaxSmem));
-    if (e != cudaSuccess) return e;
+    for (auto fn : {gemm_bf16_tcgen05<false, 1>, gemm_bf16_tcgen05<false, 2>,
+                    gemm_bf16_tcgen05<true, 1>, gemm_bf16_tcgen05<true, 2>}) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kMaxSmem));
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
+  if (plan.n_mma != 1 && plan.n_mma != 2) return cudaErrorInvalidValue;
   GemmParams p;
   p.m = m;
   p.n_out = n_out;
@@ -277,8 +365,24 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.split_stride = static_cast<int64_t>(m) * n_out;
   p.status = status;
   dim3 grid(n_out / kTileM, plan.n_chunks, plan.splits);
-  gemm_bf16_tcgen05<<<grid, 128, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
-  return cudaGetLastError();
+  if (!plan.pair) {
+    kernel<<<grid, 128, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
+    return cudaGetLastError();
+  }
+  if (grid.x % 2 != 0) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = plan.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, tmap_w, tmap_x, p);
 }
 
 }  // namespace isd

@@ -29,6 +29,7 @@ enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
 struct GemmPlan {
   int32_t n_pad = 0, n_mma = 0, mma_n = 0, box_rows = 0, n_boxes = 0;
   int32_t n_chunks = 0, splits = 0, kb_per_split = 0, stages = 0;
+  int32_t pair = 0;  // 1: clusters of two CTAs issue 2-SM (cta_group::2) MMAs
   uint32_t tmem_cols = 0;
   size_t smem_bytes = 0;
 };

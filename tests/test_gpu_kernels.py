@@ -33,10 +33,13 @@ def _bf16(a):
 # ------------------------------------------------------------------- GEMM ---
 
 @pytest.mark.parametrize("m,n,k,split", [
-    (7, 256, 256, 1),          # decode b1 rows, one tile
+    (7, 256, 256, 1),          # decode b1 rows, one 2-SM pair of tiles
+    (7, 384, 256, 1),          # odd tile count: single-CTA MMAs
     (28, 512, 1024, 3),        # ragged split-K
     (300, 384, 640, 1),        # ragged token count, n_pad not a multiple of 32
     (448, 1024, 512, 2),       # b64 x stride 4 rows, two MMAs per k-step
+    (448, 1152, 1024, 1),      # the same rows over an odd tile count
+    (96, 512, 256, 1),         # one MMA of 96 tokens split 48 / 48 over a pair
     (1000, 256, 256, 1),       # two token chunks (prefill chunk)
     (448, 6144, 4096, 3),      # Qwen3-8B QKV at b64, split 3
     (448, 4096, 12288, 4),     # Qwen3-8B down projection at b64
