@@ -159,7 +159,10 @@ __global__ void __launch_bounds__(256)
 // QKV split-K reduction, then per head: RMSNorm over head_dim for q and k,
 // NeoX rotary embedding (pairs (i, i + d/2)) at the row's absolute position,
 // q to the attention input, k and v into the row's page slot.
+// Grid (rows, ceil(heads / kQkvWarps)): one warp per (row, head), so every
+// warp has all of its split loads in flight at once.
 constexpr int kQkvWarps = 16;
+constexpr int kQkvMaxSplits = 8;
 
 template <int HD>
 __global__ void __launch_bounds__(kQkvWarps * 32) qkv_reduce_kernel(const QkvReduceArgs a) {
@@ -167,75 +170,75 @@ __global__ void __launch_bounds__(kQkvWarps * 32) qkv_reduce_kernel(const QkvRed
   constexpr int JH = J / 2;        // partner offset (d + HD/2)
   const int row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qkv_dim = (a.n_q + 2 * a.n_kv) * HD;
+  const int n_heads = a.n_q + 2 * a.n_kv;
+  const int hd = blockIdx.y * kQkvWarps + warp;
+  if (hd >= n_heads) return;
+  const int qkv_dim = n_heads * HD;
   const int64_t split_stride = static_cast<int64_t>(a.rows) * qkv_dim;
-  const float* pr = a.part + static_cast<int64_t>(row) * qkv_dim;
+  const float* pr = a.part + static_cast<int64_t>(row) * qkv_dim + hd * HD + lane;
   const int flags = a.meta.flags[row];
   int pos = a.meta.pos[row];
   const bool write_kv = (flags & kRowWriteKV) && pos >= 0;
   if (pos >= a.max_position) {
-    if (threadIdx.x == 0) flag(a.status, ISD_DEV_BAD_STATE);
+    if (lane == 0 && hd == 0) flag(a.status, ISD_DEV_BAD_STATE);
     pos = a.max_position - 1;
   }
   const int rpos = pos < 0 ? 0 : pos;
-  int64_t slot_base = -1;
-  if (write_kv) {
+  float v[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) v[j] = 0.f;
+  // splits added in ascending order (bitwise reproducible)
+#pragma unroll
+  for (int sp = 0; sp < kQkvMaxSplits; ++sp) {
+    if (sp < a.splits) {
+#pragma unroll
+      for (int j = 0; j < J; ++j) v[j] += pr[sp * split_stride + 32 * j];
+    }
+  }
+  if (a.delta && (flags & kRowMask)) {   // gated-LoRA delta: MASK rows only
+    const float* dr = a.delta + static_cast<int64_t>(row) * qkv_dim + hd * HD;
+#pragma unroll
+    for (int j = 0; j < J; ++j) v[j] += a.delta_scale * dr[lane + 32 * j];
+  }
+  if (hd < a.n_q + a.n_kv) {
+    const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) ss += v[j] * v[j];
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / HD + a.eps);
+#pragma unroll
+    for (int j = 0; j < J; ++j) v[j] *= rstd * nw[lane + 32 * j];
+    const float2* cs = a.rope + static_cast<int64_t>(rpos) * (HD / 2);
+#pragma unroll
+    for (int j = 0; j < JH; ++j) {
+      const float2 c = cs[lane + 32 * j];
+      const float x1 = v[j], x2 = v[j + JH];
+      v[j] = x1 * c.x - x2 * c.y;
+      v[j + JH] = x2 * c.x + x1 * c.y;
+    }
+  }
+  if (hd < a.n_q) {
+    __nv_bfloat16* qo = a.q_out + (static_cast<int64_t>(row) * a.n_q + hd) * HD;
+#pragma unroll
+    for (int j = 0; j < J; ++j) qo[lane + 32 * j] = __float2bfloat16_rn(v[j]);
+  } else if (write_kv) {
     const int b = row / a.rows_per_req;
     const int pidx = pos / a.page_size;
     const int page = pidx < a.max_pages_per_req
                          ? a.page_table[static_cast<int64_t>(b) * a.max_pages_per_req + pidx]
                          : -1;
     if (page < 0 || page >= a.num_pages) {
-      if (threadIdx.x == 0) flag(a.status, ISD_DEV_BAD_PAGE);
-    } else {
-      slot_base = (static_cast<int64_t>(a.layer) * a.num_pages + page) * a.n_kv;  // * P + slot below
+      if (lane == 0) flag(a.status, ISD_DEV_BAD_PAGE);
+      return;
     }
-  }
-  const int n_heads = a.n_q + 2 * a.n_kv;
-  for (int hd = warp; hd < n_heads; hd += kQkvWarps) {
-    float v[J];
+    const int64_t slot_base = (static_cast<int64_t>(a.layer) * a.num_pages + page) * a.n_kv;
+    const bool is_k = hd < a.n_q + a.n_kv;
+    const int g = is_k ? hd - a.n_q : hd - a.n_q - a.n_kv;
+    __nv_bfloat16* dst = (is_k ? a.k_pool : a.v_pool) +
+                         (((slot_base + g) * a.page_size) + pos % a.page_size) * HD;
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      const int d = lane + 32 * j;
-      float s = 0.f;
-      for (int sp = 0; sp < a.splits; ++sp) s += pr[sp * split_stride + hd * HD + d];
-      v[j] = s;
-    }
-    if (a.delta && (flags & kRowMask)) {   // gated-LoRA delta: MASK rows only
-      const float* dr = a.delta + static_cast<int64_t>(row) * qkv_dim + hd * HD;
-#pragma unroll
-      for (int j = 0; j < J; ++j) v[j] += a.delta_scale * dr[lane + 32 * j];
-    }
-    if (hd < a.n_q + a.n_kv) {
-      const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < J; ++j) ss += v[j] * v[j];
-      ss = warp_sum(ss);
-      const float rstd = rsqrtf(ss / HD + a.eps);
-#pragma unroll
-      for (int j = 0; j < J; ++j) v[j] *= rstd * nw[lane + 32 * j];
-      const float2* cs = a.rope + static_cast<int64_t>(rpos) * (HD / 2);
-#pragma unroll
-      for (int j = 0; j < JH; ++j) {
-        const float2 c = cs[lane + 32 * j];
-        const float x1 = v[j], x2 = v[j + JH];
-        v[j] = x1 * c.x - x2 * c.y;
-        v[j + JH] = x2 * c.x + x1 * c.y;
-      }
-    }
-    if (hd < a.n_q) {
-      __nv_bfloat16* qo = a.q_out + (static_cast<int64_t>(row) * a.n_q + hd) * HD;
-#pragma unroll
-      for (int j = 0; j < J; ++j) qo[lane + 32 * j] = __float2bfloat16_rn(v[j]);
-    } else if (slot_base >= 0) {
-      const bool is_k = hd < a.n_q + a.n_kv;
-      const int g = is_k ? hd - a.n_q : hd - a.n_q - a.n_kv;
-      __nv_bfloat16* dst = (is_k ? a.k_pool : a.v_pool) +
-                           (((slot_base + g) * a.page_size) + pos % a.page_size) * HD;
-#pragma unroll
-      for (int j = 0; j < J; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(v[j]);
-    }
+    for (int j = 0; j < J; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(v[j]);
   }
 }
 
@@ -266,10 +269,12 @@ cudaError_t launch_embed_norm(const __nv_bfloat16* embed, const float* norm_w, R
 }
 
 cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream) {
+  if (a.splits < 1 || a.splits > kQkvMaxSplits) return cudaErrorInvalidValue;
+  const dim3 grid(a.rows, (a.n_q + 2 * a.n_kv + kQkvWarps - 1) / kQkvWarps);
   if (a.head_dim == 128)
-    qkv_reduce_kernel<128><<<a.rows, kQkvWarps * 32, 0, stream>>>(a);
+    qkv_reduce_kernel<128><<<grid, kQkvWarps * 32, 0, stream>>>(a);
   else
-    qkv_reduce_kernel<64><<<a.rows, kQkvWarps * 32, 0, stream>>>(a);
+    qkv_reduce_kernel<64><<<grid, kQkvWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
