@@ -198,6 +198,21 @@ void isd_destroy(isd_ctx *ctx);
 int isd_gemm_bf16(const void *w_dev, const void *x_dev, float *y_dev, int32_t m, int32_t n,
                   int32_t k, int32_t split_k, int32_t *status_dev, void *stream);
 
+/* Y = X W^T as one fp32 slice, planned as a step plans its single-slice
+ * projections (the MLP gate/up, the LM head): when the 128-row weight tiles
+ * overfill one wave of SMs it runs as stream-K, CTAs sharing the (tile,
+ * K-block) iterations, and a tile cut between two CTAs is completed by the
+ * one that finishes second from the other's fp32 partial, parked in the
+ * workspace. Same operand layouts and limits as isd_gemm_bf16.
+ *  workspace_dev: isd_gemm_workspace_bytes(m, n, k) bytes (0: none needed,
+ *  may be NULL). Its first 4096 bytes must be zero before the first call;
+ *  each call leaves them zero, so a workspace serves any number of calls
+ *  in stream order (not two calls running at once). */
+size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k);
+int isd_gemm_bf16_single(const void *w_dev, const void *x_dev, float *y_dev, int32_t m,
+                         int32_t n, int32_t k, void *workspace_dev, size_t workspace_bytes,
+                         int32_t *status_dev, void *stream);
+
 /* Paged causal GQA attention for one layer.
  *  q_dev [B*R][n_q_heads][head_dim] bf16 (already QK-normed and rotated)
  *  row_pos_dev [B*R] int32: position of each row; a row sees keys t <= pos

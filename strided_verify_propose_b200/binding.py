@@ -33,7 +33,7 @@ EXPORTS = ("isd_init", "isd_load_gated_lora", "isd_step", "isd_prefill", "isd_la
            "isd_last_error", "isd_destroy", "isd_gemm_bf16", "isd_attention_workspace_bytes",
            "isd_paged_attention", "isd_accept_workspace_bytes", "isd_accept_propose",
            "isd_profile_enable", "isd_profile_read", "isd_profile_class_name",
-           "isd_accept_propose_noalloc")
+           "isd_accept_propose_noalloc", "isd_gemm_workspace_bytes", "isd_gemm_bf16_single")
 PROF_CLASSES = 16
 
 
@@ -91,6 +91,9 @@ def lib():
     L.isd_destroy.argtypes = [vp]
     L.isd_destroy.restype = None
     L.isd_gemm_bf16.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    L.isd_gemm_workspace_bytes.argtypes = [i32, i32, i32]
+    L.isd_gemm_workspace_bytes.restype = sz
+    L.isd_gemm_bf16_single.argtypes = [vp, vp, vp, i32, i32, i32, vp, sz, vp, vp]
     L.isd_attention_workspace_bytes.argtypes = [i32] * 7
     L.isd_attention_workspace_bytes.restype = sz
     L.isd_paged_attention.argtypes = [vp, vp, vp, vp, vp] + [i32] * 10 + [vp, vp, sz, vp, vp]
@@ -353,6 +356,26 @@ def gemm_bf16(w, x, split_k: int = 1, status=None):
     y = torch.empty(split_k, m, n, device=x.device, dtype=torch.float32)
     st = status if status is not None else torch.zeros(1, device=x.device, dtype=torch.int32)
     check(lib().isd_gemm_bf16(_ptr(w), _ptr(x), _ptr(y), m, n, k, split_k, _ptr(st), _stream()))
+    return y
+
+
+def gemm_workspace(m: int, n: int, k: int, device="cuda"):
+    """A zeroed workspace for gemm_bf16_single at this shape (None if not needed)."""
+    import torch
+    nb = int(lib().isd_gemm_workspace_bytes(m, n, k))
+    return torch.zeros(nb, device=device, dtype=torch.uint8) if nb else None
+
+
+def gemm_bf16_single(w, x, workspace=None, status=None):
+    """Y[m][n] = X W^T as one fp32 slice (stream-K when the tiles overfill a wave)."""
+    import torch
+    n, k = w.shape
+    m = x.shape[0]
+    y = torch.empty(m, n, device=x.device, dtype=torch.float32)
+    st = status if status is not None else torch.zeros(1, device=x.device, dtype=torch.int32)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    check(lib().isd_gemm_bf16_single(_ptr(w), _ptr(x), _ptr(y), m, n, k, ws_ptr, ws_bytes, _ptr(st),
+                                     _stream()))
     return y
 
 

@@ -148,7 +148,9 @@ struct isd_ctx {
   int32_t* prefill_lens = nullptr;  // [max_batch]
 
   std::map<std::tuple<const void*, int, int, int>, CUtensorMap> act_maps;
-  std::map<std::tuple<int, int, int>, GemmPlan> plans;
+  std::map<std::tuple<int, int, int, int>, GemmPlan> plans;
+  void* sk_ws = nullptr;            // stream-K partials + sync words (sync words zeroed)
+  size_t sk_ws_bytes = 0;
   int launches = 0;
 
   // gated LoRA (R-ISD): packed adapters per layer + their workspace
@@ -220,11 +222,16 @@ int tmap_for(isd_ctx* c, const void* base, int rows, int cols, int box_rows, CUt
   return ISD_OK;
 }
 
-const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k) {
-  auto key = std::make_tuple(m, n, k);
+// single: one output slice (the SiLU epilogue, the LM head); such plans may
+// run as stream-K when the tiles overfill one wave.
+const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k, bool single) {
+  auto key = std::make_tuple(m, n, k, single ? 1 : 0);
   auto it = c->plans.find(key);
-  if (it == c->plans.end())
-    it = c->plans.emplace(key, isd::plan_gemm(m, n, k, 0, c->max_splits, num_sms())).first;
+  if (it == c->plans.end()) {
+    const GemmPlan p = single ? isd::plan_gemm(m, n, k, 0, 1, num_sms(), true)
+                              : isd::plan_gemm(m, n, k, 0, c->max_splits, num_sms());
+    it = c->plans.emplace(key, p).first;
+  }
   return it->second;
 }
 
@@ -234,11 +241,10 @@ const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k) {
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st) {
-  GemmPlan plan = plan_for(c, m, n, k);
-  if ((epi == isd::kEpiSiluMul || max_splits == 1) && plan.splits != 1) {
-    plan = isd::plan_gemm(m, n, k, 1, 1, num_sms());
-  }
+  const GemmPlan& plan = plan_for(c, m, n, k, epi == isd::kEpiSiluMul || max_splits == 1);
   if (plan.n_pad == 0) return fail(ISD_E_UNSUPPORTED, "no GEMM plan");
+  if (isd::gemm_streamk_workspace_bytes(plan) > c->sk_ws_bytes)
+    return fail(ISD_E_UNSUPPORTED, "stream-K workspace too small for the GEMM plan");
   if (plan.splits > max_splits) return fail(ISD_E_UNSUPPORTED, "GEMM plan exceeds the split limit");
   if (epi == isd::kEpiF32 &&
       static_cast<size_t>(plan.splits) * static_cast<size_t>(m) * static_cast<size_t>(n) > out_elems)
@@ -247,7 +253,8 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   int rc = tmap_for(c, x, m, k, plan.box_rows, &tx);
   if (rc) return rc;
   cudaEvent_t e0 = prof_mark(c, st);
-  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st));
+  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
+                            c->sk_ws_bytes));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
@@ -463,6 +470,9 @@ int alloc_workspace(isd_ctx* c) {
   c->attn_ws_bytes = isd::attention_workspace_bytes(a);
   const int maxN = 8;
   c->acc_ws_bytes = isd::accept_workspace_bytes(g.max_batch, maxN, g.vocab);
+  // stream-K: one slot per SM of fp32 partials of up to 512 tokens x 128 rows
+  c->sk_ws_bytes = isd::gemm_streamk_sync_bytes() +
+                   static_cast<size_t>(num_sms()) * 512 * 128 * sizeof(float);
   size_t sizes[] = {
       R * g.hidden * sizeof(float),                       // x
       R * g.hidden * 2,                                   // hn
@@ -475,6 +485,7 @@ int alloc_workspace(isd_ctx* c) {
       static_cast<size_t>(g.max_position) * (g.head_dim / 2) * sizeof(float2),  // rope
       c->attn_ws_bytes, c->acc_ws_bytes,
       static_cast<size_t>(g.max_batch) * 4,
+      c->sk_ws_bytes,
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -501,6 +512,9 @@ int alloc_workspace(isd_ctx* c) {
   c->attn_ws = b + off[i++];
   c->acc_ws = b + off[i++];
   c->prefill_lens = reinterpret_cast<int32_t*>(b + off[i++]);
+  c->sk_ws = b + off[i++];
+  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
+    return fail(ISD_E_CUDA, "stream-K workspace clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;
   std::vector<float2> tab(static_cast<size_t>(g.max_position) * half);
@@ -865,6 +879,32 @@ int isd_gemm_bf16(const void* w_dev, const void* x_dev, float* y_dev, int32_t m,
     return fail(ISD_E_INVALID, "tensor map: " + err);
   ISD_CUDA(isd::launch_gemm(tw, tx, plan, m, n, k, isd::kEpiF32, y_dev, nullptr, status_dev,
                             static_cast<cudaStream_t>(stream)));
+  return ISD_OK;
+}
+
+size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k) {
+  if (m < 1 || m > 4096 || n < 128 || n % 128 || k < 64 || k % 64) return 0;
+  return isd::gemm_streamk_workspace_bytes(isd::plan_gemm(m, n, k, 0, 1, num_sms(), true));
+}
+
+int isd_gemm_bf16_single(const void* w_dev, const void* x_dev, float* y_dev, int32_t m, int32_t n,
+                         int32_t k, void* workspace_dev, size_t workspace_bytes,
+                         int32_t* status_dev, void* stream) {
+  if (!w_dev || !x_dev || !y_dev) return fail(ISD_E_INVALID, "null argument");
+  if (m < 1 || m > 4096 || n < 128 || n % 128 || k < 64 || k % 64)
+    return fail(ISD_E_UNSUPPORTED, "need 1<=m<=4096, n%128==0, k%64==0");
+  GemmPlan plan = isd::plan_gemm(m, n, k, 0, 1, num_sms(), true);
+  if (plan.n_pad == 0) return fail(ISD_E_UNSUPPORTED, "no GEMM plan");
+  const size_t need = isd::gemm_streamk_workspace_bytes(plan);
+  if (need > 0 && (workspace_dev == nullptr || workspace_bytes < need))
+    return fail(ISD_E_INVALID, "workspace smaller than isd_gemm_workspace_bytes");
+  std::string err;
+  CUtensorMap tw, tx;
+  if (!isd::make_tmap_bf16(&tw, w_dev, n, k, 128, &err) ||
+      !isd::make_tmap_bf16(&tx, x_dev, m, k, plan.box_rows, &err))
+    return fail(ISD_E_INVALID, "tensor map: " + err);
+  ISD_CUDA(isd::launch_gemm(tw, tx, plan, m, n, k, isd::kEpiF32, y_dev, nullptr, status_dev,
+                            static_cast<cudaStream_t>(stream), workspace_dev, workspace_bytes));
   return ISD_OK;
 }
 

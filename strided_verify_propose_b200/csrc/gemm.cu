@@ -7,19 +7,31 @@
 // 512) form N, so every weight byte is read from HBM once and the fp32
 // accumulators of the whole token range sit in tensor memory (<= 512 columns).
 //
-// Per CTA: warp 0 (one lane) issues TMA loads of a 128x64 weight tile and an
-// n_pad x 64 activation tile per K-block into a ring of shared-memory
-// stages; warp 1 (one lane) issues tcgen05.mma and releases each stage with
-// tcgen05.commit; then all four warps read the accumulators back with
-// tcgen05.ld (one TMEM lane per thread = one output feature) and store.
-// Split-K CTAs write their partial sums to separate slices that a row-wise
-// kernel adds in a fixed order, so results are bitwise reproducible.
+// Warp roles: warp 0 (one lane) issues TMA loads of a 128x64 weight tile and
+// the token tile per K-block into a ring of shared-memory stages; warp 1
+// (one lane) issues tcgen05.mma and releases each stage with tcgen05.commit;
+// warps 2..9 read the accumulators back with tcgen05.ld (a warp reads the 32
+// TMEM lanes of its quadrant, warp % 4; two warps share a quadrant and split
+// its columns) and run the epilogue.
+//
+// Work split, two modes:
+// * split-K: one (tile, token chunk, K-split) per CTA; split s writes its
+//   partial sums to slice s, which a row-wise kernel adds in a fixed order;
+// * stream-K (when there are more tiles than SMs): a persistent grid where
+//   each CTA, or 2-SM pair, owns a contiguous range of the (tile, K-block)
+//   iterations. Ranges are at least one tile long, so a tile is cut at most
+//   once; of its two parts the first to finish parks its fp32 partial in a
+//   workspace slot and the second adds it to its own and runs the epilogue.
+//   Two addends commute exactly, so results do not depend on which part
+//   finishes first, and no CTA ever waits for one that has not started.
+// Both are bitwise reproducible run to run.
 #include <algorithm>
 #include <cmath>
 #include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
+
 
 namespace isd {
 
@@ -28,7 +40,9 @@ namespace {
 constexpr int kTileM = 128;                 // weight rows per CTA
 constexpr int kTileK = 64;                  // K elements per stage (128 bytes)
 constexpr int kStageA = kTileM * kTileK * 2;  // 16 KB
-constexpr size_t kMaxSmem = 232448;         // 227 KB dynamic shared memory
+constexpr size_t kMaxSmem = 231424;         // 226 KB dynamic (+ a few static bytes <= 227 KB)
+constexpr int kEpiWarps = 8;                // epilogue warps (two per TMEM quadrant)
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 struct GemmParams {
   int32_t m, n_out, kb_total, kb_per_split;
@@ -39,31 +53,72 @@ struct GemmParams {
   __nv_bfloat16* out_act;
   int64_t split_stride;
   int32_t* status;
+  // stream-K: `units` CTAs or pairs share the iterations of all tiles
+  int32_t streamk, units;
+  int64_t iters;      // unit tiles (256-row pair tiles or 128-row tiles) x kb_total
+  float* sk_part;     // [units * (pair ? 2 : 1)][n_pad][128] fp32 partials
+  int32_t* sk_sync;   // [units * (pair ? 2 : 1)][2]: arrival count, ready flag
 };
+
+// One contiguous run of K-blocks of one tile, processed by one CTA (pair).
+struct Segment {
+  int ut;          // unit tile (pair tile for pairs)
+  int kb_lo, kb_hi;
+  bool whole;      // covers every K-block of the tile (or split-K mode)
+  int slot;        // stream-K workspace slot of a cut tile (per unit boundary)
+};
+
+// The idx-th segment of this CTA's work; false past the last one.
+template <bool kPair>
+__device__ __forceinline__ bool get_segment(const GemmParams& p, int idx, Segment& sg) {
+  if (!p.streamk) {
+    if (idx > 0) return false;
+    const int kb0 = blockIdx.z * p.kb_per_split;
+    sg.ut = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+    sg.kb_lo = kb0;
+    sg.kb_hi = min(p.kb_total, kb0 + p.kb_per_split);
+    sg.whole = true;
+    sg.slot = -1;
+    return true;
+  }
+  const int u = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+  const int64_t b = static_cast<int64_t>(u) * p.iters / p.units;
+  const int64_t e = static_cast<int64_t>(u + 1) * p.iters / p.units;
+  const int64_t kbt = p.kb_total;
+  const int64_t tile = b / kbt + idx;
+  const int64_t lo = max(b, tile * kbt), hi = min(e, (tile + 1) * kbt);
+  if (lo >= hi) return false;
+  sg.ut = static_cast<int>(tile);
+  sg.kb_lo = static_cast<int>(lo - tile * kbt);
+  sg.kb_hi = static_cast<int>(hi - tile * kbt);
+  sg.whole = sg.kb_lo == 0 && sg.kb_hi == p.kb_total;
+  // a cut tile straddles the boundary between units s and s + 1: the head
+  // part ends unit s's range (slot s = u), the tail part starts unit s + 1's
+  // (slot s = u - 1)
+  sg.slot = sg.whole ? -1 : (sg.kb_lo == 0 ? u : u - 1);
+  return true;
+}
 
 // kPair: a cluster of two CTAs (adjacent 128-row weight tiles) runs as one
 // 2-SM MMA group (tcgen05 cta_group::2, M = 256). Each CTA stages its own
 // 128 weight rows and half of every MMA's token columns, so a pair reads
-// the token tile once per 256 weight rows instead of once per 128 and each
-// SM fills 16 KB + n_pad * 64 B per K-block instead of 16 KB + n_pad * 128 B.
-// The leader CTA (rank 0) issues the MMAs; both CTAs' loads complete on the
-// leader's full barrier; each commit arrives on the barrier of both CTAs.
-// Each CTA's tensor memory ends up holding its own 128 rows x all tokens, so
-// the epilogue is the same as for a single CTA.
+// the token tile once per 256 weight rows instead of once per 128. The
+// leader CTA (rank 0) issues the MMAs; both CTAs' loads complete on the
+// leader's full barrier; each commit arrives on the barrier of both CTAs;
+// the epilogue warps of both CTAs release the accumulator on the leader's
+// tmem_empty barrier. Each CTA's tensor memory holds its own 128 rows x all
+// tokens, so the epilogue is the same as for a single CTA.
 template <bool kPair, int kNmma>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  __shared__ int epi_mode;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = blockIdx.x;
   const int tok0 = blockIdx.y * p.n_pad;
-  const int sp = blockIdx.z;
-  const int kb0 = sp * p.kb_per_split;
-  const int nkb = min(p.kb_total, kb0 + p.kb_per_split) - kb0;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
   // token rows this CTA stages per K-block
@@ -72,8 +127,9 @@ __global__ void __launch_bounds__(128, 1)
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.stages * stage_bytes);
   uint64_t* empty = full + p.stages;
-  uint64_t* accum = empty + p.stages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* tmem_full = empty + p.stages;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -81,7 +137,8 @@ __global__ void __launch_bounds__(128, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, kEpiWarps * (kPair ? 2 : 1));
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmap_w);
@@ -99,7 +156,7 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   // the peer's barriers are initialised and its tensor memory allocated
-  // before any load or MMA of the pair touches them
+  // before any load, MMA or arrive of the pair touches them
   if (kPair) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -109,37 +166,48 @@ __global__ void __launch_bounds__(128, 1)
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_x = policy_evict_last();
     const uint32_t tx = (kPair ? 2u : 1u) * stage_bytes;
-    int i = 0;
-    for (; i < nkb; ++i) {
-      const int s = i % p.stages;
-      const uint32_t ph = (i / p.stages) & 1;
-      if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
-        flag(p.status, ISD_DEV_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      uint8_t* sa = smem + s * stage_bytes;
-      uint8_t* sb = sa + kStageA;
-      const int kc = (kb0 + i) * kTileK;
-      if (kPair) {
-        const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
-        if (leader) mbar_arrive_expect_tx(&full[s], tx);
-        tma_load_2d_pair(sa, &tmap_w, bar, kc, mt * kTileM, pol_w);
-        for (int bx = 0; bx < p.n_boxes; ++bx)
-          tma_load_2d_pair(sb + bx * p.box_rows * 128, &tmap_x, bar, kc,
-                           tok0 + bx * p.mma_n + static_cast<int>(rank) * p.box_rows, pol_x);
-      } else {
-        mbar_arrive_expect_tx(&full[s], tx);
-        tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
-        for (int bx = 0; bx < p.n_boxes; ++bx)
-          tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc,
-                           tok0 + bx * p.box_rows, pol_x);
+    int s = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    bool ok = true;
+    Segment sg;
+    for (int idx = 0; ok && get_segment<kPair>(p, idx, sg); ++idx) {
+      const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
+      for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+        if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
+          flag(p.status, ISD_DEV_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * stage_bytes;
+        uint8_t* sb = sa + kStageA;
+        const int kc = kb * kTileK;
+        if (kPair) {
+          const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], tx);
+          tma_load_2d_pair(sa, &tmap_w, bar, kc, mt * kTileM, pol_w);
+          for (int bx = 0; bx < p.n_boxes; ++bx)
+            tma_load_2d_pair(sb + bx * p.box_rows * 128, &tmap_x, bar, kc,
+                             tok0 + bx * p.mma_n + static_cast<int>(rank) * p.box_rows, pol_x);
+        } else {
+          mbar_arrive_expect_tx(&full[s], tx);
+          tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
+          for (int bx = 0; bx < p.n_boxes; ++bx)
+            tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc,
+                             tok0 + bx * p.box_rows, pol_x);
+        }
+        ++issued;
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1;
+        }
       }
     }
-    if (kPair && i == nkb) {
-      // Drain: the leader's last commits still arrive on this CTA's empty
-      // barriers; wait for them so none lands after the CTA has exited.
-      for (int j = max(0, nkb - p.stages); j < nkb; ++j) {
+    if (ok) {
+      // Drain: the last commits still arrive on this CTA's empty barriers;
+      // wait for them so none lands after the CTA has exited.
+      for (int j = max(0, issued - p.stages); j < issued; ++j) {
         if (!mbar_wait(&empty[j % p.stages], (j / p.stages) & 1)) {
           flag(p.status, ISD_DEV_TIMEOUT);
           *abort_flag = 1;
@@ -163,88 +231,174 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem1 = tmem + static_cast<uint32_t>(p.mma_n);
     int s = 0;
     uint32_t ph = 0;
-    for (int i = 0; i < nkb; ++i) {
-      if (!mbar_wait(&full[s], ph)) {
+    bool ok = true;
+    Segment sg;
+    for (int idx = 0; ok && get_segment<kPair>(p, idx, sg); ++idx) {
+      // the epilogue has read the previous segment's accumulators
+      if (!mbar_wait(tmem_empty, (idx & 1) ^ 1)) {
         flag(p.status, ISD_DEV_TIMEOUT);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const uint64_t da = da0 + static_cast<uint64_t>(s) * d_stage;
-      const uint64_t db = db0 + static_cast<uint64_t>(s) * d_stage;
+      for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+        if (!mbar_wait(&full[s], ph)) {
+          flag(p.status, ISD_DEV_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t da = da0 + static_cast<uint64_t>(s) * d_stage;
+        const uint64_t db = db0 + static_cast<uint64_t>(s) * d_stage;
 #pragma unroll
-      for (int kk = 0; kk < kTileK / 16; ++kk) {
-        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        if (kPair) {
-          umma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
-          if (kNmma == 2) umma_bf16_pair(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
-        } else {
-          umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
-          if (kNmma == 2) umma_bf16(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
+        for (int kk = 0; kk < kTileK / 16; ++kk) {
+          const uint32_t acc = (kb > sg.kb_lo || kk > 0) ? 1u : 0u;
+          if (kPair) {
+            umma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
+            if (kNmma == 2) umma_bf16_pair(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
+          } else {
+            umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
+            if (kNmma == 2) umma_bf16(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
+          }
+        }
+        if (kPair)
+          umma_commit_pair(&empty[s]);
+        else
+          umma_commit(&empty[s]);
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1;
         }
       }
+      if (!ok) break;
       if (kPair)
-        umma_commit_pair(&empty[s]);
+        umma_commit_pair(tmem_full);
       else
-        umma_commit(&empty[s]);
-      if (++s == p.stages) {
-        s = 0;
-        ph ^= 1;
-      }
+        umma_commit(tmem_full);
     }
-    if (kPair)
-      umma_commit_pair(accum);
-    else
-      umma_commit(accum);
-  }
-  __syncwarp();
-
-  // ---------------- epilogue: TMEM -> registers -> global
-  const bool ok = __syncthreads_and(mbar_wait(accum, 0) && !*abort_flag);
-  tc_fence_after();
-  if (!ok) {
-    if (threadIdx.x == 0) flag(p.status, ISD_DEV_TIMEOUT);
-  } else {
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> registers -> global
+    const int ew = warp - 2;
+    const int quad = warp & 3;             // TMEM lanes 32 * quad .. + 31
+    const int half = ew >> 2;              // which of the quadrant's two warps
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const int nchunk = (p.n_pad + 31) / 32;  // tmem_cols >= 32 * nchunk
-    if (p.epi == kEpiF32) {
-      const int f = mt * kTileM + warp * 32 + lane;
-      float* outp = p.out + sp * p.split_stride + f;
-      for (int c = 0; c < nchunk; ++c) {
-        float v[32];
-        tmem_ld_32x32(lane_addr + c * 32, v);
-        const int t0 = tok0 + c * 32;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c * 32 + j < p.n_pad && t0 + j < p.m)
-            outp[static_cast<int64_t>(t0 + j) * p.n_out] = v[j];
+    const uint32_t empty_addr = kPair ? map_to_rank(smem_u32(tmem_empty), 0) : 0u;
+    const int split = p.streamk ? 0 : static_cast<int>(blockIdx.z);
+    Segment sg;
+    for (int idx = 0; get_segment<kPair>(p, idx, sg); ++idx) {
+      // every epilogue warp takes the same branch (they share named barriers)
+      const bool ok =
+          named_bar_and(1, 32 * kEpiWarps, mbar_wait(tmem_full, idx & 1) && !*abort_flag);
+      if (!ok) {
+        if (lane == 0) flag(p.status, ISD_DEV_TIMEOUT);
+        break;
       }
-    } else {
-      // Each warp's 32 TMEM lanes hold 16 gate rows then the 16 up rows of
-      // the same features (see the gate/up layout in isd.h). A lane pairs
-      // with lane ^ 16: low lanes finish even tokens, high lanes odd ones.
-      const int half_n = p.n_out / 2;
-      const bool hi = lane >= 16;
-      const int f = mt * 64 + warp * 16 + (lane & 15);
-      for (int c = 0; c < nchunk; ++c) {
+      tc_fence_after();
+      const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
+      // cut tile: 1 = first part to finish (park the partial), 2 = second
+      // (add the parked partial, then the normal epilogue), 3 = second after
+      // a timeout (status flagged, nothing written)
+      int mode = 0;
+      float* part = nullptr;
+      int32_t* sync = nullptr;
+      if (!sg.whole) {
+        const int slot = sg.slot * (kPair ? 2 : 1) + static_cast<int>(rank);
+        part = p.sk_part + static_cast<int64_t>(slot) * p.n_pad * kTileM;
+        sync = p.sk_sync + 2 * slot;
+        if (ew == 0 && lane == 0) {
+          int m_ = atomicAdd(&sync[0], 1) == 0 ? 1 : 2;
+          if (m_ == 2) {
+            // the first part's CTA is in its epilogue: wait for its flag
+            const long long t0 = clock64();
+            while (ld_acquire_gpu(&sync[1]) == 0) {
+              if (clock64() - t0 > kWaitCycles) {
+                flag(p.status, ISD_DEV_TIMEOUT);
+                m_ = 3;
+                break;
+              }
+            }
+          }
+          epi_mode = m_;
+        }
+        named_bar_sync(1, 32 * kEpiWarps);
+        mode = epi_mode;
+      }
+      for (int c = half; c < nchunk; c += 2) {
         float v[32];
         tmem_ld_32x32(lane_addr + c * 32, v);
         const int t0 = tok0 + c * 32;
+        // partial slot rows: tokens 0 .. n_pad - 1 of this CTA's 128 rows
+        if (mode == 1) {
+          float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
-          const float x_j1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 16);
-          const float g = hi ? x_j1 : v[j];
-          const float u = hi ? v[j + 1] : x_j;
-          const int jj = j + (hi ? 1 : 0);
-          if (c * 32 + jj < p.n_pad && t0 + jj < p.m) {
-            const float a = g / (1.0f + expf(-g)) * u;
-            p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] = __float2bfloat16_rn(a);
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.n_pad) pp[j * kTileM] = v[j];
+          continue;
+        }
+        if (mode == 3) continue;
+        if (mode == 2) {
+          const float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
+          // L2 loads: another SM wrote the slot
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.n_pad) v[j] += __ldcg(pp + j * kTileM);
+        }
+        if (p.epi == kEpiF32) {
+          const int f = mt * kTileM + quad * 32 + lane;
+          float* outp = p.out + split * p.split_stride + f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < p.n_pad && t0 + j < p.m)
+              outp[static_cast<int64_t>(t0 + j) * p.n_out] = v[j];
+        } else {
+          // Each quadrant's 32 TMEM lanes hold 16 gate rows then the 16 up
+          // rows of the same features (see the gate/up layout in isd.h). A
+          // lane pairs with lane ^ 16: low lanes finish even tokens, high
+          // lanes odd ones.
+          const int half_n = p.n_out / 2;
+          const bool hi = lane >= 16;
+          const int f = mt * 64 + quad * 16 + (lane & 15);
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
+            const float x_j1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 16);
+            const float g = hi ? x_j1 : v[j];
+            const float u = hi ? v[j + 1] : x_j;
+            const int jj = j + (hi ? 1 : 0);
+            if (c * 32 + jj < p.n_pad && t0 + jj < p.m) {
+              const float a = g / (1.0f + expf(-g)) * u;
+              p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] = __float2bfloat16_rn(a);
+            }
           }
         }
       }
+      // accumulators read: release them to the MMA issuer (of the pair)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair)
+          mbar_arrive_cluster(empty_addr);
+        else
+          mbar_arrive(tmem_empty);
+      }
+      if (mode == 1) {
+        // partial parked: publish it
+        __threadfence();
+        named_bar_sync(1, 32 * kEpiWarps);
+        if (ew == 0 && lane == 0) st_release_gpu(&sync[1], 1);
+      } else if (mode >= 2) {
+        // every read of the parked partial is done: reset the slot
+        named_bar_sync(1, 32 * kEpiWarps);
+        if (ew == 0 && lane == 0) {
+          sync[1] = 0;
+          sync[0] = 0;
+        }
+      }
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   // neither CTA of a pair frees its tensor memory or exits while the other
@@ -268,9 +422,8 @@ uint32_t pow2_at_least(uint32_t v) {
 }  // namespace
 
 GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, int32_t max_splits,
-                   int32_t num_sms) {
+                   int32_t num_sms, bool allow_streamk) {
   GemmPlan best;
-  const int force_chunks = 0;
   const int kb_total = k / kTileK;
   const int m_tiles = n_out / kTileM;
   const int min_chunks = (m + 511) / 512;
@@ -280,7 +433,7 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
   // projection, and split-K that fills the SMs in one wave beats two waves.
   // So: the fewest chunks that fit TMEM, then the split count whose waves
   // cost least, counting each split's partial-sum traffic.
-  const int nch = force_chunks ? force_chunks : min_chunks;
+  const int nch = min_chunks;
   {
     const int tok = (m + nch - 1) / nch;
     const int n_pad = tok <= 256 ? ((tok + 15) / 16) * 16 : ((tok + 31) / 32) * 32;
@@ -319,23 +472,50 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
     best.box_rows = best.n_pad > 256 ? best.n_pad / 2 : best.n_pad;
     best.n_boxes = best.n_pad / best.box_rows;
   }
+  // Stream-K when one chunk and one split leave more tiles than one wave
+  // holds, and the last wave would be partly idle. Every range spans at
+  // least one tile (unit_tiles > cap), so a tile is cut at most once.
+  const int per_unit = best.pair ? 2 : 1;
+  const int unit_tiles = m_tiles / per_unit;
+  const int cap = std::max(1, num_sms / per_unit);
+  if (allow_streamk && force_splits <= 0 && best.n_chunks == 1 && best.splits == 1 &&
+      unit_tiles > cap && unit_tiles % cap != 0) {
+    best.streamk = 1;
+    best.units = cap;
+  }
   const size_t stage =
       kStageA + static_cast<size_t>(best.n_boxes) * static_cast<size_t>(best.box_rows) * 128;
   const size_t extra = 1024 + 256;
   int stages = static_cast<int>((kMaxSmem - extra) / stage);
   stages = std::min(stages, 8);
-  stages = std::min(stages, std::max(best.kb_per_split, 2));
+  if (!best.streamk) stages = std::min(stages, std::max(best.kb_per_split, 2));
   best.stages = std::max(stages, 2);
   best.tmem_cols = pow2_at_least(static_cast<uint32_t>(best.n_pad));
   best.smem_bytes = best.stages * stage + extra;
   return best;
 }
 
+// Workspace layout: the sync words of up to kSkMaxSlots slots at offset 0
+// (the same place for every plan, so a plan's partials never overwrite
+// another plan's sync words), then the fp32 partials.
+constexpr size_t kSkMaxSlots = 512;
+constexpr size_t kSkSyncBytes = kSkMaxSlots * 2 * sizeof(int32_t);
+
+size_t gemm_streamk_workspace_bytes(const GemmPlan& plan) {
+  if (!plan.streamk) return 0;
+  const size_t slots = static_cast<size_t>(plan.units) * (plan.pair ? 2 : 1);
+  return kSkSyncBytes + slots * static_cast<size_t>(plan.n_pad) * kTileM * sizeof(float);
+}
+
+size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }
+
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
-                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream) {
-  auto kernel = plan.pair ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
-                         : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
+                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
+                        void* sk_workspace, size_t sk_workspace_bytes) {
+  auto kernel = plan.pair
+                    ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
+                    : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
   static bool attr_set = false;
   if (!attr_set) {
     for (auto fn : {gemm_bf16_tcgen05<false, 1>, gemm_bf16_tcgen05<false, 2>,
@@ -364,15 +544,34 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.out_act = out_act;
   p.split_stride = static_cast<int64_t>(m) * n_out;
   p.status = status;
+  p.streamk = plan.streamk;
+  p.units = plan.units;
+  p.iters = 0;
+  p.sk_part = nullptr;
+  p.sk_sync = nullptr;
+  const int per_unit = plan.pair ? 2 : 1;
   dim3 grid(n_out / kTileM, plan.n_chunks, plan.splits);
+  if (plan.streamk) {
+    const size_t need = gemm_streamk_workspace_bytes(plan);
+    if (sk_workspace == nullptr || sk_workspace_bytes < need || plan.n_chunks != 1 ||
+        plan.splits != 1 || plan.units < 1 ||
+        static_cast<size_t>(plan.units) * per_unit > kSkMaxSlots)
+      return cudaErrorInvalidValue;
+    const int64_t unit_tiles = n_out / kTileM / per_unit;
+    p.iters = unit_tiles * p.kb_total;
+    if (p.iters / plan.units < p.kb_total) return cudaErrorInvalidValue;  // a range < one tile
+    p.sk_sync = static_cast<int32_t*>(sk_workspace);
+    p.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(sk_workspace) + kSkSyncBytes);
+    grid = dim3(plan.units * per_unit, 1, 1);
+  }
   if (!plan.pair) {
-    kernel<<<grid, 128, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
+    kernel<<<grid, kThreads, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
     return cudaGetLastError();
   }
   if (grid.x % 2 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = plan.smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

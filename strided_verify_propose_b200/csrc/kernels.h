@@ -29,22 +29,31 @@ enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
 struct GemmPlan {
   int32_t n_pad = 0, n_mma = 0, mma_n = 0, box_rows = 0, n_boxes = 0;
   int32_t n_chunks = 0, splits = 0, kb_per_split = 0, stages = 0;
-  int32_t pair = 0;  // 1: clusters of two CTAs issue 2-SM (cta_group::2) MMAs
+  int32_t pair = 0;     // 1: clusters of two CTAs issue 2-SM (cta_group::2) MMAs
+  int32_t streamk = 0;  // 1: persistent ranges of (tile, K-block) iterations
+  int32_t units = 0;    // stream-K: CTAs (pairs) sharing the iterations
   uint32_t tmem_cols = 0;
   size_t smem_bytes = 0;
 };
 
 // Tile plan for Y[m][n_out] = X[m][k] W[n_out][k]^T. force_splits > 0 pins
-// the split-K factor; max_splits bounds the automatic choice.
+// the split-K factor; max_splits bounds the automatic choice; allow_streamk
+// lets a single-split plan with more tiles than one wave run as stream-K
+// (its output is one slice; it needs gemm_streamk_workspace_bytes of
+// workspace whose first gemm_streamk_sync_bytes() bytes, the sync words,
+// start at zero; every launch leaves them at zero).
 GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, int32_t max_splits,
-                   int32_t num_sms);
+                   int32_t num_sms, bool allow_streamk = false);
+size_t gemm_streamk_workspace_bytes(const GemmPlan& plan);
+size_t gemm_streamk_sync_bytes();
 
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
 // with W's rows interleaved in blocks of 16 (gate rows then up rows).
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
-                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream);
+                        __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
+                        void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {

@@ -58,6 +58,34 @@ def test_gemm_matches_fp64_product(cuda_lib, m, n, k, split):
     assert err <= 2e-4 * np.abs(ref).max(), err
 
 
+@pytest.mark.parametrize("m,n,k", [
+    (448, 19072, 256),         # 149 single-CTA tiles on 148 SMs: stream-K, cut tiles
+    (448, 20480, 512),         # 80 pair tiles on 74 pairs: stream-K with 2-SM MMAs
+    (7, 19072, 256),           # decode b1 rows through the same split
+    (300, 2048, 256),          # fewer tiles than SMs: plain single slice
+])
+def test_gemm_single_slice_streamk(cuda_lib, m, n, k):
+    """Stream-K parity with the fp64 product, and bitwise equal on a repeat
+    (the cut tiles' fixups must not depend on which part finishes first)."""
+    B = _b(0)
+    x = synth.bf16_round(synth.normal((m, k), 3, 1))
+    w = synth.bf16_round(synth.normal((n, k), 3, 2, std=0.02))
+    wd, xd = _bf16(w), _bf16(x)
+    ws = B.gemm_workspace(m, n, k)
+    st = torch.zeros(1, device="cuda", dtype=torch.int32)
+    y1 = B.gemm_bf16_single(wd, xd, ws, status=st)
+    y2 = B.gemm_bf16_single(wd, xd, ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(y1, y2)
+    if ws is not None:
+        assert int(ws[:4096].count_nonzero().item()) == 0   # sync words left at zero
+    got = y1.double().cpu().numpy()
+    ref = x.astype(np.float64) @ w.astype(np.float64).T
+    err = np.abs(got - ref).max()
+    assert err <= 2e-4 * np.abs(ref).max(), err
+
+
 # -------------------------------------------------------------- attention ---
 
 def _attention_case(shape_args, lens, R, seed, pad_row=False):
