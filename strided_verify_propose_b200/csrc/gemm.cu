@@ -56,7 +56,7 @@ struct GemmParams {
   // stream-K: `units` CTAs or pairs share the iterations of all tiles
   int32_t streamk, units;
   int64_t iters;      // unit tiles (256-row pair tiles or 128-row tiles) x kb_total
-  float* sk_part;     // [units * (pair ? 2 : 1)][n_pad][128] fp32 partials
+  float* sk_part;     // [units * (pair ? 2 : 1)][n_pad rounded up to 32][128] fp32 partials
   int32_t* sk_sync;   // [units * (pair ? 2 : 1)][2]: arrival count, ready flag
 };
 
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t* sync = nullptr;
       if (!sg.whole) {
         const int slot = sg.slot * (kPair ? 2 : 1) + static_cast<int>(rank);
-        part = p.sk_part + static_cast<int64_t>(slot) * p.n_pad * kTileM;
+        part = p.sk_part + static_cast<int64_t>(slot) * nchunk * 32 * kTileM;
         sync = p.sk_sync + 2 * slot;
         if (ew == 0 && lane == 0) {
           int m_ = atomicAdd(&sync[0], 1) == 0 ? 1 : 2;
@@ -325,16 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_sync(1, 32 * kEpiWarps);
         mode = epi_mode;
       }
+      // TMEM loads run one chunk ahead of the chunk being written out
+      uint32_t r[32];
+      if (half < nchunk) tmem_ld_32x32_async(lane_addr + half * 32, r);
       for (int c = half; c < nchunk; c += 2) {
         float v[32];
-        tmem_ld_32x32(lane_addr + c * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (c + 2 < nchunk) tmem_ld_32x32_async(lane_addr + (c + 2) * 32, r);
         const int t0 = tok0 + c * 32;
-        // partial slot rows: tokens 0 .. n_pad - 1 of this CTA's 128 rows
+        // partial slot: rows of 128 fp32, tokens 0 .. 32 * nchunk - 1
         if (mode == 1) {
           float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < p.n_pad) pp[j * kTileM] = v[j];
+          for (int j = 0; j < 32; ++j) pp[j * kTileM] = v[j];
           continue;
         }
         if (mode == 3) continue;
@@ -342,8 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
           // L2 loads: another SM wrote the slot
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < p.n_pad) v[j] += __ldcg(pp + j * kTileM);
+          for (int j = 0; j < 32; ++j) v[j] += __ldcg(pp + j * kTileM);
         }
         if (p.epi == kEpiF32) {
           const int f = mt * kTileM + quad * 32 + lane;
@@ -367,10 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float g = hi ? x_j1 : v[j];
             const float u = hi ? v[j + 1] : x_j;
             const int jj = j + (hi ? 1 : 0);
-            if (c * 32 + jj < p.n_pad && t0 + jj < p.m) {
-              const float a = g / (1.0f + expf(-g)) * u;
-              p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] = __float2bfloat16_rn(a);
-            }
+            if (c * 32 + jj < p.n_pad && t0 + jj < p.m)
+              p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] =
+                  __float2bfloat16_rn(silu_mul(g, u));
           }
         }
       }
@@ -504,7 +507,8 @@ constexpr size_t kSkSyncBytes = kSkMaxSlots * 2 * sizeof(int32_t);
 size_t gemm_streamk_workspace_bytes(const GemmPlan& plan) {
   if (!plan.streamk) return 0;
   const size_t slots = static_cast<size_t>(plan.units) * (plan.pair ? 2 : 1);
-  return kSkSyncBytes + slots * static_cast<size_t>(plan.n_pad) * kTileM * sizeof(float);
+  const size_t rows = (static_cast<size_t>(plan.n_pad) + 31) / 32 * 32;
+  return kSkSyncBytes + slots * rows * kTileM * sizeof(float);
 }
 
 size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }

@@ -41,9 +41,9 @@ __global__ void sum_cast_kernel(const float* part, int splits, int64_t split_str
 }
 
 // act[row][f] = bf16(SiLU(g) * u), g and u read from the base gate/up
-// output (16-row interleave), plus scale * delta on MASK rows only. The
-// expression is the one the fused GEMM epilogue evaluates, so verify rows get
-// the same bits as a step without the adapter.
+// output (16-row interleave), plus scale * delta on MASK rows only. silu_mul
+// is the expression the fused GEMM epilogue evaluates, so verify rows get the
+// same bits as a step without the adapter.
 __global__ void lora_silu_kernel(const float* gu, const float* delta, float scale,
                                  const int32_t* row_flags, int inter, __nv_bfloat16* act) {
   const int row = blockIdx.x;
@@ -57,8 +57,7 @@ __global__ void lora_silu_kernel(const float* gu, const float* delta, float scal
       g += scale * dr[gc];
       u += scale * dr[gc + 16];
     }
-    const float a = g / (1.0f + expf(-g)) * u;
-    act[static_cast<int64_t>(row) * inter + f] = __float2bfloat16_rn(a);
+    act[static_cast<int64_t>(row) * inter + f] = __float2bfloat16_rn(silu_mul(g, u));
   }
 }
 
