@@ -45,6 +45,9 @@ struct AttnParams {
   float* part_o;               // [item][MT*16][HD]
   float2* part_ml;             // [item][MT*16]  (max (log2 units), sum)
   int32_t* item_base;          // [B+1] first split index of each request (written by CTA 0)
+  // tcgen05 kernel: balanced contiguous tile ranges
+  int32_t max_parts;           // partial slots per (request, KV head)
+  int32_t min_tiles;           // fewest tiles per CTA (fewer CTAs for small work)
   int32_t* status;
 };
 
@@ -99,12 +102,14 @@ struct ItemTable {
   int base[kMaxBatch + 1];   // exclusive prefix of the split counts
 };
 
-__device__ void build_items(const AttnParams& p, ItemTable& t) {
+// kend[b]: keys request b attends to; base[b]: exclusive prefix of the
+// per-request split counts (base[B] = total). Ends with __syncthreads.
+__device__ void build_items(const AttnParams& p, int* kend, int* base) {
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
     int ke = 0;
     for (int r = 0; r < p.R; ++r) ke = max(ke, p.row_pos[b * p.R + r] + 1);
     ke = min(ke, p.maxp * p.page_size);
-    t.kend[b] = ke;
+    kend[b] = ke;
   }
   __syncthreads();
   if (threadIdx.x < 32) {
@@ -113,7 +118,7 @@ __device__ void build_items(const AttnParams& p, ItemTable& t) {
     const int per = (p.B + 31) / 32;
     const int b0 = lane * per, b1 = min(p.B, b0 + per);
     int local = 0;
-    for (int b = b0; b < b1; ++b) local += t.kend[b] > 0 ? (t.kend[b] + p.split_keys - 1) / p.split_keys : 0;
+    for (int b = b0; b < b1; ++b) local += kend[b] > 0 ? (kend[b] + p.split_keys - 1) / p.split_keys : 0;
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -122,27 +127,36 @@ __device__ void build_items(const AttnParams& p, ItemTable& t) {
     }
     int run = incl - local;
     for (int b = b0; b < b1; ++b) {
-      t.base[b] = run;
-      run += t.kend[b] > 0 ? (t.kend[b] + p.split_keys - 1) / p.split_keys : 0;
+      base[b] = run;
+      run += kend[b] > 0 ? (kend[b] + p.split_keys - 1) / p.split_keys : 0;
     }
-    if (lane == 31) t.base[p.B] = incl;
+    if (lane == 31) base[p.B] = incl;
   }
   __syncthreads();
 }
 
+__device__ __forceinline__ void build_items(const AttnParams& p, ItemTable& t) {
+  build_items(p, t.kend, t.base);
+}
+
 // item -> (b, g, split): items are ordered request-major, then KV head, then split.
-__device__ __forceinline__ void decode_item(const AttnParams& p, const ItemTable& t, int item,
-                                            int& b, int& g, int& sp) {
+__device__ __forceinline__ void decode_item(const AttnParams& p, const int* base, int item, int& b,
+                                            int& g, int& sp) {
   int lo = 0, hi = p.B;   // find b with base[b]*nkv <= item < base[b+1]*nkv
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (t.base[mid] * p.nkv <= item) lo = mid; else hi = mid;
+    if (base[mid] * p.nkv <= item) lo = mid; else hi = mid;
   }
   b = lo;
-  const int ns = t.base[b + 1] - t.base[b];
-  const int rem = item - t.base[b] * p.nkv;
+  const int ns = base[b + 1] - base[b];
+  const int rem = item - base[b] * p.nkv;
   g = rem / ns;
   sp = rem % ns;
+}
+
+__device__ __forceinline__ void decode_item(const AttnParams& p, const ItemTable& t, int item,
+                                            int& b, int& g, int& sp) {
+  decode_item(p, t.base, item, b, g, sp);
 }
 
 // Persistent paged attention. HD: head dim; NG: tile groups. Warp w works on
@@ -456,6 +470,517 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 variant (head_dim 128, 64-key pages, at most 32 query rows per KV
+// head): the contractions run on the 5th-generation tensor cores with fp32
+// accumulators in tensor memory, so the tile math no longer competes with
+// the HBM stream.
+//
+// Per 128-key tile (two pages) of a work item:
+//   S^T[key][row] = K Q^T     UMMA M = 128 keys, N = 32 rows, K = 128 dims
+//   P = exp2(S * scale - m)   softmax warps: TMEM lane = key, column = row
+//   O_t^T[dim][row] = V^T P^T UMMA M = 128 dims (V read MN-major), N = 32,
+//                             K = 128 keys; P^T staged in shared memory
+//   O = O * alpha + O_t       softmax warps, registers (lane = dim)
+// Warps 0-3 (one TMEM lane quadrant each) run the softmax and accumulate O;
+// warp 4 is the TMA producer, warp 5 issues the MMAs. S and O_t tiles are
+// double-buffered in tensor memory, so the MMA of tile t+1 runs while the
+// softmax warps work on tile t. Items, splits and the partial-sum format are
+// those of the mma.sync kernel; the same combine kernel finishes.
+constexpr int kTcKeys = 128;                 // keys per tile (two 64-key pages)
+constexpr int kTcNP = 32;                    // query rows per tile (UMMA N)
+constexpr int kTcSoftWarps = 8;              // two per TMEM lane quadrant
+constexpr int kTcRows = kTcNP / 2;           // query rows per softmax warp
+constexpr int kTcThreads = (kTcSoftWarps + 2) * 32;
+constexpr int kTcStage = 2 * kTcKeys * 128 * 2;   // K and V tiles, 64 KB
+constexpr int kTcHalf = 64 * 128;                 // one [64 keys][64 dims] box, 8 KB
+constexpr int kTcQBuf = 2 * kTcNP * 128;          // Q: two 64-dim halves of NP rows, 8 KB
+constexpr int kTcPBuf = 2 * kTcNP * 128;          // P^T: two 64-key halves of NP rows, 8 KB
+constexpr int kTcMisc = 2048;                     // reduction scratch, row state
+constexpr int kTcBars = 256;
+constexpr int kTcMinTiles = 2;                    // fewest tiles per working CTA
+
+// Max or sum of v[0..15] over the 32 lanes, reduce-scatter style: after 16
+// shuffles lanes 2i and 2i+1 both hold the reduction of value i.
+template <bool kMax>
+__device__ __forceinline__ float lane_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 2; off >>= 1) {
+    const int h = off / 2;               // values kept this step
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 1);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
+}
+
+// 2^x with the hardware approximation (flushes denormal results to zero;
+// 2^-126 is far below what a softmax weight needs).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo_bytes) {
+  // MN-major, 128-byte swizzle: 64 MN elements per 128-byte row, rows along
+  // K 128 B apart, 8-row groups 1024 B apart (SBO), 64-element MN blocks
+  // lbo_bytes apart (LBO).
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Work of the tcgen05 kernel: the tiles of all (request, KV head) pairs in
+// one sequence, request-major, then head, then tile; CTA c of the C working
+// CTAs takes tiles [c T / C, (c+1) T / C). A maximal run of one (request,
+// head) inside a CTA's range is a segment; it leaves its partial output in
+// slot (b * nkv + g) * max_parts + (c - first CTA of that pair).
+struct TcSeg {
+  int b, g, t0, len, slot;
+};
+
+struct TcRange {
+  int64_t x, hi, T;
+  int C;
+};
+
+__device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ int tc_cta_of(int64_t x, int64_t T, int C) {
+  return static_cast<int>(((x + 1) * C - 1) / T);
+}
+
+// tile prefix per request in base[0..B] (base[b] = tiles before request b)
+__device__ __forceinline__ TcRange tc_range(const AttnParams& p, const int* base) {
+  TcRange r;
+  r.T = static_cast<int64_t>(p.nkv) * base[p.B];
+  r.C = static_cast<int>(i64max(1, i64min(gridDim.x, r.T / p.min_tiles)));
+  const int c = blockIdx.x;
+  r.x = c < r.C ? c * r.T / r.C : 0;
+  r.hi = c < r.C ? (c + 1) * r.T / r.C : 0;
+  return r;
+}
+
+__device__ __forceinline__ bool tc_next(const AttnParams& p, const int* base, TcRange& r, TcSeg& sg) {
+  if (r.x >= r.hi) return false;
+  int lo = 0, hi = p.B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (static_cast<int64_t>(base[mid]) * p.nkv <= r.x) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int nt = base[b + 1] - base[b];
+  const int64_t x0b = static_cast<int64_t>(base[b]) * p.nkv;
+  const int rem = static_cast<int>(r.x - x0b);
+  sg.b = b;
+  sg.g = rem / nt;
+  sg.t0 = rem % nt;
+  sg.len = static_cast<int>(i64min(r.hi - r.x, nt - sg.t0));
+  const int64_t first = x0b + static_cast<int64_t>(sg.g) * nt;
+  const int part = static_cast<int>(blockIdx.x) - tc_cta_of(first, r.T, r.C);
+  sg.slot = part < p.max_parts ? (b * p.nkv + sg.g) * p.max_parts + part : -1;
+  r.x += sg.len;
+  return true;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                   const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
+  constexpr int NP = kTcNP;
+  constexpr int NR = kTcRows;
+  constexpr int kSoftThreads = kTcSoftWarps * 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = smem;                                   // stages x [K | V]
+  uint8_t* qs = ring + p.stages * kTcStage;               // 2 x Q
+  uint8_t* ps = qs + 2 * kTcQBuf;                         // P^T
+  float* red = reinterpret_cast<float*>(ps + kTcPBuf);    // [4 quadrants][NP]
+  float* m_sh = red + 4 * NP;                             // running max per row (log2 units)
+  float* alpha_sh = m_sh + NP;                            // [2][NP] per-tile rescale
+  float* l_sh = alpha_sh + 2 * NP;                        // row sums at item end
+  int* pos_sh = reinterpret_cast<int*>(l_sh + NP);        // row positions of the item
+  int* minpos_sh = pos_sh + NP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kTcMisc);
+  uint64_t* full = bars;
+  uint64_t* empty = full + p.stages;
+  uint64_t* q_full = empty + p.stages;     // [2]
+  uint64_t* q_empty = q_full + 2;          // [2]
+  uint64_t* s_full = q_empty + 2;          // [2]
+  uint64_t* s_empty = s_full + 2;          // [2]
+  uint64_t* o_full = s_empty + 2;          // [2]
+  uint64_t* o_empty = o_full + 2;          // [2]
+  uint64_t* p_full = o_empty + 2;
+  uint64_t* p_empty = p_full + 1;
+  uint64_t* drain = p_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + kTcBars);
+  int* kend = reinterpret_cast<int*>(tmem_slot + 4);
+  int* base = kend + p.B;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kTcSoftWarps);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], kTcSoftWarps);
+    }
+    mbar_init(p_full, kTcSoftWarps);
+    mbar_init(p_empty, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  // query rows past the tile's RG rows are never loaded: keep them zero
+  for (int i = threadIdx.x; i < 2 * kTcQBuf / 16; i += blockDim.x)
+    reinterpret_cast<int4*>(qs)[i] = make_int4(0, 0, 0, 0);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 4 * NP);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  build_items(p, kend, base);     // ends with __syncthreads
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // base[b]: tiles of the requests before b (128-key tiles, split_keys = 128)
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.item_base[b] = base[b];
+  const bool fits = true;
+
+  if (warp == kTcSoftWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && fits) {
+      int tc = 0, it = 0, q_issued = 0;
+      bool ok = true;
+      TcRange rg = tc_range(p, base);
+      TcSeg sg;
+      for (; ok && tc_next(p, base, rg, sg); ++it) {
+        const int b = sg.b, g = sg.g;
+        const int k_lo = sg.t0 * kTcKeys;
+        const int k_hi = min(kend[b], k_lo + sg.len * kTcKeys);
+        const int n_tiles = sg.len;
+        const int qb = it & 1;
+        if (!mbar_wait(&q_empty[qb], ((it >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[qb], 2 * p.RG * 128);
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_3d(qs + qb * kTcQBuf + hh * (NP * 128), &qmap, &q_full[qb], hh * 64, g * p.G,
+                      b * p.R);
+        ++q_issued;
+        const int32_t* pt = p.page_table + static_cast<int64_t>(b) * p.maxp;
+        for (int t = 0; t < n_tiles; ++t, ++tc) {
+          const int st = tc % p.stages;
+          if (!mbar_wait(&empty[st], ((tc / p.stages) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* ks = ring + st * kTcStage;
+          uint8_t* vs = ks + kTcStage / 2;
+          mbar_arrive_expect_tx(&full[st], kTcStage);
+          for (int j = 0; j < 2; ++j) {
+            const int key0 = k_lo + t * kTcKeys + j * 64;
+            int row = p.oob_row;
+            if (key0 < k_hi) {
+              const int page = pt[key0 / 64];
+              if (page >= 0 && page < p.num_pages)
+                row = ((p.layer * p.num_pages + page) * p.nkv + g) * 64;
+              else
+                flag(p.status, ISD_DEV_BAD_PAGE);
+            }
+            for (int hh = 0; hh < 2; ++hh) {
+              // K as [dim half][page][64 keys][64 dims]: the 128 keys of a
+              // dim half are one K-major operand; V as [page][dim half]:
+              // each page is 16 keys per MMA k-step, dim halves LBO apart.
+              tma_load_2d(ks + hh * 2 * kTcHalf + j * kTcHalf, &kmap, &full[st], hh * 64, row);
+              tma_load_2d(vs + j * 2 * kTcHalf + hh * kTcHalf, &vmap, &full[st], hh * 64, row);
+            }
+          }
+        }
+      }
+      if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
+      // copies in flight land before the CTA exits
+      for (int j = max(0, tc - p.stages); j < tc; ++j)
+        if (!mbar_wait(&full[j % p.stages], (j / p.stages) & 1)) break;
+      if (q_issued > 0) mbar_wait(&q_full[(q_issued - 1) & 1], ((q_issued - 1) >> 1) & 1);
+    }
+  } else if (warp == kTcSoftWarps + 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && fits) {
+      const uint32_t idesc_s = idesc_bf16(128, NP);
+      const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15);   // A (V^T) MN-major
+      const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(qs), p_a = smem_u32(ps);
+      int tc = 0, it = 0;
+      int pend = -1, pend_st = 0;   // tile whose PV is not yet issued
+      bool ok = true;
+      auto issue_pv = [&](int j, int st) -> bool {
+        if (!mbar_wait(p_full, j & 1)) return false;
+        if (!mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + 2 * NP + (j & 1) * NP;
+        const uint32_t va = ring_a + st * kTcStage + kTcStage / 2;
+#pragma unroll
+        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+          const uint64_t a = sw128_desc_mn(va + (kk >> 2) * 2 * kTcHalf + (kk & 3) * 2048, kTcHalf);
+          const uint64_t bdesc = sw128_desc(p_a + (kk >> 2) * (NP * 128) + (kk & 3) * 32);
+          umma_bf16(d, a, bdesc, idesc_o, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&o_full[j & 1]);
+        umma_commit(&empty[st]);
+        umma_commit(p_empty);
+        return true;
+      };
+      TcRange rg = tc_range(p, base);
+      TcSeg sg;
+      for (; ok && tc_next(p, base, rg, sg); ++it) {
+        const int n_tiles = sg.len;
+        const int qb = it & 1;
+        if (!mbar_wait(&q_full[qb], (it >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < n_tiles; ++t, ++tc) {
+          const int st = tc % p.stages;
+          if (!mbar_wait(&full[st], (tc / p.stages) & 1) ||
+              !mbar_wait(&s_empty[tc & 1], ((tc >> 1) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (tc & 1) * NP;
+          const uint32_t ka = ring_a + st * kTcStage;
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint64_t a = sw128_desc(ka + (kk >> 2) * 2 * kTcHalf + (kk & 3) * 32);
+            const uint64_t bdesc = sw128_desc(q_a + qb * kTcQBuf + (kk >> 2) * (NP * 128) + (kk & 3) * 32);
+            umma_bf16(d, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[tc & 1]);
+          if (pend >= 0 && !issue_pv(pend, pend_st)) {
+            ok = false;
+            break;
+          }
+          pend = tc;
+          pend_st = st;
+        }
+        if (!ok) break;
+        umma_commit(&q_empty[qb]);   // this item's S MMAs are the last readers of Q
+      }
+      if (ok && pend >= 0 && !issue_pv(pend, pend_st)) ok = false;
+      if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
+      // every MMA has finished before tensor memory is freed
+      umma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+  } else if (fits) {
+    // -------------------------------------------- softmax / accumulate warps
+    // warp w: TMEM lane quadrant w % 4 (keys of S, dims of O) and query
+    // rows r0 .. r0 + 15 (TMEM columns), r0 = 16 * (w / 4)
+    const int quad = warp & 3;
+    const int r0 = (warp >> 2) * NR;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const int kl = quad * 32 + lane;           // key within the tile; dim for O
+    // P^T store: key half kh, key kk in the half (128-byte swizzle by row)
+    const int kh = kl >> 6, kk = kl & 63;
+    uint8_t* p_col = ps + kh * (NP * 128) + (kk & 7) * 2;
+    float o[NR];
+    float ls[NR];
+    int tc = 0;
+    bool fine = true;
+    TcRange rg = tc_range(p, base);
+    TcSeg sg;
+    while (tc_next(p, base, rg, sg)) {
+      const int b = sg.b;
+      const int k_lo = sg.t0 * kTcKeys;
+      const int k_hi = min(kend[b], k_lo + sg.len * kTcKeys);
+      const int n_tiles = sg.len;
+      if (warp == 0) {
+        const int pr = lane < p.RG ? p.row_pos[b * p.R + lane / p.G] : -1;
+        pos_sh[lane] = pr;
+        m_sh[lane] = -INFINITY;
+        int mn = lane < p.RG ? pr : INT_MAX;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o2));
+        if (lane == 0) *minpos_sh = mn;
+      }
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        o[r] = 0.f;
+        ls[r] = 0.f;
+      }
+      named_bar_sync(2, kSoftThreads);
+      const int minpos = *minpos_sh;
+      for (int t = 0; t < n_tiles; ++t, ++tc) {
+        const int sb = tc & 1;
+        // ---- S tile -> registers
+        fine = fine && mbar_wait(&s_full[sb], (tc >> 1) & 1);
+        tc_fence_after();
+        float x[NR];
+        {
+          uint32_t r16[16];
+          tmem_ld_32x32_x16(lane_base + sb * NP + r0, r16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int r = 0; r < NR; ++r) x[r] = __uint_as_float(r16[r]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        const int key = k_lo + t * kTcKeys + kl;
+        const int last = k_lo + t * kTcKeys + kTcKeys - 1;
+        if (last < k_hi && last <= minpos) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r) x[r] *= p.scale_log2;
+        } else {
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            x[r] = (key < k_hi && key <= pos_sh[r0 + r]) ? x[r] * p.scale_log2 : -INFINITY;
+        }
+        // ---- row max over the tile's 128 keys
+        {
+          float xm[NR];
+#pragma unroll
+          for (int r = 0; r < NR; ++r) xm[r] = x[r];
+          const float mx = lane_reduce16<true>(xm, lane);
+          if ((lane & 1) == 0) red[quad * NP + r0 + (lane >> 1)] = mx;
+        }
+        // all softmax warps agree on going on (they share named barriers)
+        if (!named_bar_and(2, kSoftThreads, fine)) {
+          fine = false;
+          break;
+        }
+        if (warp == 0) {
+          const float m_old = m_sh[lane];
+          const float mt = fmaxf(fmaxf(red[lane], red[NP + lane]), fmaxf(red[2 * NP + lane], red[3 * NP + lane]));
+          const float m_new = fmaxf(m_old, mt);
+          alpha_sh[sb * NP + lane] = m_new == -INFINITY ? 1.f : ex2(m_old - m_new);
+          m_sh[lane] = m_new;
+        }
+        named_bar_sync(2, kSoftThreads);
+        // ---- P = 2^(x - m), partial row sums, P^T to shared memory
+        // (all shared-memory reads first: a store between them would
+        // serialise every row on the possible aliasing)
+#pragma unroll
+        for (int r = 0; r < NR; r += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(m_sh + r0 + r);
+          const float4 a4 = *reinterpret_cast<const float4*>(alpha_sh + sb * NP + r0 + r);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+          const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float e = mm[i] == -INFINITY ? 0.f : ex2(x[r + i] - mm[i]);
+            ls[r + i] = ls[r + i] * aa[i] + e;
+            x[r + i] = e;
+          }
+        }
+        fine = fine && mbar_wait(p_empty, (tc & 1) ^ 1);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const int row = r0 + r;
+          *reinterpret_cast<__nv_bfloat16*>(p_col + row * 128 + (((kk >> 3) ^ (row & 7)) << 4)) =
+              __float2bfloat16_rn(x[r]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        // ---- O += previous tile's O_t (its PV ran while this tile's S did)
+        if (t > 0) {
+          const int j = tc - 1;
+          fine = fine && mbar_wait(&o_full[j & 1], (j >> 1) & 1);
+          tc_fence_after();
+          uint32_t r16[16];
+          tmem_ld_32x32_x16(lane_base + 2 * NP + (j & 1) * NP + r0, r16);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[j & 1]);
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] + __uint_as_float(r16[r]);
+        }
+      }
+      if (!fine) break;
+      if (n_tiles > 0) {
+        const int j = tc - 1;
+        fine = mbar_wait(&o_full[j & 1], (j >> 1) & 1);
+        tc_fence_after();
+        uint32_t r16[16];
+        tmem_ld_32x32_x16(lane_base + 2 * NP + (j & 1) * NP + r0, r16);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[j & 1]);
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+          o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] + __uint_as_float(r16[r]);
+      }
+      // ---- row sums over the 128 key lanes, then the partial output
+      {
+        const float sm = lane_reduce16<false>(ls, lane);
+        if ((lane & 1) == 0) red[quad * NP + r0 + (lane >> 1)] = sm;
+      }
+      if (!named_bar_and(2, kSoftThreads, fine)) {
+        fine = false;
+        break;
+      }
+      if (warp == 0) {
+        const float L = (red[lane] + red[NP + lane]) + (red[2 * NP + lane] + red[3 * NP + lane]);
+        l_sh[lane] = L;
+        if (sg.slot >= 0)
+          p.part_ml[static_cast<int64_t>(sg.slot) * NP + lane] = make_float2(m_sh[lane], L);
+        else if (lane == 0)
+          flag(p.status, ISD_DEV_BAD_STATE);
+      }
+      named_bar_sync(2, kSoftThreads);
+      if (sg.slot >= 0) {
+        float* po = p.part_o + (static_cast<int64_t>(sg.slot) * NP + r0) * 128 + kl;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const float L = l_sh[r0 + r];
+          po[r * 128] = L > 0.f ? o[r] / L : 0.f;
+        }
+      }
+      named_bar_sync(2, kSoftThreads);   // row state is rewritten by the next segment
+    }
+    if (!fine && lane == 0) flag(p.status, ISD_DEV_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 4 * NP);
+  }
+}
+
 // out[b*R + r][(g*G + h)*HD + d] = sum over the request's key splits,
 // weighted by each split's softmax mass: per-(row, split) weights once in
 // shared memory, then float4 accumulation.
@@ -505,15 +1030,98 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p, _
   }
 }
 
+// Combine for the tcgen05 kernel's balanced ranges: (request b, KV head g)
+// has parts from CTAs c(first tile) .. c(last tile), in slots
+// (b * nkv + g) * max_parts + 0 .. parts - 1. Same merge as above.
+__global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p, int C_grid,
+                                                              __nv_bfloat16* out) {
+  constexpr int HD = 128;
+  const int g = blockIdx.x, b = blockIdx.y;
+  __shared__ float w[kTcNP][kMaxSplits];
+  const int* base = p.item_base;
+  const int64_t T = static_cast<int64_t>(p.nkv) * base[p.B];
+  const int nt = base[b + 1] - base[b];
+  int parts = 0;
+  if (nt > 0 && T > 0) {
+    const int C = static_cast<int>(i64max(1, i64min(C_grid, T / p.min_tiles)));
+    const int64_t first = static_cast<int64_t>(base[b]) * p.nkv + static_cast<int64_t>(g) * nt;
+    parts = tc_cta_of(first + nt - 1, T, C) - tc_cta_of(first, T, C) + 1;
+  }
+  if (parts > p.max_parts || parts > kMaxSplits) {
+    if (threadIdx.x == 0) flag(p.status, ISD_DEV_BAD_STATE);
+    return;
+  }
+  const int64_t slot0 = static_cast<int64_t>(b * p.nkv + g) * p.max_parts;
+  for (int qi = threadIdx.x; qi < p.RG; qi += blockDim.x) {
+    float M = -INFINITY;
+    for (int s = 0; s < parts; ++s) M = fmaxf(M, p.part_ml[(slot0 + s) * kTcNP + qi].x);
+    const float Rm = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    for (int s = 0; s < parts; ++s) {
+      const float2 ml = p.part_ml[(slot0 + s) * kTcNP + qi];
+      const float ws = ml.y * exp2f(ml.x - Rm);
+      w[qi][s] = ws;
+      L += ws;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int s = 0; s < parts; ++s) w[qi][s] *= inv;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.RG * (HD / 4); i += blockDim.x) {
+    const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < parts; ++s) {
+      const float ws = w[qi][s];
+      const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * kTcNP + qi) * HD + d);
+      acc.x += ws * v.x;
+      acc.y += ws * v.y;
+      acc.z += ws * v.z;
+      acc.w += ws * v.w;
+    }
+    const int r = qi / p.G, h = qi % p.G;
+    __align__(8) __nv_bfloat16 o4[4] = {__float2bfloat16_rn(acc.x), __float2bfloat16_rn(acc.y),
+                                        __float2bfloat16_rn(acc.z), __float2bfloat16_rn(acc.w)};
+    *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b * p.R + r) * p.nq + g * p.G + h) * HD + d) =
+        *reinterpret_cast<const uint2*>(o4);
+  }
+}
+
 struct Derived {
   int RG, MT, NG, split_keys, max_splits, stages, max_items;
+  int min_tiles = 1;
+  bool tc;        // the tcgen05 kernel serves this shape
   size_t smem;
 };
+
+// Shared memory of the tcgen05 kernel for a batch of B requests.
+size_t tc_smem(int stages, int B) {
+  return 1024 + static_cast<size_t>(stages) * kTcStage + 2 * kTcQBuf + kTcPBuf + kTcMisc + kTcBars +
+         16 + (2 * static_cast<size_t>(B) + 1) * sizeof(int);
+}
 
 Derived derive(const AttnShape& s) {
   Derived d;
   const int G = s.n_q_heads / s.n_kv_heads;
   d.RG = s.rows_per_req * G;
+  d.tc = s.head_dim == 128 && s.page_size == 64 && d.RG <= kTcNP && tc_smem(2, s.batch) <= 232448;
+  if (d.tc) {
+    // one CTA per SM, equal contiguous tile ranges of at least kTcMinTiles
+    // tiles; a (request, head) run of n tiles then spans at most
+    // ceil(n / kTcMinTiles) + 1 CTAs
+    const int64_t max_tiles =
+        (static_cast<int64_t>(s.max_pages_per_req) * s.page_size + kTcKeys - 1) / kTcKeys;
+    d.split_keys = kTcKeys;
+    d.min_tiles = static_cast<int>(
+        std::max<int64_t>(kTcMinTiles, (max_tiles + kMaxSplits - 2) / (kMaxSplits - 1)));
+    d.max_splits = static_cast<int>((max_tiles + d.min_tiles - 1) / d.min_tiles + 1);
+    d.max_items = s.batch * s.n_kv_heads * d.max_splits;
+    d.MT = kTcNP / 16;
+    d.NG = 1;
+    d.stages = 4;
+    while (d.stages > 2 && tc_smem(d.stages, s.batch) > 232448) --d.stages;
+    d.smem = tc_smem(d.stages, s.batch);
+    return d;
+  }
   d.MT = (d.RG + 15) / 16;
   if (d.MT == 3) d.MT = 4;
   d.NG = kConsumerWarps / d.MT;               // consumer warps = MT query tiles x NG groups
@@ -625,6 +1233,24 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
   const dim3 grid(sms * kCtasPerSm);
+  if (d.tc) {
+    static bool tc_attr = false;
+    if (!tc_attr) {
+      const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel),
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+      if (e != cudaSuccess) return e;
+      tc_attr = true;
+    }
+    p.max_parts = d.max_splits;
+    p.min_tiles = d.min_tiles;
+    attn_tc_kernel<<<sms, kTcThreads, d.smem, stream>>>(k_map, v_map, qmap, p);
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess) return le;   // the combine reads what this kernel writes
+    if (between) cudaEventRecord(between, stream);
+    attn_combine_tc_kernel<<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
+    if (launches) *launches += 2;
+    return cudaGetLastError();
+  }
   if (s.head_dim == 128) {
     if (d.NG == 4)
       attn_persistent_kernel<128, 4><<<grid, kThreads, d.smem, stream>>>(k_map, v_map, qmap, p);

@@ -468,6 +468,11 @@ int alloc_workspace(isd_ctx* c) {
   a.max_pages_per_req = (g.max_position + g.page_size - 1) / g.page_size;
   a.n_layers = 1;
   c->attn_ws_bytes = isd::attention_workspace_bytes(a);
+  // decode blocks of up to 32 query rows per KV head take the tcgen05 path,
+  // whose work split differs: size for both
+  isd::AttnShape a_dec = a;
+  a_dec.rows_per_req = std::max(1, 32 / (g.n_q_heads / g.n_kv_heads));
+  c->attn_ws_bytes = std::max(c->attn_ws_bytes, isd::attention_workspace_bytes(a_dec));
   const int maxN = 8;
   c->acc_ws_bytes = isd::accept_workspace_bytes(g.max_batch, maxN, g.vocab);
   // stream-K: one slot per SM of fp32 partials of up to 512 tokens x 128 rows

@@ -132,6 +132,8 @@ def _oracle_attention(q, kp, vp, table, pos, lens, R, P, b):
     ((128, 32, 8, 64), [130, 257], 16, False),              # prefill chunk: 64 query rows
     ((128, 8, 1, 64), [40, 300], 8, True),                  # 8:1 grouping, a row with no keys
     ((128, 16, 16, 32), [90, 33], 5, False),                # multi-head (1:1), page 32
+    ((128, 8, 1, 64), [200, 5], 4, True),                   # 8:1, 32 rows, a row with no keys
+    ((128, 16, 4, 64), [0, 127, 128, 129, 1000], 5, False),  # tile and page edges, 20 rows
 ])
 def test_paged_attention_matches_oracle(cuda_lib, shape_args, lens, R, pad):
     hd, nq, nkv, P = shape_args
