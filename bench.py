@@ -20,10 +20,11 @@ step); time is the max over ranks, value the sum of all ranks' tokens.
 --impl reference times the CPU oracle (fp64 numpy) on a bounded sample of
 the same workload on rank 0 and extrapolates to the same metric.
 
---component gemm:MxNxKxS | attention:WORKLOAD times one kernel of the step
-through its C-ABI component entry (isd_gemm_bf16: Y = X W^T with M tokens,
-N outputs, K inputs, S K-splits; isd_paged_attention on the workload's
-block rows and KV lengths), one launch per step with an L2 flush between,
+--component gemm:MxNxKxS | gemm1:MxNxK | attention:WORKLOAD times one kernel
+of the step through its C-ABI component entry (isd_gemm_bf16: Y = X W^T with
+M tokens, N outputs, K inputs, S K-splits; isd_gemm_bf16_single: the same as
+one slice, stream-K when the tiles overfill a wave; isd_paged_attention on
+the workload's block rows and KV lengths), one launch per step with an L2 flush between,
 and prints its duration and throughput. It is the command the kernel
 profiles are taken with.
 """
@@ -340,6 +341,13 @@ def run_cuda(args, ws, rank, local):
     return result
 
 
+# DRAM bytes (read + write) per byte of K + V of the tcgen05 attention kernel,
+# from the ncu capture summarised in profiles/attn_tc_kernel_qwen3_8b_b64.md
+# (603.7 MB for a launch over 580.4 MB of K + V at the same workload shape);
+# the roofline's `traffic` scales it to this run's launch.
+ATTN_DRAM_PER_KV_BYTE = 603.7 / 580.4
+
+
 def roofline_entry(prof, shape, B, N, lens, steps, peaks):
     """Roofline of the kernel class with the largest device time."""
     if not prof:
@@ -364,8 +372,13 @@ def roofline_entry(prof, shape, B, N, lens, steps, peaks):
         kv = sum(int(L) + R for L in lens) * shape.kv_dim * 2 * 2   # one layer's K+V
         achieved = kv / avg_s / 1e9
         peak = peaks["hbm"]
+        traffic = None
+        if top == "attention_split" and shape.head_dim == 128 and shape.page_size == 64:
+            traffic = ATTN_DRAM_PER_KV_BYTE * kv   # bytes per launch (scaled ncu capture)
         return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "peak_kind": f"{peaks['source']} HBM copy",
+                "frac": achieved / peak, "traffic": traffic,
+                "traffic_note": "ncu dram read+write of one capture, scaled by K+V bytes",
+                "peak_kind": f"{peaks['source']} HBM copy",
                 "avg_launch_ms": avg_s * 1e3, "launches": cnt}
     return {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s",
             "frac": None, "traffic": None, "avg_launch_ms": avg_s * 1e3, "launches": cnt}
@@ -472,6 +485,16 @@ def run_component(args):
             Bd.gemm_bf16(w, x, split, status=st)
         work = {"flops": 2.0 * m * n * k,
                 "bytes": 2.0 * n * k + 2.0 * m * k + 4.0 * split * m * n}
+    elif kind == "gemm1":
+        # one output slice, planned like the step's gate/up and LM head (stream-K)
+        m, n, k = (int(v) for v in spec.split("x"))
+        w = (torch.randn(n, k, device="cuda") * 0.02).to(torch.bfloat16)
+        x = torch.randn(m, k, device="cuda").to(torch.bfloat16)
+        wsp = Bd.gemm_workspace(m, n, k)
+
+        def fn():
+            Bd.gemm_bf16_single(w, x, wsp, status=st)
+        work = {"flops": 2.0 * m * n * k, "bytes": 2.0 * n * k + 2.0 * m * k + 4.0 * m * n}
     elif kind == "attention":
         wl = WORKLOADS[spec]
         shape, Bn, N = wl["shape"], wl["batch"], wl["stride"]
@@ -526,7 +549,7 @@ def main():
     ap.add_argument("--workload", default="qwen3_8b_b64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--component", default=None,
-                    help="gemm:MxNxKxS or attention:WORKLOAD (one kernel, for profiling)")
+                    help="gemm:MxNxKxS, gemm1:MxNxK or attention:WORKLOAD (one kernel, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
