@@ -349,13 +349,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] += __ldcg(pp + j * kTileM);
         }
+        // a chunk whose 32 tokens all exist needs no per-store bounds check
+        const bool full_chunk = c * 32 + 32 <= p.n_pad && t0 + 32 <= p.m;
         if (p.epi == kEpiF32) {
           const int f = mt * kTileM + quad * 32 + lane;
-          float* outp = p.out + split * p.split_stride + f;
+          float* rowp = p.out + split * p.split_stride + static_cast<int64_t>(t0) * p.n_out + f;
+          if (full_chunk) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < p.n_pad && t0 + j < p.m)
-              outp[static_cast<int64_t>(t0 + j) * p.n_out] = v[j];
+            for (int j = 0; j < 32; ++j) {
+              *rowp = v[j];
+              rowp += p.n_out;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c * 32 + j < p.n_pad && t0 + j < p.m) *rowp = v[j];
+              rowp += p.n_out;
+            }
+          }
         } else {
           // Each quadrant's 32 TMEM lanes hold 16 gate rows then the 16 up
           // rows of the same features (see the gate/up layout in isd.h). A
@@ -364,6 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int half_n = p.n_out / 2;
           const bool hi = lane >= 16;
           const int f = mt * 64 + quad * 16 + (lane & 15);
+          __nv_bfloat16* rowp =
+              p.out_act + static_cast<int64_t>(t0 + (hi ? 1 : 0)) * half_n + f;
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
             const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
@@ -371,9 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float g = hi ? x_j1 : v[j];
             const float u = hi ? v[j + 1] : x_j;
             const int jj = j + (hi ? 1 : 0);
-            if (c * 32 + jj < p.n_pad && t0 + jj < p.m)
-              p.out_act[static_cast<int64_t>(t0 + jj) * half_n + f] =
-                  __float2bfloat16_rn(silu_mul(g, u));
+            if (full_chunk || (c * 32 + jj < p.n_pad && t0 + jj < p.m))
+              *rowp = __float2bfloat16_rn(silu_mul(g, u));
+            rowp += 2 * half_n;
           }
         }
       }
