@@ -113,7 +113,14 @@ __global__ void __launch_bounds__(256)
 }
 
 // x[row] += sum_s part[s][row] (fixed order); hn[row] = bf16(RMSNorm(x[row]) * w).
-__global__ void __launch_bounds__(256)
+// Each thread holds up to kResIters float4 of the row, so every split's loads
+// are in flight together; the sum order (x, then splits ascending, then the
+// MASK-row delta) is fixed.
+constexpr int kResThreads = 256;
+constexpr int kResIters = 8;        // hidden <= 8192
+constexpr int kResMaxSplits = 8;
+
+__global__ void __launch_bounds__(kResThreads)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
                          const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
                          const float* delta, float delta_scale, const int32_t* row_flags) {
@@ -123,36 +130,57 @@ __global__ void __launch_bounds__(256)
   const float* pr = part + static_cast<int64_t>(row) * hidden;
   const float* dr = (delta && (row_flags[row] & kRowMask)) ? delta + static_cast<int64_t>(row) * hidden
                                                           : nullptr;
-  float ss = 0.f;
-  for (int i = threadIdx.x * 4; i < hidden; i += 256 * 4) {
-    float4 v = *reinterpret_cast<const float4*>(xr + i);
-    for (int s = 0; s < splits; ++s) {
-      const float4 d = *reinterpret_cast<const float4*>(pr + s * split_stride + i);
-      v.x += d.x;
-      v.y += d.y;
-      v.z += d.z;
-      v.w += d.w;
-    }
-    if (dr) {   // gated-LoRA delta: MASK rows only
-      const float4 d = *reinterpret_cast<const float4*>(dr + i);
-      v.x += delta_scale * d.x;
-      v.y += delta_scale * d.y;
-      v.z += delta_scale * d.z;
-      v.w += delta_scale * d.w;
-    }
-    *reinterpret_cast<float4*>(xr + i) = v;
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  float4 v[kResIters];
+#pragma unroll
+  for (int it = 0; it < kResIters; ++it) {
+    const int i = (it * kResThreads + threadIdx.x) * 4;
+    v[it] = i < hidden ? *reinterpret_cast<const float4*>(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const float tot = block_sum<256>(ss, red);
+#pragma unroll
+  for (int s = 0; s < kResMaxSplits; ++s) {
+    if (s < splits) {
+#pragma unroll
+      for (int it = 0; it < kResIters; ++it) {
+        const int i = (it * kResThreads + threadIdx.x) * 4;
+        if (i < hidden) {
+          const float4 d = *reinterpret_cast<const float4*>(pr + s * split_stride + i);
+          v[it].x += d.x;
+          v[it].y += d.y;
+          v[it].z += d.z;
+          v[it].w += d.w;
+        }
+      }
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int it = 0; it < kResIters; ++it) {
+    const int i = (it * kResThreads + threadIdx.x) * 4;
+    if (i < hidden) {
+      if (dr) {   // gated-LoRA delta: MASK rows only
+        const float4 d = *reinterpret_cast<const float4*>(dr + i);
+        v[it].x += delta_scale * d.x;
+        v[it].y += delta_scale * d.y;
+        v[it].z += delta_scale * d.z;
+        v[it].w += delta_scale * d.w;
+      }
+      *reinterpret_cast<float4*>(xr + i) = v[it];
+      ss += v[it].x * v[it].x + v[it].y * v[it].y + v[it].z * v[it].z + v[it].w * v[it].w;
+    }
+  }
+  const float tot = block_sum<kResThreads>(ss, red);
   const float rstd = rsqrtf(tot / hidden + eps);
   __nv_bfloat16* hr = hn + static_cast<int64_t>(row) * hidden;
-  for (int i = threadIdx.x * 4; i < hidden; i += 256 * 4) {
-    const float4 v = *reinterpret_cast<const float4*>(xr + i);
-    __align__(8) __nv_bfloat16 o4[4] = {
-        __float2bfloat16_rn(v.x * rstd * norm_w[i]), __float2bfloat16_rn(v.y * rstd * norm_w[i + 1]),
-        __float2bfloat16_rn(v.z * rstd * norm_w[i + 2]),
-        __float2bfloat16_rn(v.w * rstd * norm_w[i + 3])};
-    *reinterpret_cast<uint2*>(hr + i) = *reinterpret_cast<const uint2*>(o4);
+#pragma unroll
+  for (int it = 0; it < kResIters; ++it) {
+    const int i = (it * kResThreads + threadIdx.x) * 4;
+    if (i < hidden) {
+      const float4 w = *reinterpret_cast<const float4*>(norm_w + i);
+      __align__(8) __nv_bfloat16 o4[4] = {
+          __float2bfloat16_rn(v[it].x * rstd * w.x), __float2bfloat16_rn(v[it].y * rstd * w.y),
+          __float2bfloat16_rn(v[it].z * rstd * w.z), __float2bfloat16_rn(v[it].w * rstd * w.w)};
+      *reinterpret_cast<uint2*>(hr + i) = *reinterpret_cast<const uint2*>(o4);
+    }
   }
 }
 
@@ -282,7 +310,9 @@ cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows
                                  const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
                                  cudaStream_t stream, const float* delta, float delta_scale,
                                  const int32_t* row_flags) {
-  residual_norm_kernel<<<rows, 256, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
+  if (hidden % 4 || hidden > kResThreads * 4 * kResIters || splits < 0 || splits > kResMaxSplits)
+    return cudaErrorInvalidValue;
+  residual_norm_kernel<<<rows, kResThreads, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
                                                  hidden, norm_w, eps, x, hn, delta, delta_scale,
                                                  row_flags);
   return cudaGetLastError();
