@@ -13,6 +13,10 @@ isd_prefill before timing. Accept-test uniforms are acceptance-controlled
 committed tokens per forward match a trained model's regime; the run with
 natural uniforms is reported beside it.
 
+The K timed steps are captured once into a CUDA graph (before timing) and
+replayed once inside the timed region; the same number of steps launched
+one by one is reported as "eager" (--no-graph times those instead).
+
 Multi-GPU (torchrun): the method shards by request, so every rank runs an
 independent replica with its own batch (weak scaling, no collective in the
 step); time is the max over ranks, value the sum of all ranks' tokens.
@@ -156,7 +160,7 @@ def run_cuda(args, ws, rank, local):
     shape, B, N = wl["shape"], wl["batch"], wl["stride"]
     R, P, V = 2 * N - 1, shape.page_size, shape.vocab
     seed = 1000 + rank
-    total_steps = args.warmup + 5 * args.steps + 4   # every step run below grows the sequences
+    total_steps = args.warmup + 6 * args.steps + 4   # every step run below grows the sequences
     lens = synth.prompt_lengths(B, wl["len_lo"], wl["len_hi"], seed)
     prompts = synth.prompts(shape, lens, seed)
     maxp = -(-(int(lens.max()) + total_steps * N + R + 1) // P) + 1
@@ -204,26 +208,57 @@ def run_cuda(args, ws, rank, local):
         if ws > 1:
             dist.barrier()
 
-    # ---- timed region: K steps, inputs resident in HBM
+    # ---- timed region: K steps, inputs resident in HBM. By default the K
+    # steps are one CUDA graph (captured here, before timing) replayed once;
+    # the same K steps launched one by one are timed next as "eager".
     stream = torch.cuda.current_stream()
+    graph = None
+    if not args.no_graph:
+        graph = Bd.StepGraph(model, kv, st, args.steps, flags)
+        torch.cuda.synchronize()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         torch.cuda.nvtx.range_push("isd_timed")
-        e_start.record(stream)
-        for i in range(args.steps):
-            one(unif_d[step_i]); step_i += 1
-            hist[i].copy_(st.accepted)
-        e_stop.record(stream)
+        if graph is not None:
+            u_g = unif_d[step_i:step_i + args.steps].clone()
+            step_i += args.steps
+            e_start.record(stream)
+            graph.replay(u_g)
+            e_stop.record(stream)
+        else:
+            e_start.record(stream)
+            for i in range(args.steps):
+                one(unif_d[step_i]); step_i += 1
+                hist[i].copy_(st.accepted)
+            e_stop.record(stream)
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
     barrier()
     ms = e_start.elapsed_time(e_stop)
+    if graph is not None:
+        hist.copy_(graph.accepted)
+        del graph
     launches_per_step = model.launches()
     committed = int((hist.long() + 1).sum().item())
     if int(st.status.item()) != 0:
         raise RuntimeError(f"step status {int(st.status.item())}")
+
+    # ---- the same number of steps launched one by one
+    eager_ms, eager_committed = None, 0
+    if not args.no_graph:
+        h_start, h_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eager_hist = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
+        torch.cuda.synchronize()
+        h_start.record(stream)
+        for i in range(args.steps):
+            one(unif_d[step_i]); step_i += 1
+            eager_hist[i].copy_(st.accepted)
+        h_stop.record(stream)
+        torch.cuda.synchronize()
+        eager_ms = h_start.elapsed_time(h_stop)
+        eager_committed = int((eager_hist.long() + 1).sum().item())
 
     # ---- profiled region: same steps with per-kernel-class CUDA events
     model.profile(True)
@@ -279,13 +314,14 @@ def run_cuda(args, ws, rank, local):
     e2e_committed = int((pin_acc.long() + 1).sum().item())
 
     # ---- reduce over ranks: max time, summed tokens
-    vals = torch.tensor([ms, e2e_ms, nat_ms], device="cuda", dtype=torch.float64)
-    toks = torch.tensor([committed, e2e_committed, nat_committed], device="cuda", dtype=torch.float64)
+    vals = torch.tensor([ms, e2e_ms, nat_ms, eager_ms or 0.0], device="cuda", dtype=torch.float64)
+    toks = torch.tensor([committed, e2e_committed, nat_committed, eager_committed], device="cuda",
+                        dtype=torch.float64)
     if ws > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
         dist.all_reduce(toks, op=dist.ReduceOp.SUM)
-    ms, e2e_ms, nat_ms = vals.tolist()
-    committed, e2e_committed, nat_committed = toks.tolist()
+    ms, e2e_ms, nat_ms, eager_ms_all = vals.tolist()
+    committed, e2e_committed, nat_committed, eager_committed = toks.tolist()
 
     result = None
     if rank == 0:
@@ -324,6 +360,12 @@ def run_cuda(args, ws, rank, local):
             "risd_overhead_alpha": (ms / base_ms) if base_ms else None,
             "natural_uniforms": {"value": nat_committed / (nat_ms * 1e-3), "unit": "tokens/s",
                                  "tokens_per_forward": nat_committed / (args.steps * B * ws)},
+            "timed_as": "one CUDA graph of the K steps, replayed once" if eager_ms is not None
+            else "K steps launched one by one",
+            "eager": None if eager_ms is None else {
+                "value": eager_committed / (eager_ms_all * 1e-3), "unit": "tokens/s",
+                "ms_per_step": eager_ms_all / args.steps,
+                "note": "the same number of steps launched one by one"},
             "prefill_s": t_prefill, "setup_s": t_setup,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
@@ -548,6 +590,8 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="qwen3_8b_b64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the steps launched one by one instead of replaying a CUDA graph")
     ap.add_argument("--component", default=None,
                     help="gemm:MxNxKxS, gemm1:MxNxK or attention:WORKLOAD (one kernel, for profiling)")
     args = ap.parse_args()

@@ -331,6 +331,42 @@ def step(model: Model, kv: KVCache, st: StepState, uniforms, flags: int = 0, log
                          _stream()))
 
 
+class StepGraph:
+    """`steps` consecutive isd_step calls captured once into a CUDA graph.
+
+    The graph holds the launches of every kernel of the steps with their
+    arguments fixed: the model, cache and state objects given here, and a
+    static uniforms buffer `u` of shape [steps, B, 2N-1] that replay() fills.
+    Replaying runs the same device work as calling step() `steps` times with
+    those uniforms, without host launch overhead. Run at least one eager step
+    first (the library sets kernel attributes on first use) and keep every
+    object alive while the graph is used.
+    """
+
+    def __init__(self, model: Model, kv: KVCache, st: StepState, steps: int, flags: int = 0):
+        import torch
+        self.steps = steps
+        R = 2 * st.N - 1
+        self.u = torch.zeros(steps, st.B, R, device=st.seq_len.device, dtype=torch.float32)
+        # per-step acceptance counts, recorded inside the graph
+        self.accepted = torch.zeros(steps, st.B, device=st.seq_len.device, dtype=torch.int32)
+        self.graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(self.graph, stream=side):
+                for i in range(steps):
+                    step(model, kv, st, self.u[i], flags)
+                    self.accepted[i].copy_(st.accepted)
+        torch.cuda.current_stream().wait_stream(side)
+
+    def replay(self, uniforms=None):
+        """Run the captured steps (uniforms: [steps, B, 2N-1] float32 device, optional)."""
+        if uniforms is not None:
+            self.u.copy_(uniforms)
+        self.graph.replay()
+
+
 def prefill(model: Model, kv: KVCache, st: StepState, prompts: List[np.ndarray]):
     """isd_prefill of one prompt per request (host token lists)."""
     import torch
