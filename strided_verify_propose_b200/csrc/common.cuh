@@ -301,7 +301,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 
 // SiLU(g) * u with the fast exponential and division intrinsics. Every
 // kernel that forms the SwiGLU product uses this one expression, so the
-// fused GEMM epilogue and the separate LoRA path give the same bits.
+// base gate/up epilogue and the gated-LoRA one give verify rows the same bits.
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g, 1.0f + __expf(-g)) * u;
 }

@@ -165,7 +165,6 @@ struct isd_ctx {
   std::vector<LoraLayer> lora;
   float* lora_xa_part = nullptr;         // [max_splits][max_rows][3r]
   __nv_bfloat16* lora_xa = nullptr;      // [max_rows][3r]
-  float* lora_delta = nullptr;           // [max_rows][max(qkv_dim, hidden, 2 I)]
   float* lora_gu = nullptr;              // [max_rows][2 I] base gate/up in fp32
 
   // per-kernel-class event timing (isd_profile_enable)
@@ -185,7 +184,7 @@ enum ProfClass {
 const char* kProfNames[ISD_PROF_CLASSES] = {
     "assemble", "embed_norm", "gemm_qkv", "qkv_reduce_rope_kvwrite", "attention_split",
     "attention_combine", "gemm_o", "residual_norm", "gemm_gate_up_silu", "gemm_down",
-    "gemm_lm_head", "accept_stats", "accept_decide", "bookkeep", "lora_delta", "unused"};
+    "gemm_lm_head", "accept_stats", "accept_decide", "bookkeep", "lora", "unused"};
 
 cudaEvent_t prof_event(isd_ctx* c) {
   if (!c->prof_on) return nullptr;
@@ -238,10 +237,19 @@ const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k, bool single) {
 // One projection: X [m][k] (bf16 workspace buffer) times W^T. kEpiF32
 // writes `splits` partial slices of m x n floats, so the output must hold
 // out_elems >= splits * m * n; max_splits = 1 asks for the plain product.
+// A second operand pair for the last split of a split-K GEMM (the gated
+// adapter's B with xa, see lora_xa): W2 [n][k2], X2 [m][k2].
+struct AugSpec {
+  const CUtensorMap* tw2;
+  const __nv_bfloat16* x2;
+  int k2;
+};
+
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
-         __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st) {
-  const GemmPlan& plan = plan_for(c, m, n, k, epi == isd::kEpiSiluMul || max_splits == 1);
+         __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
+         const isd::GemmLoraEpilogue* lora = nullptr, const AugSpec* aug = nullptr) {
+  const GemmPlan& plan = plan_for(c, m, n, k, epi != isd::kEpiF32 || max_splits == 1);
   if (plan.n_pad == 0) return fail(ISD_E_UNSUPPORTED, "no GEMM plan");
   if (isd::gemm_streamk_workspace_bytes(plan) > c->sk_ws_bytes)
     return fail(ISD_E_UNSUPPORTED, "stream-K workspace too small for the GEMM plan");
@@ -252,9 +260,17 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   CUtensorMap* tx = nullptr;
   int rc = tmap_for(c, x, m, k, plan.box_rows, &tx);
   if (rc) return rc;
+  isd::GemmAugment ga{nullptr, nullptr, 0};
+  if (aug) {
+    if (plan.streamk) return fail(ISD_E_UNSUPPORTED, "adapter product on a stream-K GEMM");
+    CUtensorMap* tx2 = nullptr;
+    rc = tmap_for(c, aug->x2, m, aug->k2, plan.box_rows, &tx2);
+    if (rc) return rc;
+    ga = isd::GemmAugment{aug->tw2, tx2, aug->k2};
+  }
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes));
+                            c->sk_ws_bytes, lora, aug ? &ga : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
@@ -317,20 +333,23 @@ isd::AttnShape attn_shape(const isd_ctx* c, const isd_kv* kv, int batch, int row
 // Gated-LoRA delta of one projection for every row: delta = (x A^T) B^T,
 // with x A^T summed over its K splits in fixed order and cast to bf16.
 // Consumers add scale * delta on MASK rows only.
-int lora_delta(isd_ctx* c, const CUtensorMap& ta, const CUtensorMap& tb, const __nv_bfloat16* x,
-               int M, int in, int n_a, int out, int32_t* status, cudaStream_t st) {
+// xa = bf16(scale * x A^T) on MASK rows, 0 on the others, into c->lora_xa
+// ([M][n_a]): split-K GEMM, fixed-order sum. Multiplied by B inside the base
+// GEMM (or the gate/up delta GEMM), it adds the gated delta on MASK rows and
+// exact zeros on verify rows.
+int lora_xa(isd_ctx* c, const CUtensorMap& ta, const __nv_bfloat16* x, int M, int in, int n_a,
+            int32_t* status, cudaStream_t st) {
   int s = 1;
   int rc = gemm(c, kPOther, ta, x, M, n_a, in, isd::kEpiF32, c->lora_xa_part,
                 static_cast<size_t>(c->max_splits) * c->cfg.max_rows * 3 * c->lora_rank,
                 c->max_splits, nullptr, &s, status, st);
   if (rc) return rc;
   cudaEvent_t e0 = prof_mark(c, st);
-  ISD_CUDA(isd::launch_sum_cast(c->lora_xa_part, s, M, n_a, c->lora_xa, st));
+  ISD_CUDA(isd::launch_sum_cast(c->lora_xa_part, s, M, n_a, c->meta_flags, c->lora_scale,
+                                c->lora_xa, st));
   prof_add(c, kPOther, e0, prof_mark(c, st));
   c->launches += 1;
-  const size_t wide = std::max(std::max(c->qkv_dim, c->cfg.hidden), 2 * c->cfg.intermediate);
-  return gemm(c, kPOther, tb, c->lora_xa, M, out, n_a, isd::kEpiF32, c->lora_delta,
-              static_cast<size_t>(c->cfg.max_rows) * wide, 1, nullptr, nullptr, status, st);
+  return ISD_OK;
 }
 
 int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, int32_t* status,
@@ -359,15 +378,18 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
 
   for (int l = 0; l < g.n_layers; ++l) {
     int s = 1;
-    int rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
-                  c->part_elems, c->max_splits, nullptr, &s, status, st);
-    if (rc) return rc;
+    int rc = ISD_OK;
     const int r = c->lora_rank;
     const isd_ctx::LoraLayer* ll = use_lora ? &c->lora[l] : nullptr;
+    // gated adapter on q/k/v: xa first, then B rides on the base GEMM's last split
+    AugSpec aug_qkv{ll ? &ll->tb_qkv : nullptr, c->lora_xa, 3 * r};
     if (ll) {
-      rc = lora_delta(c, ll->ta_qkv, ll->tb_qkv, c->hn, M, H, 3 * r, c->qkv_dim, status, st);
+      rc = lora_xa(c, ll->ta_qkv, c->hn, M, H, 3 * r, status, st);
       if (rc) return rc;
     }
+    rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
+              c->part_elems, c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_qkv : nullptr);
+    if (rc) return rc;
     isd::QkvReduceArgs qa;
     qa.part = c->part;
     qa.splits = s;
@@ -390,7 +412,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.k_pool = static_cast<__nv_bfloat16*>(kv->k_pool_dev);
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
-    qa.delta = ll ? c->lora_delta : nullptr;
+    qa.delta = nullptr;   // the adapter's delta is already in the last split
     qa.delta_scale = c->lora_scale;
     qa.status = status;
     cudaEvent_t a0 = prof_mark(c, st);
@@ -404,16 +426,17 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     cudaEvent_t a2 = prof_mark(c, st);
     prof_add(c, kPAttnSplit, a1, amid);
     prof_add(c, kPAttnCombine, amid, a2);
-    rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
-              c->max_splits, nullptr, &s, status, st);
-    if (rc) return rc;
+    AugSpec aug_o{ll ? &ll->tb_o : nullptr, c->lora_xa, r};
     if (ll) {
-      rc = lora_delta(c, ll->ta_o, ll->tb_o, c->attn, M, c->q_dim, r, H, status, st);
+      rc = lora_xa(c, ll->ta_o, c->attn, M, c->q_dim, r, status, st);
       if (rc) return rc;
     }
+    rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
+              c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_o : nullptr);
+    if (rc) return rc;
     cudaEvent_t r0 = prof_mark(c, st);
     ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st,
-                                       ll ? c->lora_delta : nullptr, c->lora_scale, c->meta_flags));
+                                       nullptr, 0.f, c->meta_flags));
     prof_add(c, kPResNorm, r0, prof_mark(c, st));
     c->launches += 1;
     if (!ll) {
@@ -427,25 +450,27 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
                 c->lora_gu, static_cast<size_t>(g.max_rows) * 2 * g.intermediate, 1, nullptr,
                 nullptr, status, st);
       if (rc) return rc;
-      rc = lora_delta(c, ll->ta_gu, ll->tb_gu, c->hn, M, H, 2 * r, 2 * g.intermediate, status, st);
+      // xa, then xa B^T whose epilogue adds scale * delta to the base on
+      // MASK rows (base alone elsewhere) and forms SiLU(gate) * up
+      rc = lora_xa(c, ll->ta_gu, c->hn, M, H, 2 * r, status, st);
       if (rc) return rc;
-      cudaEvent_t s0 = prof_mark(c, st);
-      ISD_CUDA(isd::launch_lora_silu(c->lora_gu, c->lora_delta, c->lora_scale, c->meta_flags, M,
-                                     g.intermediate, c->act, st));
-      prof_add(c, kPOther, s0, prof_mark(c, st));
-      c->launches += 1;
+      const isd::GemmLoraEpilogue le{c->lora_gu, c->meta_flags, 1.0f};   // xa carries the scale
+      rc = gemm(c, kPOther, ll->tb_gu, c->lora_xa, M, 2 * g.intermediate, 2 * r,
+                isd::kEpiSiluMulLora, nullptr, 0, 1, c->act, nullptr, status, st, &le);
+      if (rc) return rc;
+    }
+    AugSpec aug_d{ll ? &ll->tb_d : nullptr, c->lora_xa, r};
+    if (ll) {
+      rc = lora_xa(c, ll->ta_d, c->act, M, g.intermediate, r, status, st);
+      if (rc) return rc;
     }
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_d : nullptr);
     if (rc) return rc;
-    if (ll) {
-      rc = lora_delta(c, ll->ta_d, ll->tb_d, c->act, M, g.intermediate, r, H, status, st);
-      if (rc) return rc;
-    }
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
     cudaEvent_t r1 = prof_mark(c, st);
     ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st,
-                                       ll ? c->lora_delta : nullptr, c->lora_scale, c->meta_flags));
+                                       nullptr, 0.f, c->meta_flags));
     prof_add(c, kPResNorm, r1, prof_mark(c, st));
     c->launches += 1;
   }
@@ -634,8 +659,9 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
                e_bd = 1ull * H * r;
   const size_t per_layer = e_aqkv + e_bqkv + e_ao + e_bo + e_agu + e_bgu + e_ad + e_bd;
   const size_t R = g.max_rows;
-  const size_t wide = std::max(std::max<size_t>(ctx->qkv_dim, H), static_cast<size_t>(2) * I);
-  const size_t ws_bytes = ctx->max_splits * R * 3 * r * 4 + R * 3 * r * 2 + R * wide * 4 + R * 2 * I * 4;
+  // x A^T split slices, xa (bf16), the base gate/up product (fp32)
+  const size_t ws_bytes =
+      ctx->max_splits * R * 3 * r * 4 + ((R * 3 * r * 2 + 255) / 256) * 256 + R * 2 * I * 4;
   if (ctx->lora_mem) {
     cudaFree(ctx->lora_mem);
     ctx->lora_mem = nullptr;
@@ -709,8 +735,6 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
   w += ctx->max_splits * R * 3 * r * 4;
   ctx->lora_xa = reinterpret_cast<__nv_bfloat16*>(w);
   w += ((R * 3 * r * 2 + 255) / 256) * 256;
-  ctx->lora_delta = reinterpret_cast<float*>(w);
-  w += R * wide * 4;
   ctx->lora_gu = reinterpret_cast<float*>(w);
   ctx->lora_rank = r;
   ctx->lora_scale = lora->scale;

@@ -58,12 +58,20 @@ struct GemmParams {
   int64_t iters;      // unit tiles (256-row pair tiles or 128-row tiles) x kb_total
   float* sk_part;     // [units * (pair ? 2 : 1)][n_pad rounded up to 32][128] fp32 partials
   int32_t* sk_sync;   // [units * (pair ? 2 : 1)][2]: arrival count, ready flag
+  // split-K mode: the last split continues over aug_kb K-blocks of a second
+  // operand pair (tmap_w2, tmap_x2), accumulating into the same slice
+  int32_t aug_kb;
+  // kEpiSiluMulLora
+  const float* lora_base;
+  const int32_t* lora_flags;
+  float lora_scale;
 };
 
 // One contiguous run of K-blocks of one tile, processed by one CTA (pair).
 struct Segment {
   int ut;          // unit tile (pair tile for pairs)
   int kb_lo, kb_hi;
+  int aug;         // K-blocks of the second operand pair after kb_hi (split-K, last split)
   bool whole;      // covers every K-block of the tile (or split-K mode)
   int slot;        // stream-K workspace slot of a cut tile (per unit boundary)
 };
@@ -77,6 +85,7 @@ __device__ __forceinline__ bool get_segment(const GemmParams& p, int idx, Segmen
     sg.ut = kPair ? (blockIdx.x >> 1) : blockIdx.x;
     sg.kb_lo = kb0;
     sg.kb_hi = min(p.kb_total, kb0 + p.kb_per_split);
+    sg.aug = blockIdx.z == gridDim.z - 1 ? p.aug_kb : 0;
     sg.whole = true;
     sg.slot = -1;
     return true;
@@ -92,6 +101,7 @@ __device__ __forceinline__ bool get_segment(const GemmParams& p, int idx, Segmen
   sg.kb_lo = static_cast<int>(lo - tile * kbt);
   sg.kb_hi = static_cast<int>(hi - tile * kbt);
   sg.whole = sg.kb_lo == 0 && sg.kb_hi == p.kb_total;
+  sg.aug = 0;
   // a cut tile straddles the boundary between units s and s + 1: the head
   // part ends unit s's range (slot s = u), the tail part starts unit s + 1's
   // (slot s = u - 1)
@@ -111,7 +121,9 @@ __device__ __forceinline__ bool get_segment(const GemmParams& p, int idx, Segmen
 template <bool kPair, int kNmma>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmap_x,
+                      const __grid_constant__ CUtensorMap tmap_w2,
+                      const __grid_constant__ CUtensorMap tmap_x2, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -143,6 +155,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     prefetch_tensormap(&tmap_w);
     prefetch_tensormap(&tmap_x);
+    if (p.aug_kb > 0) {
+      prefetch_tensormap(&tmap_w2);
+      prefetch_tensormap(&tmap_x2);
+    }
   }
   if (warp == 0) {
     if (kPair) {
@@ -173,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     Segment sg;
     for (int idx = 0; ok && get_segment<kPair>(p, idx, sg); ++idx) {
       const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
-      for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+      const int n_base = sg.kb_hi - sg.kb_lo;
+      for (int i = 0; i < n_base + sg.aug; ++i) {
         if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
           flag(p.status, ISD_DEV_TIMEOUT);
           *abort_flag = 1;
@@ -182,19 +199,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* sa = smem + s * stage_bytes;
         uint8_t* sb = sa + kStageA;
-        const int kc = kb * kTileK;
+        const bool aug = i >= n_base;
+        const int kc = (aug ? i - n_base : sg.kb_lo + i) * kTileK;
+        const CUtensorMap* mw = aug ? &tmap_w2 : &tmap_w;
+        const CUtensorMap* mx = aug ? &tmap_x2 : &tmap_x;
         if (kPair) {
           const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d_pair(sa, &tmap_w, bar, kc, mt * kTileM, pol_w);
+          tma_load_2d_pair(sa, mw, bar, kc, mt * kTileM, pol_w);
           for (int bx = 0; bx < p.n_boxes; ++bx)
-            tma_load_2d_pair(sb + bx * p.box_rows * 128, &tmap_x, bar, kc,
+            tma_load_2d_pair(sb + bx * p.box_rows * 128, mx, bar, kc,
                              tok0 + bx * p.mma_n + static_cast<int>(rank) * p.box_rows, pol_x);
         } else {
           mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d_hint(sa, &tmap_w, &full[s], kc, mt * kTileM, pol_w);
+          tma_load_2d_hint(sa, mw, &full[s], kc, mt * kTileM, pol_w);
           for (int bx = 0; bx < p.n_boxes; ++bx)
-            tma_load_2d_hint(sb + bx * p.box_rows * 128, &tmap_x, &full[s], kc,
+            tma_load_2d_hint(sb + bx * p.box_rows * 128, mx, &full[s], kc,
                              tok0 + bx * p.box_rows, pol_x);
         }
         ++issued;
@@ -241,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+      const int n_kb = sg.kb_hi - sg.kb_lo + sg.aug;
+      for (int i = 0; i < n_kb; ++i) {
         if (!mbar_wait(&full[s], ph)) {
           flag(p.status, ISD_DEV_TIMEOUT);
           *abort_flag = 1;
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t db = db0 + static_cast<uint64_t>(s) * d_stage;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
-          const uint32_t acc = (kb > sg.kb_lo || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           if (kPair) {
             umma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, idesc, acc);
             if (kNmma == 2) umma_bf16_pair(tmem1, da + 2 * kk, db + d_mma + 2 * kk, idesc, acc);
@@ -368,6 +389,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          if (p.epi == kEpiSiluMulLora) {
+            // the accumulator is the LoRA delta: base + scale * delta on MASK
+            // rows, the base value itself on every other row
+            const float* bp = p.lora_base + static_cast<int64_t>(t0) * p.n_out + mt * kTileM +
+                              quad * 32 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (full_chunk || (c * 32 + j < p.n_pad && t0 + j < p.m)) {
+                const float b = *bp;
+                v[j] = (p.lora_flags[t0 + j] & kRowMask) ? b + p.lora_scale * v[j] : b;
+              }
+              bp += p.n_out;
+            }
+          }
           // Each quadrant's 32 TMEM lanes hold 16 gate rows then the 16 up
           // rows of the same features (see the gate/up layout in isd.h). A
           // lane pairs with lane ^ 16: low lanes finish even tokens, high
@@ -529,7 +564,8 @@ size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
-                        void* sk_workspace, size_t sk_workspace_bytes) {
+                        void* sk_workspace, size_t sk_workspace_bytes,
+                        const GemmLoraEpilogue* lora, const GemmAugment* augment) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -566,6 +602,28 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.iters = 0;
   p.sk_part = nullptr;
   p.sk_sync = nullptr;
+  p.lora_base = nullptr;
+  p.lora_flags = nullptr;
+  p.lora_scale = 0.f;
+  p.aug_kb = 0;
+  const CUtensorMap* tw2 = &tmap_w;
+  const CUtensorMap* tx2 = &tmap_x;
+  if (augment != nullptr && augment->k > 0) {
+    // the extra K-blocks ride on the last split of a split-K plan
+    if (plan.streamk || augment->k % kTileK != 0 || augment->tmap_w == nullptr ||
+        augment->tmap_x == nullptr)
+      return cudaErrorInvalidValue;
+    p.aug_kb = augment->k / kTileK;
+    tw2 = augment->tmap_w;
+    tx2 = augment->tmap_x;
+  }
+  if (epi == kEpiSiluMulLora) {
+    if (lora == nullptr || lora->base == nullptr || lora->row_flags == nullptr)
+      return cudaErrorInvalidValue;
+    p.lora_base = lora->base;
+    p.lora_flags = lora->row_flags;
+    p.lora_scale = lora->scale;
+  }
   const int per_unit = plan.pair ? 2 : 1;
   dim3 grid(n_out / kTileM, plan.n_chunks, plan.splits);
   if (plan.streamk) {
@@ -582,7 +640,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
     grid = dim3(plan.units * per_unit, 1, 1);
   }
   if (!plan.pair) {
-    kernel<<<grid, kThreads, plan.smem_bytes, stream>>>(tmap_w, tmap_x, p);
+    kernel<<<grid, kThreads, plan.smem_bytes, stream>>>(tmap_w, tmap_x, *tw2, *tx2, p);
     return cudaGetLastError();
   }
   if (grid.x % 2 != 0) return cudaErrorInvalidValue;
@@ -598,7 +656,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, tmap_w, tmap_x, p);
+  return cudaLaunchKernelEx(&cfg, kernel, tmap_w, tmap_x, *tw2, *tx2, p);
 }
 
 }  // namespace isd

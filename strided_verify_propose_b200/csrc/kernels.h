@@ -24,7 +24,26 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
                        uint32_t b0, uint32_t b1, uint32_t b2, std::string* err);
 
 // ---------------------------------------------------------------------- GEMM
-enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
+enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1, kEpiSiluMulLora = 2 };
+
+// kEpiSiluMulLora: the GEMM computes the gated-LoRA delta of the gate/up
+// projection; the epilogue forms base + scale * delta on MASK rows (base
+// alone on every other row, untouched), then SiLU(gate) * up as kEpiSiluMul.
+// A second operand pair whose product is added into the last split-K slice:
+// the last split runs k / 64 more K-blocks with W2 (box rows 128, the same
+// n_out rows) and X2 (box rows = plan.box_rows, the same m rows). Split-K
+// plans only.
+struct GemmAugment {
+  const CUtensorMap* tmap_w;
+  const CUtensorMap* tmap_x;
+  int32_t k;
+};
+
+struct GemmLoraEpilogue {
+  const float* base;          // [m][n_out] fp32: the base gate/up product
+  const int32_t* row_flags;   // [m]: kRowMask marks the rows that take the delta
+  float scale;
+};
 
 struct GemmPlan {
   int32_t n_pad = 0, n_mma = 0, mma_n = 0, box_rows = 0, n_boxes = 0;
@@ -53,7 +72,9 @@ size_t gemm_streamk_sync_bytes();
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
-                        void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0);
+                        void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
+                        const GemmLoraEpilogue* lora = nullptr,
+                        const GemmAugment* augment = nullptr);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {
@@ -121,11 +142,10 @@ cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows
 cudaError_t launch_pack_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst,
                              int dst_ld, int row0, int col0, int interleave_off,
                              cudaStream_t stream);
-cudaError_t launch_sum_cast(const float* part, int splits, int rows, int n, __nv_bfloat16* out,
-                            cudaStream_t stream);
-cudaError_t launch_lora_silu(const float* gu, const float* delta, float scale,
-                             const int32_t* row_flags, int rows, int inter, __nv_bfloat16* act,
-                             cudaStream_t stream);
+// out = bf16(scale * sum of the splits) on MASK rows (row_flags), 0 elsewhere.
+cudaError_t launch_sum_cast(const float* part, int splits, int rows, int n, const int32_t* row_flags,
+                            float scale, __nv_bfloat16* out, cudaStream_t stream);
+
 
 // ---------------------------------------------------------- accept / propose
 struct AcceptArgs {
