@@ -115,6 +115,9 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
 
 using isd::GemmPlan;
 
+// K-splits allowed for the adapter's thin x A^T products
+constexpr int kLoraSplits = 32;
+
 struct isd_ctx {
   isd_model_cfg cfg{};
   const void* embed = nullptr;
@@ -163,9 +166,8 @@ struct isd_ctx {
     CUtensorMap ta_qkv, tb_qkv, ta_o, tb_o, ta_gu, tb_gu, ta_d, tb_d;
   };
   std::vector<LoraLayer> lora;
-  float* lora_xa_part = nullptr;         // [max_splits][max_rows][3r]
+  float* lora_xa_part = nullptr;         // [kLoraSplits][max_rows][3r]
   __nv_bfloat16* lora_xa = nullptr;      // [max_rows][3r]
-  float* lora_gu = nullptr;              // [max_rows][2 I] base gate/up in fp32
 
   // per-kernel-class event timing (isd_profile_enable)
   bool prof_on = false;
@@ -222,13 +224,14 @@ int tmap_for(isd_ctx* c, const void* base, int rows, int cols, int box_rows, CUt
 }
 
 // single: one output slice (the SiLU epilogue, the LM head); such plans may
-// run as stream-K when the tiles overfill one wave.
-const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k, bool single) {
-  auto key = std::make_tuple(m, n, k, single ? 1 : 0);
+// run as stream-K when the tiles overfill one wave. Otherwise up to
+// max_splits K-splits.
+const GemmPlan& plan_for(isd_ctx* c, int m, int n, int k, bool single, int max_splits) {
+  auto key = std::make_tuple(m, n, k, single ? 1 : max_splits);
   auto it = c->plans.find(key);
   if (it == c->plans.end()) {
     const GemmPlan p = single ? isd::plan_gemm(m, n, k, 0, 1, num_sms(), true)
-                              : isd::plan_gemm(m, n, k, 0, c->max_splits, num_sms());
+                              : isd::plan_gemm(m, n, k, 0, max_splits, num_sms());
     it = c->plans.emplace(key, p).first;
   }
   return it->second;
@@ -248,8 +251,9 @@ struct AugSpec {
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
-         const isd::GemmLoraEpilogue* lora = nullptr, const AugSpec* aug = nullptr) {
-  const GemmPlan& plan = plan_for(c, m, n, k, epi != isd::kEpiF32 || max_splits == 1);
+         const AugSpec* aug = nullptr) {
+  const GemmPlan& plan =
+      plan_for(c, m, n, k, epi != isd::kEpiF32 || max_splits == 1, std::min(max_splits, kLoraSplits));
   if (plan.n_pad == 0) return fail(ISD_E_UNSUPPORTED, "no GEMM plan");
   if (isd::gemm_streamk_workspace_bytes(plan) > c->sk_ws_bytes)
     return fail(ISD_E_UNSUPPORTED, "stream-K workspace too small for the GEMM plan");
@@ -262,7 +266,6 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   if (rc) return rc;
   isd::GemmAugment ga{nullptr, nullptr, 0};
   if (aug) {
-    if (plan.streamk) return fail(ISD_E_UNSUPPORTED, "adapter product on a stream-K GEMM");
     CUtensorMap* tx2 = nullptr;
     rc = tmap_for(c, aug->x2, m, aug->k2, plan.box_rows, &tx2);
     if (rc) return rc;
@@ -270,7 +273,7 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   }
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, lora, aug ? &ga : nullptr));
+                            c->sk_ws_bytes, aug ? &ga : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
@@ -340,9 +343,10 @@ isd::AttnShape attn_shape(const isd_ctx* c, const isd_kv* kv, int batch, int row
 int lora_xa(isd_ctx* c, const CUtensorMap& ta, const __nv_bfloat16* x, int M, int in, int n_a,
             int32_t* status, cudaStream_t st) {
   int s = 1;
+  // a thin product (1-3 tiles of 128 outputs): many K-splits keep the SMs busy
   int rc = gemm(c, kPOther, ta, x, M, n_a, in, isd::kEpiF32, c->lora_xa_part,
-                static_cast<size_t>(c->max_splits) * c->cfg.max_rows * 3 * c->lora_rank,
-                c->max_splits, nullptr, &s, status, st);
+                static_cast<size_t>(kLoraSplits) * c->cfg.max_rows * 3 * c->lora_rank,
+                kLoraSplits, nullptr, &s, status, st);
   if (rc) return rc;
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_sum_cast(c->lora_xa_part, s, M, n_a, c->meta_flags, c->lora_scale,
@@ -388,7 +392,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_qkv : nullptr);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr);
     if (rc) return rc;
     isd::QkvReduceArgs qa;
     qa.part = c->part;
@@ -432,40 +436,30 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
-              c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_o : nullptr);
+              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
     if (rc) return rc;
     cudaEvent_t r0 = prof_mark(c, st);
     ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st,
                                        nullptr, 0.f, c->meta_flags));
     prof_add(c, kPResNorm, r0, prof_mark(c, st));
     c->launches += 1;
-    if (!ll) {
-      rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiSiluMul,
-                nullptr, 0, 1, c->act, nullptr, status, st);
-      if (rc) return rc;
-    } else {
-      // base gate/up in fp32 (one split, the same sums the fused epilogue sees),
-      // the delta, then SwiGLU with the delta on MASK rows only
-      rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiF32,
-                c->lora_gu, static_cast<size_t>(g.max_rows) * 2 * g.intermediate, 1, nullptr,
-                nullptr, status, st);
-      if (rc) return rc;
-      // xa, then xa B^T whose epilogue adds scale * delta to the base on
-      // MASK rows (base alone elsewhere) and forms SiLU(gate) * up
+    // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
+    // K-blocks follow each tile's base K-blocks (stream-K cuts unchanged)
+    AugSpec aug_gu{ll ? &ll->tb_gu : nullptr, c->lora_xa, 2 * r};
+    if (ll) {
       rc = lora_xa(c, ll->ta_gu, c->hn, M, H, 2 * r, status, st);
       if (rc) return rc;
-      const isd::GemmLoraEpilogue le{c->lora_gu, c->meta_flags, 1.0f};   // xa carries the scale
-      rc = gemm(c, kPOther, ll->tb_gu, c->lora_xa, M, 2 * g.intermediate, 2 * r,
-                isd::kEpiSiluMulLora, nullptr, 0, 1, c->act, nullptr, status, st, &le);
-      if (rc) return rc;
     }
+    rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiSiluMul,
+              nullptr, 0, 1, c->act, nullptr, status, st, ll ? &aug_gu : nullptr);
+    if (rc) return rc;
     AugSpec aug_d{ll ? &ll->tb_d : nullptr, c->lora_xa, r};
     if (ll) {
       rc = lora_xa(c, ll->ta_d, c->act, M, g.intermediate, r, status, st);
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, nullptr, ll ? &aug_d : nullptr);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr);
     if (rc) return rc;
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
     cudaEvent_t r1 = prof_mark(c, st);
@@ -659,9 +653,8 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
                e_bd = 1ull * H * r;
   const size_t per_layer = e_aqkv + e_bqkv + e_ao + e_bo + e_agu + e_bgu + e_ad + e_bd;
   const size_t R = g.max_rows;
-  // x A^T split slices, xa (bf16), the base gate/up product (fp32)
-  const size_t ws_bytes =
-      ctx->max_splits * R * 3 * r * 4 + ((R * 3 * r * 2 + 255) / 256) * 256 + R * 2 * I * 4;
+  // x A^T split slices, xa (bf16)
+  const size_t ws_bytes = kLoraSplits * R * 3 * r * 4 + ((R * 3 * r * 2 + 255) / 256) * 256;
   if (ctx->lora_mem) {
     cudaFree(ctx->lora_mem);
     ctx->lora_mem = nullptr;
@@ -732,10 +725,9 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
   }
   char* w = mem + ((w_bytes + 1023) & ~static_cast<size_t>(1023));
   ctx->lora_xa_part = reinterpret_cast<float*>(w);
-  w += ctx->max_splits * R * 3 * r * 4;
+  w += kLoraSplits * R * 3 * r * 4;
   ctx->lora_xa = reinterpret_cast<__nv_bfloat16*>(w);
   w += ((R * 3 * r * 2 + 255) / 256) * 256;
-  ctx->lora_gu = reinterpret_cast<float*>(w);
   ctx->lora_rank = r;
   ctx->lora_scale = lora->scale;
   ctx->has_lora = true;

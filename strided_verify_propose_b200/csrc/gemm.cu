@@ -58,20 +58,18 @@ struct GemmParams {
   int64_t iters;      // unit tiles (256-row pair tiles or 128-row tiles) x kb_total
   float* sk_part;     // [units * (pair ? 2 : 1)][n_pad rounded up to 32][128] fp32 partials
   int32_t* sk_sync;   // [units * (pair ? 2 : 1)][2]: arrival count, ready flag
-  // split-K mode: the last split continues over aug_kb K-blocks of a second
-  // operand pair (tmap_w2, tmap_x2), accumulating into the same slice
+  // the last split (stream-K: the segment ending the tile's base K-blocks)
+  // continues over aug_kb K-blocks of a second operand pair (tmap_w2,
+  // tmap_x2), accumulating into the same result
   int32_t aug_kb;
-  // kEpiSiluMulLora
-  const float* lora_base;
-  const int32_t* lora_flags;
-  float lora_scale;
 };
 
 // One contiguous run of K-blocks of one tile, processed by one CTA (pair).
 struct Segment {
   int ut;          // unit tile (pair tile for pairs)
   int kb_lo, kb_hi;
-  int aug;         // K-blocks of the second operand pair after kb_hi (split-K, last split)
+  int aug;         // K-blocks of the second operand pair after kb_hi (the last split, or
+                   // the stream-K segment that holds the tile's last base K-block)
   bool whole;      // covers every K-block of the tile (or split-K mode)
   int slot;        // stream-K workspace slot of a cut tile (per unit boundary)
 };
@@ -101,7 +99,9 @@ __device__ __forceinline__ bool get_segment(const GemmParams& p, int idx, Segmen
   sg.kb_lo = static_cast<int>(lo - tile * kbt);
   sg.kb_hi = static_cast<int>(hi - tile * kbt);
   sg.whole = sg.kb_lo == 0 && sg.kb_hi == p.kb_total;
-  sg.aug = 0;
+  // the second operand pair follows a tile's last base K-block; the ranges
+  // are cut on base K-blocks only, so the cut points do not depend on it
+  sg.aug = sg.kb_hi == p.kb_total ? p.aug_kb : 0;
   // a cut tile straddles the boundary between units s and s + 1: the head
   // part ends unit s's range (slot s = u), the tail part starts unit s + 1's
   // (slot s = u - 1)
@@ -389,20 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          if (p.epi == kEpiSiluMulLora) {
-            // the accumulator is the LoRA delta: base + scale * delta on MASK
-            // rows, the base value itself on every other row
-            const float* bp = p.lora_base + static_cast<int64_t>(t0) * p.n_out + mt * kTileM +
-                              quad * 32 + lane;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (full_chunk || (c * 32 + j < p.n_pad && t0 + j < p.m)) {
-                const float b = *bp;
-                v[j] = (p.lora_flags[t0 + j] & kRowMask) ? b + p.lora_scale * v[j] : b;
-              }
-              bp += p.n_out;
-            }
-          }
           // Each quadrant's 32 TMEM lanes hold 16 gate rows then the 16 up
           // rows of the same features (see the gate/up layout in isd.h). A
           // lane pairs with lane ^ 16: low lanes finish even tokens, high
@@ -565,7 +551,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace, size_t sk_workspace_bytes,
-                        const GemmLoraEpilogue* lora, const GemmAugment* augment) {
+                        const GemmAugment* augment) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -602,27 +588,15 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.iters = 0;
   p.sk_part = nullptr;
   p.sk_sync = nullptr;
-  p.lora_base = nullptr;
-  p.lora_flags = nullptr;
-  p.lora_scale = 0.f;
   p.aug_kb = 0;
   const CUtensorMap* tw2 = &tmap_w;
   const CUtensorMap* tx2 = &tmap_x;
   if (augment != nullptr && augment->k > 0) {
-    // the extra K-blocks ride on the last split of a split-K plan
-    if (plan.streamk || augment->k % kTileK != 0 || augment->tmap_w == nullptr ||
-        augment->tmap_x == nullptr)
+    if (augment->k % kTileK != 0 || augment->tmap_w == nullptr || augment->tmap_x == nullptr)
       return cudaErrorInvalidValue;
     p.aug_kb = augment->k / kTileK;
     tw2 = augment->tmap_w;
     tx2 = augment->tmap_x;
-  }
-  if (epi == kEpiSiluMulLora) {
-    if (lora == nullptr || lora->base == nullptr || lora->row_flags == nullptr)
-      return cudaErrorInvalidValue;
-    p.lora_base = lora->base;
-    p.lora_flags = lora->row_flags;
-    p.lora_scale = lora->scale;
   }
   const int per_unit = plan.pair ? 2 : 1;
   dim3 grid(n_out / kTileM, plan.n_chunks, plan.splits);

@@ -24,26 +24,7 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
                        uint32_t b0, uint32_t b1, uint32_t b2, std::string* err);
 
 // ---------------------------------------------------------------------- GEMM
-enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1, kEpiSiluMulLora = 2 };
-
-// kEpiSiluMulLora: the GEMM computes the gated-LoRA delta of the gate/up
-// projection; the epilogue forms base + scale * delta on MASK rows (base
-// alone on every other row, untouched), then SiLU(gate) * up as kEpiSiluMul.
-// A second operand pair whose product is added into the last split-K slice:
-// the last split runs k / 64 more K-blocks with W2 (box rows 128, the same
-// n_out rows) and X2 (box rows = plan.box_rows, the same m rows). Split-K
-// plans only.
-struct GemmAugment {
-  const CUtensorMap* tmap_w;
-  const CUtensorMap* tmap_x;
-  int32_t k;
-};
-
-struct GemmLoraEpilogue {
-  const float* base;          // [m][n_out] fp32: the base gate/up product
-  const int32_t* row_flags;   // [m]: kRowMask marks the rows that take the delta
-  float scale;
-};
+enum GemmEpilogue : int32_t { kEpiF32 = 0, kEpiSiluMul = 1 };
 
 struct GemmPlan {
   int32_t n_pad = 0, n_mma = 0, mma_n = 0, box_rows = 0, n_boxes = 0;
@@ -66,6 +47,18 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
 size_t gemm_streamk_workspace_bytes(const GemmPlan& plan);
 size_t gemm_streamk_sync_bytes();
 
+// A second operand pair whose product is added to the result: the last
+// split (under stream-K, the segment that ends a tile's base K-blocks) runs
+// k / 64 more K-blocks with W2 (box rows 128, the same n_out rows) and X2
+// (box rows = plan.box_rows, the same m rows). Stream-K ranges are cut on the
+// base K-blocks alone, so the base part of every result is summed exactly as
+// without the second pair.
+struct GemmAugment {
+  const CUtensorMap* tmap_w;
+  const CUtensorMap* tmap_x;
+  int32_t k;
+};
+
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
 // with W's rows interleaved in blocks of 16 (gate rows then up rows).
@@ -73,7 +66,6 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmLoraEpilogue* lora = nullptr,
                         const GemmAugment* augment = nullptr);
 
 // ----------------------------------------------------------------- attention

@@ -39,8 +39,11 @@ __global__ void sum_cast_kernel(const float* part, int splits, int64_t split_str
   const bool mask_row = row_flags[row] & kRowMask;
   for (int c = threadIdx.x; c < n; c += blockDim.x) {
     float v = 0.f;
-    if (mask_row)
-      for (int s = 0; s < splits; ++s) v += part[s * split_stride + static_cast<int64_t>(row) * n + c];
+    if (mask_row) {
+      const float* pc = part + static_cast<int64_t>(row) * n + c;
+#pragma unroll 8
+      for (int s = 0; s < splits; ++s) v += pc[s * split_stride];   // loads ahead, adds in order
+    }
     out[static_cast<int64_t>(row) * n + c] = __float2bfloat16_rn(mask_row ? scale * v : 0.f);
   }
 }
