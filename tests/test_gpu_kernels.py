@@ -216,6 +216,7 @@ def _run_accept_gpu(c, Bn, N, V, flags):
     (5, 1, 512, oi.ARGMAX, oi.STOCHASTIC, 0.0),       # N = 1: plain AR sampling
     (12, 4, 20000, oi.ARGMAX, oi.STOCHASTIC, 6.0),    # several vocab chunks, ragged tail
     (64, 4, 151936, oi.ARGMAX, oi.STOCHASTIC, 7.5),   # benchmark config, p_top ~ 0.9
+    (16, 4, 151936, oi.SAMPLE, oi.STOCHASTIC, 7.5),   # sampled proposals, full-vocabulary q rows
 ])
 def test_accept_propose_matches_oracle(cuda_lib, Bn, N, V, propose, verify, boost):
     c = _accept_case(Bn, N, V, propose, verify, seed=Bn * 31 + N, boost=boost)
