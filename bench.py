@@ -128,6 +128,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def reduce_over_ranks(times_ms, tokens, ws, device):
+    """Whole-job figures from every rank's own: each time is the max over the
+    ranks (the job ends with its slowest replica), each token count the sum.
+    Every rank calls it with the same number of values."""
+    import torch
+    vals = torch.tensor(list(times_ms), device=device, dtype=torch.float64)
+    toks = torch.tensor(list(tokens), device=device, dtype=torch.float64)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(toks, op=dist.ReduceOp.SUM)
+    return vals.tolist(), toks.tolist()
+
+
 def setup_dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -319,14 +333,9 @@ def run_cuda(args, ws, rank, local):
     e2e_committed = int((pin_acc.long() + 1).sum().item())
 
     # ---- reduce over ranks: max time, summed tokens
-    vals = torch.tensor([ms, e2e_ms, nat_ms, eager_ms or 0.0], device="cuda", dtype=torch.float64)
-    toks = torch.tensor([committed, e2e_committed, nat_committed, eager_committed], device="cuda",
-                        dtype=torch.float64)
-    if ws > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        dist.all_reduce(toks, op=dist.ReduceOp.SUM)
-    ms, e2e_ms, nat_ms, eager_ms_all = vals.tolist()
-    committed, e2e_committed, nat_committed, eager_committed = toks.tolist()
+    (ms, e2e_ms, nat_ms, eager_ms_all), (committed, e2e_committed, nat_committed, eager_committed) = \
+        reduce_over_ranks([ms, e2e_ms, nat_ms, eager_ms or 0.0],
+                          [committed, e2e_committed, nat_committed, eager_committed], ws, "cuda")
 
     result = None
     if rank == 0:
