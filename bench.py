@@ -188,7 +188,8 @@ def run_cuda(args, ws, rank, local):
     t0 = time.time()
     weights = Bd.random_device_weights(shape, seed=seed)
     G = shape.n_q_heads // shape.n_kv_heads
-    model = Bd.Model(shape, weights, max_batch=B, max_rows=max(B * R, B * (64 // G)),
+    # 64 rows per request per prefill pass (several attention query tiles)
+    model = Bd.Model(shape, weights, max_batch=B, max_rows=max(B * R, B * 64),
                      max_position=maxp * P)
     lora_rank = wl.get("lora_rank", 0)
     flags = 0

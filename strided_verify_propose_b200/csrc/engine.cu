@@ -136,10 +136,13 @@ struct isd_ctx {
   __nv_bfloat16* hn = nullptr;      // [max_rows][hidden] normalised GEMM input
   float* part = nullptr;            // [max_splits][max_rows][max(qkv_dim, hidden)]
   size_t part_elems = 0;
+  size_t logit_rows = 0;            // rows the logits buffer holds (steps only)
+  int prefill_sub_max = 1;          // attention sub-requests per request in a prefill chunk
+  int32_t* prefill_table = nullptr; // [max_batch * prefill_sub_max][max pages] repeated page rows
   __nv_bfloat16* qbuf = nullptr;    // [max_rows][q_dim]
   __nv_bfloat16* attn = nullptr;    // [max_rows][q_dim]
   __nv_bfloat16* act = nullptr;     // [max_rows][intermediate]
-  float* logits = nullptr;          // [max_rows][vocab]
+  float* logits = nullptr;          // [logit_rows][vocab]
   int32_t* meta_tok = nullptr;
   int32_t* meta_pos = nullptr;
   int32_t* meta_flags = nullptr;
@@ -252,6 +255,11 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
          const AugSpec* aug = nullptr) {
+  if (epi == isd::kEpiF32 && out_elems > 0) {
+    // large prefill chunks: no more splits than the partial buffer holds
+    const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
+    max_splits = static_cast<int>(std::max<size_t>(1, std::min<size_t>(max_splits, fit)));
+  }
   const GemmPlan& plan =
       plan_for(c, m, n, k, epi != isd::kEpiF32 || max_splits == 1, std::min(max_splits, kLoraSplits));
   if (plan.n_pad == 0) return fail(ISD_E_UNSUPPORTED, "no GEMM plan");
@@ -331,21 +339,17 @@ isd::AttnShape attn_shape(const isd_ctx* c, const isd_kv* kv, int batch, int row
   return s;
 }
 
-// The decoder layers over the rows described by the row metadata; leaves
-// bf16(final RMSNorm(x)) in c->hn.
-// Gated-LoRA delta of one projection for every row: delta = (x A^T) B^T,
-// with x A^T summed over its K splits in fixed order and cast to bf16.
-// Consumers add scale * delta on MASK rows only.
 // xa = bf16(scale * x A^T) on MASK rows, 0 on the others, into c->lora_xa
 // ([M][n_a]): split-K GEMM, fixed-order sum. Multiplied by B inside the base
-// GEMM (or the gate/up delta GEMM), it adds the gated delta on MASK rows and
-// exact zeros on verify rows.
+// GEMM, it adds the gated delta on MASK rows and exact zeros on verify rows.
 int lora_xa(isd_ctx* c, const CUtensorMap& ta, const __nv_bfloat16* x, int M, int in, int n_a,
             int32_t* status, cudaStream_t st) {
   int s = 1;
   // a thin product (1-3 tiles of 128 outputs): many K-splits keep the SMs busy
   int rc = gemm(c, kPOther, ta, x, M, n_a, in, isd::kEpiF32, c->lora_xa_part,
-                static_cast<size_t>(kLoraSplits) * c->cfg.max_rows * 3 * c->lora_rank,
+                static_cast<size_t>(kLoraSplits) *
+                    std::min<size_t>(c->cfg.max_rows, static_cast<size_t>(c->cfg.max_batch) * 15) *
+                    3 * c->lora_rank,
                 kLoraSplits, nullptr, &s, status, st);
   if (rc) return rc;
   cudaEvent_t e0 = prof_mark(c, st);
@@ -356,8 +360,16 @@ int lora_xa(isd_ctx* c, const CUtensorMap& ta, const __nv_bfloat16* x, int M, in
   return ISD_OK;
 }
 
+// The decoder layers over the rows described by the row metadata; leaves
+// bf16(final RMSNorm(x)) in c->hn. attn_sub > 1 (prefill): the attention sees
+// each request's rows_per_req rows as attn_sub consecutive sub-requests of
+// rows_per_req / attn_sub rows that share the request's pages (attn_table:
+// the page table with each row repeated attn_sub times); attention is
+// read-only on the cache, so this is the same computation in query tiles the
+// attention kernel holds.
 int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, int32_t* status,
-                   cudaStream_t st, bool use_lora = false) {
+                   cudaStream_t st, bool use_lora = false, int attn_sub = 1,
+                   const int32_t* attn_table = nullptr) {
   const isd_model_cfg& g = c->cfg;
   const int M = batch * rows_per_req;
   const int H = g.hidden;
@@ -376,7 +388,10 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
   if (!isd::make_tmap_bf16(&kmap, kv->k_pool_dev, pool_rows, g.head_dim, g.page_size, &err) ||
       !isd::make_tmap_bf16(&vmap, kv->v_pool_dev, pool_rows, g.head_dim, g.page_size, &err))
     return fail(ISD_E_INVALID, "KV pool tensor map: " + err);
-  const isd::AttnShape ash = attn_shape(c, kv, batch, rows_per_req);
+  if (attn_sub < 1 || rows_per_req % attn_sub || (attn_sub > 1 && attn_table == nullptr))
+    return fail(ISD_E_INVALID, "attention sub-requests must split the rows evenly");
+  const isd::AttnShape ash = attn_shape(c, kv, batch * attn_sub, rows_per_req / attn_sub);
+  const int32_t* ash_table = attn_sub > 1 ? attn_table : kv->page_table_dev;
   if (isd::attention_workspace_bytes(ash) > c->attn_ws_bytes)
     return fail(ISD_E_UNSUPPORTED, "attention workspace too small for this batch shape");
 
@@ -425,7 +440,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     cudaEvent_t a1 = prof_mark(c, st);
     prof_add(c, kPQkvReduce, a0, a1);
     cudaEvent_t amid = prof_event(c);
-    ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, kv->page_table_dev,
+    ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid));
     cudaEvent_t a2 = prof_mark(c, st);
     prof_add(c, kPAttnSplit, a1, amid);
@@ -475,6 +490,15 @@ int alloc_workspace(isd_ctx* c) {
   const isd_model_cfg& g = c->cfg;
   const size_t R = g.max_rows;
   const size_t wide = std::max(c->qkv_dim, g.hidden);
+  // a step has at most batch x (2N - 1) <= max_batch x 15 rows; only steps
+  // need logits and many K-splits, prefill chunks may use all max_rows
+  const size_t step_rows = std::min(R, static_cast<size_t>(g.max_batch) * 15);
+  const size_t part_rows = std::max(static_cast<size_t>(c->max_splits) * step_rows, R);
+  const int G = g.n_q_heads / g.n_kv_heads;
+  const int att_rows = std::max(1, 64 / G);   // rows per request in one attention query tile
+  c->prefill_sub_max = static_cast<int>(std::max<size_t>(
+      1, std::min<size_t>(G, R / (static_cast<size_t>(g.max_batch) * att_rows))));
+  const size_t max_pages = (g.max_position + g.page_size - 1) / g.page_size;
   // attention workspace: the largest query tile (64 rows) at max_batch, longest requests
   isd::AttnShape a;
   a.batch = g.max_batch;
@@ -492,6 +516,10 @@ int alloc_workspace(isd_ctx* c) {
   isd::AttnShape a_dec = a;
   a_dec.rows_per_req = std::max(1, 32 / (g.n_q_heads / g.n_kv_heads));
   c->attn_ws_bytes = std::max(c->attn_ws_bytes, isd::attention_workspace_bytes(a_dec));
+  // prefill chunks: up to prefill_sub_max query tiles per request
+  isd::AttnShape a_pre = a;
+  a_pre.batch = g.max_batch * c->prefill_sub_max;
+  c->attn_ws_bytes = std::max(c->attn_ws_bytes, isd::attention_workspace_bytes(a_pre));
   const int maxN = 8;
   c->acc_ws_bytes = isd::accept_workspace_bytes(g.max_batch, maxN, g.vocab);
   // stream-K: one slot per SM of fp32 partials of up to 512 tokens x 128 rows
@@ -500,16 +528,17 @@ int alloc_workspace(isd_ctx* c) {
   size_t sizes[] = {
       R * g.hidden * sizeof(float),                       // x
       R * g.hidden * 2,                                   // hn
-      c->max_splits * R * wide * sizeof(float),           // part
+      part_rows * wide * sizeof(float),                   // part
       R * c->q_dim * 2,                                   // qbuf
       R * c->q_dim * 2,                                   // attn
       R * g.intermediate * 2,                             // act
-      R * static_cast<size_t>(g.vocab) * sizeof(float),   // logits
+      step_rows * static_cast<size_t>(g.vocab) * sizeof(float),  // logits
       R * 4, R * 4, R * 4,                                // meta
       static_cast<size_t>(g.max_position) * (g.head_dim / 2) * sizeof(float2),  // rope
       c->attn_ws_bytes, c->acc_ws_bytes,
       static_cast<size_t>(g.max_batch) * 4,
       c->sk_ws_bytes,
+      static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -524,7 +553,8 @@ int alloc_workspace(isd_ctx* c) {
   c->x = reinterpret_cast<float*>(b + off[i++]);
   c->hn = reinterpret_cast<__nv_bfloat16*>(b + off[i++]);
   c->part = reinterpret_cast<float*>(b + off[i++]);
-  c->part_elems = c->max_splits * R * wide;
+  c->part_elems = part_rows * wide;
+  c->logit_rows = step_rows;
   c->qbuf = reinterpret_cast<__nv_bfloat16*>(b + off[i++]);
   c->attn = reinterpret_cast<__nv_bfloat16*>(b + off[i++]);
   c->act = reinterpret_cast<__nv_bfloat16*>(b + off[i++]);
@@ -537,6 +567,7 @@ int alloc_workspace(isd_ctx* c) {
   c->acc_ws = b + off[i++];
   c->prefill_lens = reinterpret_cast<int32_t*>(b + off[i++]);
   c->sk_ws = b + off[i++];
+  c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
   if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
     return fail(ISD_E_CUDA, "stream-K workspace clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
@@ -653,8 +684,9 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
                e_bd = 1ull * H * r;
   const size_t per_layer = e_aqkv + e_bqkv + e_ao + e_bo + e_agu + e_bgu + e_ad + e_bd;
   const size_t R = g.max_rows;
-  // x A^T split slices, xa (bf16)
-  const size_t ws_bytes = kLoraSplits * R * 3 * r * 4 + ((R * 3 * r * 2 + 255) / 256) * 256;
+  // x A^T split slices, xa (bf16); the adapter runs in steps only
+  const size_t Rs = std::min(R, static_cast<size_t>(ctx->cfg.max_batch) * 15);
+  const size_t ws_bytes = kLoraSplits * Rs * 3 * r * 4 + ((Rs * 3 * r * 2 + 255) / 256) * 256;
   if (ctx->lora_mem) {
     cudaFree(ctx->lora_mem);
     ctx->lora_mem = nullptr;
@@ -725,9 +757,8 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
   }
   char* w = mem + ((w_bytes + 1023) & ~static_cast<size_t>(1023));
   ctx->lora_xa_part = reinterpret_cast<float*>(w);
-  w += kLoraSplits * R * 3 * r * 4;
+  w += kLoraSplits * Rs * 3 * r * 4;
   ctx->lora_xa = reinterpret_cast<__nv_bfloat16*>(w);
-  w += ((R * 3 * r * 2 + 255) / 256) * 256;
   ctx->lora_rank = r;
   ctx->lora_scale = lora->scale;
   ctx->has_lora = true;
@@ -770,6 +801,8 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
   rc = forward_layers(ctx, kv, B, R, status_dev, st, use_lora);
   if (rc) return rc;
   const int M = B * R;
+  if (!batch->logits_out_dev && static_cast<size_t>(M) > ctx->logit_rows)
+    return fail(ISD_E_UNSUPPORTED, "more block rows than the logits workspace holds");
   float* logits = batch->logits_out_dev ? batch->logits_out_dev : ctx->logits;
   // the LM head writes the logits themselves: never split-K
   rc = gemm(ctx, kPGemmLmHead, ctx->tm_lm, ctx->hn, M, g.vocab, g.hidden, isd::kEpiF32, logits,
@@ -857,17 +890,33 @@ int isd_prefill(isd_ctx* ctx, const isd_kv* kv, const int32_t* tokens_dev, int32
   if (rc) return rc;
   const isd_model_cfg& g = ctx->cfg;
   const int G = g.n_q_heads / g.n_kv_heads;
-  const int chunk = std::max(1, std::min(64 / G, g.max_rows / batch));
+  // rows per request and pass: up to prefill_sub_max attention query tiles
+  // (each 64 / G rows of one request), as far as max_rows allows
+  const int att_rows = std::max(1, 64 / G);
+  int chunk = std::max(1, std::min(att_rows * ctx->prefill_sub_max, g.max_rows / batch));
+  int sub = 1;
+  if (chunk > att_rows) {
+    sub = chunk / att_rows;
+    chunk = sub * att_rows;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ctx->launches = 0;
   ISD_CUDA(cudaMemcpyAsync(ctx->prefill_lens, lens_host, sizeof(int32_t) * batch,
                            cudaMemcpyHostToDevice, st));
+  if (sub > 1) {
+    // the page table with every request's row repeated once per sub-request
+    const size_t row_bytes = static_cast<size_t>(kv->max_pages_per_req) * sizeof(int32_t);
+    for (int j = 0; j < sub; ++j)
+      ISD_CUDA(cudaMemcpy2DAsync(ctx->prefill_table + static_cast<size_t>(j) * kv->max_pages_per_req,
+                                 row_bytes * sub, kv->page_table_dev, row_bytes, row_bytes, batch,
+                                 cudaMemcpyDeviceToDevice, st));
+  }
   isd::RowMeta meta{ctx->meta_tok, ctx->meta_pos, ctx->meta_flags};
   for (int start = 0; start < longest - 1; start += chunk) {
     ISD_CUDA(isd::launch_assemble_prefill(tokens_dev, max_len, ctx->prefill_lens, batch, chunk,
                                           start, meta, st));
     ctx->launches += 1;
-    rc = forward_layers(ctx, kv, batch, chunk, status_dev, st);
+    rc = forward_layers(ctx, kv, batch, chunk, status_dev, st, false, sub, ctx->prefill_table);
     if (rc) return rc;
   }
   // starting state: L = len - 1, x* = last prompt token, no drafts

@@ -26,7 +26,7 @@ torch = pytest.importorskip("torch")
 
 
 def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exact=0.7,
-             useed=None, lora=False):
+             useed=None, lora=False, prefill_rows=None):
     from strided_verify_propose_b200 import binding as B
     R = 2 * N - 1
     P = shape.page_size
@@ -42,7 +42,7 @@ def run_pair(shape, Bn, N, steps, propose, verify, seed, len_lo, len_hi, min_exa
     table, free = synth.page_layout(need, num_pages, maxp, seed)
     G = shape.n_q_heads // shape.n_kv_heads
     model = B.Model(shape, B.pack_weights(shape, w), max_batch=Bn,
-                    max_rows=max(Bn * R, Bn * (64 // G)), max_position=maxp * P)
+                    max_rows=max(Bn * R, Bn * (prefill_rows or 64 // G)), max_position=maxp * P)
     if lora:
         model.load_lora(lw, rank=128)
     kv = B.KVCache(shape, num_pages, table, free)
@@ -156,3 +156,16 @@ def test_qwen3_8b_widths_two_layers():
     fp32 rounding band of a CDF boundary)."""
     run_pair(synth.QWEN3_8B_2L, 3, 4, 4, oi.ARGMAX, oi.GREEDY, seed=1, len_lo=20, len_hi=90,
              min_exact=0.5)
+
+
+@pytest.mark.parametrize("shape_name,Bn,N,verify,len_lo,len_hi", [
+    ("TINY", 3, 2, oi.STOCHASTIC, 70, 200),       # 64-row chunks, 2 attention tiles per request
+    ("QWEN3_8B_2L", 3, 4, oi.GREEDY, 90, 220),    # 64-row chunks, 4 attention tiles per request
+])
+def test_prefill_in_large_chunks(shape_name, Bn, N, verify, len_lo, len_hi):
+    """Prefill passes of 64 rows per request, whose attention runs as several
+    query tiles of the same request (pages shared): the oracle's prefill and
+    the following steps must agree as with the small chunks."""
+    shape = getattr(synth, shape_name)
+    run_pair(shape, Bn, N, 3, oi.ARGMAX, verify, seed=5, len_lo=len_lo, len_hi=len_hi,
+             min_exact=0.5, prefill_rows=64)
