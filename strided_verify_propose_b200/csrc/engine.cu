@@ -431,8 +431,6 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.k_pool = static_cast<__nv_bfloat16*>(kv->k_pool_dev);
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
-    qa.delta = nullptr;   // the adapter's delta is already in the last split
-    qa.delta_scale = c->lora_scale;
     qa.status = status;
     cudaEvent_t a0 = prof_mark(c, st);
     ISD_CUDA(isd::launch_qkv_reduce(qa, st));
@@ -454,8 +452,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
               c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
     if (rc) return rc;
     cudaEvent_t r0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st,
-                                       nullptr, 0.f, c->meta_flags));
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
     prof_add(c, kPResNorm, r0, prof_mark(c, st));
     c->launches += 1;
     // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
@@ -478,8 +475,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     if (rc) return rc;
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
     cudaEvent_t r1 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st,
-                                       nullptr, 0.f, c->meta_flags));
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
     prof_add(c, kPResNorm, r1, prof_mark(c, st));
     c->launches += 1;
   }

@@ -117,18 +117,14 @@ struct QkvReduceArgs {
   __nv_bfloat16* k_pool;
   __nv_bfloat16* v_pool;
   __nv_bfloat16* q_out;     // [rows][n_q][head_dim]
-  const float* delta;       // optional [rows][qkv_dim] gated-LoRA delta (MASK rows only)
-  float delta_scale;
   int32_t* status;
 };
 cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream);
 
-// x[row] += sum_s part[s][row] (+ delta_scale * delta[row] on MASK rows when
-// delta is given); hn[row] = bf16(RMSNorm(x[row]) * norm_w).
+// x[row] += sum_s part[s][row] (splits in order); hn[row] = bf16(RMSNorm(x[row]) * norm_w).
 cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
                                  const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
-                                 cudaStream_t stream, const float* delta = nullptr,
-                                 float delta_scale = 0.f, const int32_t* row_flags = nullptr);
+                                 cudaStream_t stream);
 
 // ---------------------------------------------------------------- gated LoRA
 cudaError_t launch_pack_rows(const __nv_bfloat16* src, int rows, int cols, __nv_bfloat16* dst,

@@ -114,22 +114,18 @@ __global__ void __launch_bounds__(256)
 
 // x[row] += sum_s part[s][row] (fixed order); hn[row] = bf16(RMSNorm(x[row]) * w).
 // Each thread holds up to kResIters float4 of the row, so every split's loads
-// are in flight together; the sum order (x, then splits ascending, then the
-// MASK-row delta) is fixed.
+// are in flight together; the sum order (x, then splits ascending) is fixed.
 constexpr int kResThreads = 256;
 constexpr int kResIters = 8;        // hidden <= 8192
 constexpr int kResMaxSplits = 8;
 
 __global__ void __launch_bounds__(kResThreads)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
-                         const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
-                         const float* delta, float delta_scale, const int32_t* row_flags) {
+                         const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   float* xr = x + static_cast<int64_t>(row) * hidden;
   const float* pr = part + static_cast<int64_t>(row) * hidden;
-  const float* dr = (delta && (row_flags[row] & kRowMask)) ? delta + static_cast<int64_t>(row) * hidden
-                                                          : nullptr;
   float4 v[kResIters];
 #pragma unroll
   for (int it = 0; it < kResIters; ++it) {
@@ -157,13 +153,6 @@ __global__ void __launch_bounds__(kResThreads)
   for (int it = 0; it < kResIters; ++it) {
     const int i = (it * kResThreads + threadIdx.x) * 4;
     if (i < hidden) {
-      if (dr) {   // gated-LoRA delta: MASK rows only
-        const float4 d = *reinterpret_cast<const float4*>(dr + i);
-        v[it].x += delta_scale * d.x;
-        v[it].y += delta_scale * d.y;
-        v[it].z += delta_scale * d.z;
-        v[it].w += delta_scale * d.w;
-      }
       *reinterpret_cast<float4*>(xr + i) = v[it];
       ss += v[it].x * v[it].x + v[it].y * v[it].y + v[it].z * v[it].z + v[it].w * v[it].w;
     }
@@ -222,11 +211,6 @@ __global__ void __launch_bounds__(kQkvWarps * 32) qkv_reduce_kernel(const QkvRed
 #pragma unroll
       for (int j = 0; j < J; ++j) v[j] += pr[sp * split_stride + 32 * j];
     }
-  }
-  if (a.delta && (flags & kRowMask)) {   // gated-LoRA delta: MASK rows only
-    const float* dr = a.delta + static_cast<int64_t>(row) * qkv_dim + hd * HD;
-#pragma unroll
-    for (int j = 0; j < J; ++j) v[j] += a.delta_scale * dr[lane + 32 * j];
   }
   if (hd < a.n_q + a.n_kv) {
     const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
@@ -308,13 +292,11 @@ cudaError_t launch_qkv_reduce(const QkvReduceArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows, int32_t hidden,
                                  const float* norm_w, float eps, float* x, __nv_bfloat16* hn,
-                                 cudaStream_t stream, const float* delta, float delta_scale,
-                                 const int32_t* row_flags) {
+                                 cudaStream_t stream) {
   if (hidden % 4 || hidden > kResThreads * 4 * kResIters || splits < 0 || splits > kResMaxSplits)
     return cudaErrorInvalidValue;
   residual_norm_kernel<<<rows, kResThreads, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
-                                                 hidden, norm_w, eps, x, hn, delta, delta_scale,
-                                                 row_flags);
+                                                         hidden, norm_w, eps, x, hn);
   return cudaGetLastError();
 }
 
