@@ -119,16 +119,19 @@ constexpr int kResThreads = 256;
 constexpr int kResIters = 8;        // hidden <= 8192
 constexpr int kResMaxSplits = 8;
 
-__global__ void __launch_bounds__(kResThreads)
+// (4 CTAs of 256 threads per SM: at most 64 registers per thread; kIters
+// float4 per thread cover hidden <= kIters * 1024)
+template <int kIters>
+__global__ void __launch_bounds__(kResThreads, 4)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
                          const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   float* xr = x + static_cast<int64_t>(row) * hidden;
   const float* pr = part + static_cast<int64_t>(row) * hidden;
-  float4 v[kResIters];
+  float4 v[kIters];
 #pragma unroll
-  for (int it = 0; it < kResIters; ++it) {
+  for (int it = 0; it < kIters; ++it) {
     const int i = (it * kResThreads + threadIdx.x) * 4;
     v[it] = i < hidden ? *reinterpret_cast<const float4*>(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kResThreads)
   for (int s = 0; s < kResMaxSplits; ++s) {
     if (s < splits) {
 #pragma unroll
-      for (int it = 0; it < kResIters; ++it) {
+      for (int it = 0; it < kIters; ++it) {
         const int i = (it * kResThreads + threadIdx.x) * 4;
         if (i < hidden) {
           const float4 d = *reinterpret_cast<const float4*>(pr + s * split_stride + i);
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(kResThreads)
   }
   float ss = 0.f;
 #pragma unroll
-  for (int it = 0; it < kResIters; ++it) {
+  for (int it = 0; it < kIters; ++it) {
     const int i = (it * kResThreads + threadIdx.x) * 4;
     if (i < hidden) {
       *reinterpret_cast<float4*>(xr + i) = v[it];
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(kResThreads)
   const float rstd = rsqrtf(tot / hidden + eps);
   __nv_bfloat16* hr = hn + static_cast<int64_t>(row) * hidden;
 #pragma unroll
-  for (int it = 0; it < kResIters; ++it) {
+  for (int it = 0; it < kIters; ++it) {
     const int i = (it * kResThreads + threadIdx.x) * 4;
     if (i < hidden) {
       const float4 w = *reinterpret_cast<const float4*>(norm_w + i);
@@ -182,7 +185,8 @@ constexpr int kQkvWarps = 16;
 constexpr int kQkvMaxSplits = 8;
 
 template <int HD>
-__global__ void __launch_bounds__(kQkvWarps * 32) qkv_reduce_kernel(const QkvReduceArgs a) {
+// (4 CTAs of 512 threads per SM: at most 32 registers per thread)
+__global__ void __launch_bounds__(kQkvWarps * 32, 4) qkv_reduce_kernel(const QkvReduceArgs a) {
   constexpr int J = HD / 32;       // values per lane
   constexpr int JH = J / 2;        // partner offset (d + HD/2)
   const int row = blockIdx.x;
@@ -295,8 +299,12 @@ cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows
                                  cudaStream_t stream) {
   if (hidden % 4 || hidden > kResThreads * 4 * kResIters || splits < 0 || splits > kResMaxSplits)
     return cudaErrorInvalidValue;
-  residual_norm_kernel<<<rows, kResThreads, 0, stream>>>(part, splits, static_cast<int64_t>(rows) * hidden,
-                                                         hidden, norm_w, eps, x, hn);
+  if (hidden <= kResThreads * 4 * 4)
+    residual_norm_kernel<4><<<rows, kResThreads, 0, stream>>>(
+        part, splits, static_cast<int64_t>(rows) * hidden, hidden, norm_w, eps, x, hn);
+  else
+    residual_norm_kernel<kResIters><<<rows, kResThreads, 0, stream>>>(
+        part, splits, static_cast<int64_t>(rows) * hidden, hidden, norm_w, eps, x, hn);
   return cudaGetLastError();
 }
 
