@@ -209,6 +209,18 @@ int isd_gemm_bf16(const void *w_dev, const void *x_dev, float *y_dev, int32_t m,
  *  each call leaves them zero, so a workspace serves any number of calls
  *  in stream order (not two calls running at once). */
 size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k);
+
+/* The tile plan the library would use for Y = X W^T with m rows, n outputs
+ * and k inputs on a GPU with num_sms SMs (host computation only; no device
+ * access). single != 0: one output slice (stream-K when the tiles overfill a
+ * wave), else up to max_splits K-splits. out[ISD_GEMM_PLAN_FIELDS] receives
+ * n_pad (token columns per CTA), token chunks, splits, K-blocks per split,
+ * MMAs per k-step, MMA N, TMA box rows, boxes, pipeline stages, 2-SM pair
+ * (0/1), stream-K (0/1), stream-K units, TMEM columns, dynamic shared
+ * memory bytes. Returns ISD_E_UNSUPPORTED when no plan exists. */
+#define ISD_GEMM_PLAN_FIELDS 14
+int isd_gemm_plan(int32_t m, int32_t n, int32_t k, int32_t single, int32_t max_splits,
+                  int32_t num_sms, int32_t *out);
 int isd_gemm_bf16_single(const void *w_dev, const void *x_dev, float *y_dev, int32_t m,
                          int32_t n, int32_t k, void *workspace_dev, size_t workspace_bytes,
                          int32_t *status_dev, void *stream);

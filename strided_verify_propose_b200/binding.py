@@ -33,7 +33,8 @@ EXPORTS = ("isd_init", "isd_load_gated_lora", "isd_step", "isd_prefill", "isd_la
            "isd_last_error", "isd_destroy", "isd_gemm_bf16", "isd_attention_workspace_bytes",
            "isd_paged_attention", "isd_accept_workspace_bytes", "isd_accept_propose",
            "isd_profile_enable", "isd_profile_read", "isd_profile_class_name",
-           "isd_accept_propose_noalloc", "isd_gemm_workspace_bytes", "isd_gemm_bf16_single")
+           "isd_accept_propose_noalloc", "isd_gemm_workspace_bytes", "isd_gemm_bf16_single",
+           "isd_gemm_plan")
 PROF_CLASSES = 16
 
 
@@ -94,6 +95,7 @@ def lib():
     L.isd_gemm_workspace_bytes.argtypes = [i32, i32, i32]
     L.isd_gemm_workspace_bytes.restype = sz
     L.isd_gemm_bf16_single.argtypes = [vp, vp, vp, i32, i32, i32, vp, sz, vp, vp]
+    L.isd_gemm_plan.argtypes = [i32, i32, i32, i32, i32, i32, C.POINTER(i32)]
     L.isd_attention_workspace_bytes.argtypes = [i32] * 7
     L.isd_attention_workspace_bytes.restype = sz
     L.isd_paged_attention.argtypes = [vp, vp, vp, vp, vp] + [i32] * 10 + [vp, vp, sz, vp, vp]
@@ -393,6 +395,19 @@ def gemm_bf16(w, x, split_k: int = 1, status=None):
     st = status if status is not None else torch.zeros(1, device=x.device, dtype=torch.int32)
     check(lib().isd_gemm_bf16(_ptr(w), _ptr(x), _ptr(y), m, n, k, split_k, _ptr(st), _stream()))
     return y
+
+
+GEMM_PLAN_FIELDS = ("n_pad", "n_chunks", "splits", "kb_per_split", "n_mma", "mma_n", "box_rows",
+                    "n_boxes", "stages", "pair", "streamk", "units", "tmem_cols", "smem_bytes")
+
+
+def gemm_plan(m: int, n: int, k: int, single: bool = False, max_splits: int = 8,
+              num_sms: int = 148) -> Optional[dict]:
+    """The library's tile plan for an m x n x k projection (host only), or None."""
+    out = (C.c_int32 * len(GEMM_PLAN_FIELDS))()
+    if lib().isd_gemm_plan(m, n, k, int(single), max_splits, num_sms, out) != 0:
+        return None
+    return dict(zip(GEMM_PLAN_FIELDS, list(out)))
 
 
 def gemm_workspace(m: int, n: int, k: int, device="cuda"):
