@@ -12,7 +12,7 @@
 // back to HBM except the q rows that SAMPLE mode must keep for the next step.
 //
 // Kernels:
-//  1. accept_stats: one CTA per (row, 8192-token chunk): running max, sum of
+//  1. accept_stats: one CTA per (row, 8192-token chunk): max, sum of
 //     exp(z - max) and the first argmax of the chunk.
 //  2. accept_decide: one CTA per request: combines the chunk statistics,
 //     runs the sequential accept tests, draws the new token by inverse CDF
@@ -62,24 +62,37 @@ __device__ __forceinline__ void merge_arg(float& v, int& i, float v2, int i2) {
 
 __global__ void __launch_bounds__(kThreads)
     accept_stats_kernel(const float* logits, int32_t vocab, int32_t n_chunks, ChunkStat* stats) {
+  // every load of the thread is issued before any arithmetic (vocab is a
+  // multiple of 4, so a float4 is either wholly inside the chunk or outside)
+  constexpr int kVec = kChunk / (kThreads * 4);
   const int c = blockIdx.x, row = blockIdx.y;
   const int lo = c * kChunk, hi = min(vocab, lo + kChunk);
   const float* z = logits + static_cast<int64_t>(row) * vocab;
-  float m = -INFINITY, s = 0.f, av = -INFINITY;
-  int ai = INT_MAX;
-  for (int i = lo + threadIdx.x * 4; i < hi; i += kThreads * 4) {
-    const float4 v4 = *reinterpret_cast<const float4*>(z + i);
-    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+  float4 v4[kVec];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      merge_arg(av, ai, v[k], i + k);
-      if (v[k] > m) {
-        s = (m == -INFINITY ? 0.f : s * expf(m - v[k])) + 1.f;
-        m = v[k];
-      } else {
-        s += expf(v[k] - m);
-      }
+  for (int j = 0; j < kVec; ++j) {
+    const int i = lo + (j * kThreads + threadIdx.x) * 4;
+    v4[j] = i < hi ? *reinterpret_cast<const float4*>(z + i)
+                   : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+  }
+  // the thread's max with its first index, then the sum of exp(z - max)
+  float av = -INFINITY;
+  int ai = INT_MAX;
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int i = lo + (j * kThreads + threadIdx.x) * 4;
+    if (i < hi) {
+      merge_arg(av, ai, v4[j].x, i);
+      merge_arg(av, ai, v4[j].y, i + 1);
+      merge_arg(av, ai, v4[j].z, i + 2);
+      merge_arg(av, ai, v4[j].w, i + 3);
     }
+  }
+  float m = av, s = 0.f;
+  if (m != -INFINITY) {
+#pragma unroll
+    for (int j = 0; j < kVec; ++j)
+      s += (expf(v4[j].x - m) + expf(v4[j].y - m)) + (expf(v4[j].z - m) + expf(v4[j].w - m));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

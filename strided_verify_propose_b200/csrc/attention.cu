@@ -480,7 +480,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 //   S^T[key][row] = K Q^T     UMMA M = 128 keys, N = 32 rows, K = 128 dims
 //   P = exp2(S * scale - m)   softmax warps: TMEM lane = key, column = row
 //   O_t^T[dim][row] = V^T P^T UMMA M = 128 dims (V read MN-major), N = 32,
-//                             K = 128 keys; P^T staged in shared memory
+//                             K = 128 keys; P^T staged in shared memory as
+//                             [key][row] (MN-major B, 64-byte swizzle), so
+//                             a thread's 16 rows of one key are two 16-byte
+//                             stores
 //   O = O * alpha + O_t       softmax warps, registers (lane = dim)
 // Warps 0-3 (one TMEM lane quadrant each) run the softmax and accumulate O;
 // warp 4 is the TMA producer, warp 5 issues the MMAs. S and O_t tiles are
@@ -495,7 +498,7 @@ constexpr int kTcThreads = (kTcSoftWarps + 2) * 32;
 constexpr int kTcStage = 2 * kTcKeys * 128 * 2;   // K and V tiles, 64 KB
 constexpr int kTcHalf = 64 * 128;                 // one [64 keys][64 dims] box, 8 KB
 constexpr int kTcQBuf = 2 * kTcNP * 128;          // Q: two 64-dim halves of NP rows, 8 KB
-constexpr int kTcPBuf = 2 * kTcNP * 128;          // P^T: two 64-key halves of NP rows, 8 KB
+constexpr int kTcPBuf = kTcKeys * kTcNP * 2;      // P^T: [128 keys][NP rows] bf16, 8 KB
 constexpr int kTcMisc = 2048;                     // reduction scratch, row state
 constexpr int kTcBars = 256;
 constexpr int kTcMinTiles = 2;                    // fewest tiles per working CTA
@@ -536,6 +539,25 @@ __device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+
+// Max of v over the 32 lanes of the warp, returned to every lane.
+__device__ __forceinline__ float warp_redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// MN-major, 64-byte swizzle: 32 MN elements per 64-byte row, rows along K
+// 64 B apart, 8-row groups 512 B apart (SBO); one 32-element MN block.
+__device__ __forceinline__ uint64_t sw64_desc_mn(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>(8192 >> 4) << 16;
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
 }
 
 __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo_bytes) {
@@ -622,7 +644,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* m_sh = red + 4 * NP;                             // running max per row (log2 units)
   float* alpha_sh = m_sh + NP;                            // [2][NP] per-tile rescale
   float* l_sh = alpha_sh + 2 * NP;                        // row sums at item end
-  int* pos_sh = reinterpret_cast<int*>(l_sh + NP);        // row positions of the item
+  float* mu_sh = l_sh + NP;                               // exponent offset (m, 0 while m = -inf)
+  int* pos_sh = reinterpret_cast<int*>(mu_sh + NP);       // row positions of the item
   int* minpos_sh = pos_sh + NP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kTcMisc);
   uint64_t* full = bars;
@@ -737,7 +760,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && fits) {
       const uint32_t idesc_s = idesc_bf16(128, NP);
-      const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15);   // A (V^T) MN-major
+      // A (V^T) and B (P^T) both MN-major
+      const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15) | (1u << 16);
       const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(qs), p_a = smem_u32(ps);
       int tc = 0, it = 0;
       int pend = -1, pend_st = 0;   // tile whose PV is not yet issued
@@ -751,7 +775,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
           const uint64_t a = sw128_desc_mn(va + (kk >> 2) * 2 * kTcHalf + (kk & 3) * 2048, kTcHalf);
-          const uint64_t bdesc = sw128_desc(p_a + (kk >> 2) * (NP * 128) + (kk & 3) * 32);
+          const uint64_t bdesc = sw64_desc_mn(p_a + kk * 16 * (NP * 2));
           umma_bf16(d, a, bdesc, idesc_o, kk > 0 ? 1u : 0u);
         }
         umma_commit(&o_full[j & 1]);
@@ -809,9 +833,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r0 = (warp >> 2) * NR;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const int kl = quad * 32 + lane;           // key within the tile; dim for O
-    // P^T store: key half kh, key kk in the half (128-byte swizzle by row)
-    const int kh = kl >> 6, kk = kl & 63;
-    uint8_t* p_col = ps + kh * (NP * 128) + (kk & 7) * 2;
+    // P^T row of this thread's key: 64 bytes, 16-byte chunks swizzled by key
+    uint8_t* p_row = ps + kl * (NP * 2);
+    const int p_sw = (kl >> 1) & 3;
     float o[NR];
     float ls[NR];
     int tc = 0;
@@ -857,21 +881,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) mbar_arrive(&s_empty[sb]);
         const int key = k_lo + t * kTcKeys + kl;
         const int last = k_lo + t * kTcKeys + kTcKeys - 1;
-        if (last < k_hi && last <= minpos) {
-#pragma unroll
-          for (int r = 0; r < NR; ++r) x[r] *= p.scale_log2;
-        } else {
+        if (!(last < k_hi && last <= minpos)) {
 #pragma unroll
           for (int r = 0; r < NR; ++r)
-            x[r] = (key < k_hi && key <= pos_sh[r0 + r]) ? x[r] * p.scale_log2 : -INFINITY;
+            if (!(key < k_hi && key <= pos_sh[r0 + r])) x[r] = -INFINITY;
         }
-        // ---- row max over the tile's 128 keys
+        // ---- row max over the tile's 128 keys (raw scores: the scale is
+        // positive, so it is applied to the max)
         {
-          float xm[NR];
+          float mx[NR];
 #pragma unroll
-          for (int r = 0; r < NR; ++r) xm[r] = x[r];
-          const float mx = lane_reduce16<true>(xm, lane);
-          if ((lane & 1) == 0) red[quad * NP + r0 + (lane >> 1)] = mx;
+          for (int r = 0; r < NR; ++r) mx[r] = warp_redux_max(x[r]);
+          if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < NR; r += 4)
+              *reinterpret_cast<float4*>(red + quad * NP + r0 + r) =
+                  make_float4(mx[r], mx[r + 1], mx[r + 2], mx[r + 3]);
+          }
         }
         // all softmax warps agree on going on (they share named barriers)
         if (!named_bar_and(2, kSoftThreads, fine)) {
@@ -881,33 +907,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (warp == 0) {
           const float m_old = m_sh[lane];
           const float mt = fmaxf(fmaxf(red[lane], red[NP + lane]), fmaxf(red[2 * NP + lane], red[3 * NP + lane]));
-          const float m_new = fmaxf(m_old, mt);
+          const float m_new = fmaxf(m_old, mt * p.scale_log2);
           alpha_sh[sb * NP + lane] = m_new == -INFINITY ? 1.f : ex2(m_old - m_new);
           m_sh[lane] = m_new;
+          // a row with no key yet: every x is -inf and 2^(x - 0) = 0
+          mu_sh[lane] = m_new == -INFINITY ? 0.f : m_new;
         }
         named_bar_sync(2, kSoftThreads);
-        // ---- P = 2^(x - m), partial row sums, P^T to shared memory
+        // ---- P = 2^(x scale - m), partial row sums, P^T to shared memory
         // (all shared-memory reads first: a store between them would
         // serialise every row on the possible aliasing)
 #pragma unroll
         for (int r = 0; r < NR; r += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(m_sh + r0 + r);
+          const float4 m4 = *reinterpret_cast<const float4*>(mu_sh + r0 + r);
           const float4 a4 = *reinterpret_cast<const float4*>(alpha_sh + sb * NP + r0 + r);
           const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
           const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float e = mm[i] == -INFINITY ? 0.f : ex2(x[r + i] - mm[i]);
+            const float e = ex2(fmaf(x[r + i], p.scale_log2, -mm[i]));
             ls[r + i] = ls[r + i] * aa[i] + e;
             x[r + i] = e;
           }
         }
         fine = fine && mbar_wait(p_empty, (tc & 1) ^ 1);
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const int row = r0 + r;
-          *reinterpret_cast<__nv_bfloat16*>(p_col + row * 128 + (((kk >> 3) ^ (row & 7)) << 4)) =
-              __float2bfloat16_rn(x[r]);
+        {
+          // rows r0 .. r0 + 7 and r0 + 8 .. r0 + 15: 16-byte chunks r0/8 and r0/8 + 1
+          const uint4 c0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
+                                      pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+          const uint4 c1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
+                                      pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
+          const int ch = r0 >> 3;
+          *reinterpret_cast<uint4*>(p_row + ((ch ^ p_sw) << 4)) = c0;
+          *reinterpret_cast<uint4*>(p_row + (((ch + 1) ^ p_sw) << 4)) = c1;
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
