@@ -485,23 +485,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 //                             a thread's 16 rows of one key are two 16-byte
 //                             stores
 //   O = O * alpha + O_t       softmax warps, registers (lane = dim)
-// Warps 0-3 (one TMEM lane quadrant each) run the softmax and accumulate O;
-// warp 4 is the TMA producer, warp 5 issues the MMAs. S and O_t tiles are
-// double-buffered in tensor memory, so the MMA of tile t+1 runs while the
-// softmax warps work on tile t. Items, splits and the partial-sum format are
-// those of the mma.sync kernel; the same combine kernel finishes.
+// Warps 0-7 (two per TMEM lane quadrant) run the softmax and accumulate O;
+// warp 8 is the TMA producer, warp 9 issues the S MMAs and warp 10 the PV
+// MMAs, so neither kind waits behind the other. S and O_t tiles are
+// double-buffered in tensor memory: the S MMA of tile t+1 runs while the
+// softmax warps work on tile t. K and V tiles sit in separate rings: a K
+// slot is free again as soon as S has been computed from it, and only the V
+// slot is held through the softmax, which keeps more of the ring's bytes in
+// flight from HBM. Each contraction accumulates into two column blocks (S:
+// dims 0-63 and 64-127; PV: keys 0-63 and 64-127) issued alternately: one
+// chain of dependent small MMAs is latency-bound, two interleaved chains are
+// not, and the softmax warps add the two halves as they read them. The row
+// positions of the next work segment are loaded while the current one runs.
+// The work split and the partial-sum format are shared with the mma.sync
+// kernel; the same combine kernel finishes.
 constexpr int kTcKeys = 128;                 // keys per tile (two 64-key pages)
 constexpr int kTcNP = 32;                    // query rows per tile (UMMA N)
 constexpr int kTcSoftWarps = 8;              // two per TMEM lane quadrant
 constexpr int kTcRows = kTcNP / 2;           // query rows per softmax warp
-constexpr int kTcThreads = (kTcSoftWarps + 2) * 32;
-constexpr int kTcStage = 2 * kTcKeys * 128 * 2;   // K and V tiles, 64 KB
+constexpr int kTcThreads = (kTcSoftWarps + 3) * 32;
+constexpr int kTcSlot = kTcKeys * 128 * 2;        // one K or V tile, 32 KB
+constexpr int kTcStage = 2 * kTcSlot;             // a K slot and a V slot, 64 KB
 constexpr int kTcHalf = 64 * 128;                 // one [64 keys][64 dims] box, 8 KB
 constexpr int kTcQBuf = 2 * kTcNP * 128;          // Q: two 64-dim halves of NP rows, 8 KB
 constexpr int kTcPBuf = kTcKeys * kTcNP * 2;      // P^T: [128 keys][NP rows] bf16, 8 KB
 constexpr int kTcMisc = 2048;                     // reduction scratch, row state
 constexpr int kTcBars = 256;
 constexpr int kTcMinTiles = 2;                    // fewest tiles per working CTA
+constexpr int kTcMaxStages = (kTcBars / 8 - 16) / 4;   // barriers: 4 per stage + 16
 
 // Max or sum of v[0..15] over the 32 lanes, reduce-scatter style: after 16
 // shuffles lanes 2i and 2i+1 both hold the reduction of value i.
@@ -573,58 +584,81 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo_by
   return d;
 }
 
-// Work of the tcgen05 kernel: the tiles of all (request, KV head) pairs in
-// one sequence, request-major, then head, then tile; CTA c of the C working
-// CTAs takes tiles [c T / C, (c+1) T / C). A maximal run of one (request,
-// head) inside a CTA's range is a segment; it leaves its partial output in
-// slot (b * nkv + g) * max_parts + (c - first CTA of that pair).
+// Work of the tcgen05 kernel: the (request, KV head) pairs in one sequence,
+// request-major, then head. Pair (b, g) occupies nt_b + kTcSegCost units: the
+// first kTcSegCost stand for the fixed cost of starting and finishing a
+// segment (row state, partial-output write, the pipeline drain at its end),
+// then one unit per 128-key tile. CTA c of the C working CTAs takes units
+// [c U / C, (c+1) U / C), so a CTA whose range crosses many short pairs gets
+// fewer tiles. A maximal run of one pair's tiles inside a CTA's range is a
+// segment; it leaves its partial output in slot (b * nkv + g) * max_parts +
+// (c - the CTA of the pair's first tile).
+constexpr int kTcSegCost = 2;
+
 struct TcSeg {
   int b, g, t0, len, slot;
 };
 
 struct TcRange {
-  int64_t x, hi, T;
+  int64_t x, hi, U;
   int C;
 };
 
 __device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
 
-__device__ __forceinline__ int tc_cta_of(int64_t x, int64_t T, int C) {
-  return static_cast<int>(((x + 1) * C - 1) / T);
+__device__ __forceinline__ int tc_cta_of(int64_t x, int64_t U, int C) {
+  return static_cast<int>(((x + 1) * C - 1) / U);
 }
 
-// tile prefix per request in base[0..B] (base[b] = tiles before request b)
+// First unit of request b (base[b] = 128-key tiles of the requests before b).
+__device__ __forceinline__ int64_t tc_ubase(const AttnParams& p, const int* base, int b) {
+  return static_cast<int64_t>(p.nkv) * (base[b] + static_cast<int64_t>(kTcSegCost) * b);
+}
+
+// Working CTAs: each takes at least min_tiles units.
+__device__ __forceinline__ int tc_ctas(const AttnParams& p, int64_t U, int grid) {
+  return static_cast<int>(i64max(1, i64min(grid, U / p.min_tiles)));
+}
+
 __device__ __forceinline__ TcRange tc_range(const AttnParams& p, const int* base) {
   TcRange r;
-  r.T = static_cast<int64_t>(p.nkv) * base[p.B];
-  r.C = static_cast<int>(i64max(1, i64min(gridDim.x, r.T / p.min_tiles)));
+  r.U = tc_ubase(p, base, p.B);
+  r.C = tc_ctas(p, r.U, gridDim.x);
   const int c = blockIdx.x;
-  r.x = c < r.C ? c * r.T / r.C : 0;
-  r.hi = c < r.C ? (c + 1) * r.T / r.C : 0;
+  r.x = c < r.C ? c * r.U / r.C : 0;
+  r.hi = c < r.C ? (c + 1) * r.U / r.C : 0;
   return r;
 }
 
 __device__ __forceinline__ bool tc_next(const AttnParams& p, const int* base, TcRange& r, TcSeg& sg) {
-  if (r.x >= r.hi) return false;
-  int lo = 0, hi = p.B;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (static_cast<int64_t>(base[mid]) * p.nkv <= r.x) lo = mid; else hi = mid;
+  while (r.x < r.hi) {
+    int lo = 0, hi = p.B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tc_ubase(p, base, mid) <= r.x) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int nt = base[b + 1] - base[b];
+    const int w = nt + kTcSegCost;
+    const int64_t x0b = tc_ubase(p, base, b);
+    const int rem = static_cast<int>(r.x - x0b);
+    const int g = rem / w, off = rem % w;
+    const int64_t first = x0b + static_cast<int64_t>(g) * w + kTcSegCost;   // the pair's first tile
+    if (off < kTcSegCost) {
+      r.x = first;   // start of the pair's tiles (of the next pair when nt = 0)
+      continue;
+    }
+    sg.b = b;
+    sg.g = g;
+    sg.t0 = off - kTcSegCost;
+    sg.len = static_cast<int>(i64min(r.hi - r.x, nt - sg.t0));
+    const int part = static_cast<int>(blockIdx.x) - tc_cta_of(first, r.U, r.C);
+    sg.slot = part < p.max_parts ? (b * p.nkv + sg.g) * p.max_parts + part : -1;
+    r.x += sg.len;
+    return true;
   }
-  const int b = lo;
-  const int nt = base[b + 1] - base[b];
-  const int64_t x0b = static_cast<int64_t>(base[b]) * p.nkv;
-  const int rem = static_cast<int>(r.x - x0b);
-  sg.b = b;
-  sg.g = rem / nt;
-  sg.t0 = rem % nt;
-  sg.len = static_cast<int>(i64min(r.hi - r.x, nt - sg.t0));
-  const int64_t first = x0b + static_cast<int64_t>(sg.g) * nt;
-  const int part = static_cast<int>(blockIdx.x) - tc_cta_of(first, r.T, r.C);
-  sg.slot = part < p.max_parts ? (b * p.nkv + sg.g) * p.max_parts + part : -1;
-  r.x += sg.len;
-  return true;
+  return false;
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -637,8 +671,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* ring = smem;                                   // stages x [K | V]
-  uint8_t* qs = ring + p.stages * kTcStage;               // 2 x Q
+  uint8_t* ring_k = smem;                                 // stages x K tile
+  uint8_t* ring_v = ring_k + p.stages * kTcSlot;          // stages x V tile
+  uint8_t* qs = ring_v + p.stages * kTcSlot;              // 2 x Q
   uint8_t* ps = qs + 2 * kTcQBuf;                         // P^T
   float* red = reinterpret_cast<float*>(ps + kTcPBuf);    // [4 quadrants][NP]
   float* m_sh = red + 4 * NP;                             // running max per row (log2 units)
@@ -648,9 +683,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* pos_sh = reinterpret_cast<int*>(mu_sh + NP);       // row positions of the item
   int* minpos_sh = pos_sh + NP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kTcMisc);
-  uint64_t* full = bars;
-  uint64_t* empty = full + p.stages;
-  uint64_t* q_full = empty + p.stages;     // [2]
+  uint64_t* full_k = bars;                 // [stages] each
+  uint64_t* empty_k = full_k + p.stages;
+  uint64_t* full_v = empty_k + p.stages;
+  uint64_t* empty_v = full_v + p.stages;
+  uint64_t* q_full = empty_v + p.stages;   // [2]
   uint64_t* q_empty = q_full + 2;          // [2]
   uint64_t* s_full = q_empty + 2;          // [2]
   uint64_t* s_empty = s_full + 2;          // [2]
@@ -658,15 +695,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* o_empty = o_full + 2;          // [2]
   uint64_t* p_full = o_empty + 2;
   uint64_t* p_empty = p_full + 1;
-  uint64_t* drain = p_empty + 1;
+  uint64_t* drain = p_empty + 1;           // [2]: S issuer, PV issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + kTcBars);
   int* kend = reinterpret_cast<int*>(tmem_slot + 4);
   int* base = kend + p.B;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.stages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&full_k[i], 1);
+      mbar_init(&empty_k[i], 1);
+      mbar_init(&full_v[i], 1);
+      mbar_init(&empty_v[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
@@ -678,7 +717,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(p_full, kTcSoftWarps);
     mbar_init(p_empty, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     fence_barrier_init();
   }
   // query rows past the tile's RG rows are never loaded: keep them zero
@@ -686,7 +726,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     reinterpret_cast<int4*>(qs)[i] = make_int4(0, 0, 0, 0);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 4 * NP);
+    tmem_alloc(tmem_slot, 8 * NP);
     tmem_relinquish();
     tc_fence_before();
   }
@@ -701,7 +741,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == kTcSoftWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && fits) {
-      int tc = 0, it = 0, q_issued = 0;
+      int tc = 0, it = 0, q_issued = 0, nk = 0;
       bool ok = true;
       TcRange rg = tc_range(p, base);
       TcSeg sg;
@@ -723,66 +763,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int32_t* pt = p.page_table + static_cast<int64_t>(b) * p.maxp;
         for (int t = 0; t < n_tiles; ++t, ++tc) {
           const int st = tc % p.stages;
-          if (!mbar_wait(&empty[st], ((tc / p.stages) & 1) ^ 1)) {
-            ok = false;
-            break;
-          }
-          uint8_t* ks = ring + st * kTcStage;
-          uint8_t* vs = ks + kTcStage / 2;
-          mbar_arrive_expect_tx(&full[st], kTcStage);
+          const uint32_t ph = ((tc / p.stages) & 1) ^ 1;
+          int rows[2];
           for (int j = 0; j < 2; ++j) {
             const int key0 = k_lo + t * kTcKeys + j * 64;
-            int row = p.oob_row;
+            rows[j] = p.oob_row;
             if (key0 < k_hi) {
               const int page = pt[key0 / 64];
               if (page >= 0 && page < p.num_pages)
-                row = ((p.layer * p.num_pages + page) * p.nkv + g) * 64;
+                rows[j] = ((p.layer * p.num_pages + page) * p.nkv + g) * 64;
               else
                 flag(p.status, ISD_DEV_BAD_PAGE);
             }
-            for (int hh = 0; hh < 2; ++hh) {
-              // K as [dim half][page][64 keys][64 dims]: the 128 keys of a
-              // dim half are one K-major operand; V as [page][dim half]:
-              // each page is 16 keys per MMA k-step, dim halves LBO apart.
-              tma_load_2d(ks + hh * 2 * kTcHalf + j * kTcHalf, &kmap, &full[st], hh * 64, row);
-              tma_load_2d(vs + j * 2 * kTcHalf + hh * kTcHalf, &vmap, &full[st], hh * 64, row);
-            }
           }
+          // K as [dim half][page][64 keys][64 dims]: the 128 keys of a dim
+          // half are one K-major operand
+          if (!mbar_wait(&empty_k[st], ph)) {
+            ok = false;
+            break;
+          }
+          uint8_t* ks = ring_k + st * kTcSlot;
+          mbar_arrive_expect_tx(&full_k[st], kTcSlot);
+          for (int j = 0; j < 2; ++j)
+            for (int hh = 0; hh < 2; ++hh)
+              tma_load_2d(ks + hh * 2 * kTcHalf + j * kTcHalf, &kmap, &full_k[st], hh * 64, rows[j]);
+          ++nk;
+          // V as [page][dim half]: each page is 16 keys per MMA k-step, dim
+          // halves LBO apart
+          if (!mbar_wait(&empty_v[st], ph)) {
+            ok = false;
+            break;
+          }
+          uint8_t* vs = ring_v + st * kTcSlot;
+          mbar_arrive_expect_tx(&full_v[st], kTcSlot);
+          for (int j = 0; j < 2; ++j)
+            for (int hh = 0; hh < 2; ++hh)
+              tma_load_2d(vs + j * 2 * kTcHalf + hh * kTcHalf, &vmap, &full_v[st], hh * 64, rows[j]);
         }
       }
       if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
-      // copies in flight land before the CTA exits
+      // copies in flight land before the CTA exits (after a timeout the last
+      // K load may have no V load beside it)
+      for (int j = max(0, nk - p.stages); j < nk; ++j)
+        if (!mbar_wait(&full_k[j % p.stages], (j / p.stages) & 1)) break;
       for (int j = max(0, tc - p.stages); j < tc; ++j)
-        if (!mbar_wait(&full[j % p.stages], (j / p.stages) & 1)) break;
+        if (!mbar_wait(&full_v[j % p.stages], (j / p.stages) & 1)) break;
       if (q_issued > 0) mbar_wait(&q_full[(q_issued - 1) & 1], ((q_issued - 1) >> 1) & 1);
     }
   } else if (warp == kTcSoftWarps + 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
     if (lane == 0 && fits) {
       const uint32_t idesc_s = idesc_bf16(128, NP);
-      // A (V^T) and B (P^T) both MN-major
-      const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15) | (1u << 16);
-      const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(qs), p_a = smem_u32(ps);
+      const uint32_t rk_a = smem_u32(ring_k), q_a = smem_u32(qs);
       int tc = 0, it = 0;
-      int pend = -1, pend_st = 0;   // tile whose PV is not yet issued
       bool ok = true;
-      auto issue_pv = [&](int j, int st) -> bool {
-        if (!mbar_wait(p_full, j & 1)) return false;
-        if (!mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + 2 * NP + (j & 1) * NP;
-        const uint32_t va = ring_a + st * kTcStage + kTcStage / 2;
-#pragma unroll
-        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-          const uint64_t a = sw128_desc_mn(va + (kk >> 2) * 2 * kTcHalf + (kk & 3) * 2048, kTcHalf);
-          const uint64_t bdesc = sw64_desc_mn(p_a + kk * 16 * (NP * 2));
-          umma_bf16(d, a, bdesc, idesc_o, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&o_full[j & 1]);
-        umma_commit(&empty[st]);
-        umma_commit(p_empty);
-        return true;
-      };
       TcRange rg = tc_range(p, base);
       TcSeg sg;
       for (; ok && tc_next(p, base, rg, sg); ++it) {
@@ -792,41 +826,78 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
+        const uint64_t b0 = sw128_desc(q_a + qb * kTcQBuf);
         for (int t = 0; t < n_tiles; ++t, ++tc) {
           const int st = tc % p.stages;
-          if (!mbar_wait(&full[st], (tc / p.stages) & 1) ||
+          if (!mbar_wait(&full_k[st], (tc / p.stages) & 1) ||
               !mbar_wait(&s_empty[tc & 1], ((tc >> 1) & 1) ^ 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + (tc & 1) * NP;
-          const uint32_t ka = ring_a + st * kTcStage;
+          // dims 0-63 and 64-127 accumulate into two column blocks, issued
+          // alternately so that consecutive MMAs do not depend on each other
+          const uint32_t d = tmem + (tc & 1) * 2 * NP;
+          const uint64_t a0 = sw128_desc(rk_a + st * kTcSlot);
+          // descriptor start addresses count 16-byte units
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint64_t a = sw128_desc(ka + (kk >> 2) * 2 * kTcHalf + (kk & 3) * 32);
-            const uint64_t bdesc = sw128_desc(q_a + qb * kTcQBuf + (kk >> 2) * (NP * 128) + (kk & 3) * 32);
-            umma_bf16(d, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+          for (int i = 0; i < 128 / 16; ++i) {
+            const int hh = i & 1, kk = i >> 1;
+            umma_bf16(d + hh * NP, a0 + ((hh * 2 * kTcHalf + kk * 32) >> 4),
+                      b0 + ((hh * (NP * 128) + kk * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[tc & 1]);
-          if (pend >= 0 && !issue_pv(pend, pend_st)) {
-            ok = false;
-            break;
-          }
-          pend = tc;
-          pend_st = st;
+          umma_commit(&empty_k[st]);
         }
         if (!ok) break;
         umma_commit(&q_empty[qb]);   // this item's S MMAs are the last readers of Q
       }
-      if (ok && pend >= 0 && !issue_pv(pend, pend_st)) ok = false;
       if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
       // every MMA has finished before tensor memory is freed
-      umma_commit(drain);
-      mbar_wait(drain, 0);
+      umma_commit(&drain[0]);
+      mbar_wait(&drain[0], 0);
+    }
+  } else if (warp == kTcSoftWarps + 2) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0 && fits) {
+      // A (V^T) and B (P^T) both MN-major
+      const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15) | (1u << 16);
+      const uint32_t rv_a = smem_u32(ring_v);
+      const uint64_t b0 = sw64_desc_mn(smem_u32(ps));
+      int n_total = 0;
+      {
+        TcRange rg = tc_range(p, base);
+        TcSeg sg;
+        while (tc_next(p, base, rg, sg)) n_total += sg.len;
+      }
+      bool ok = true;
+      for (int j = 0; j < n_total; ++j) {
+        const int st = j % p.stages;
+        if (!mbar_wait(p_full, j & 1) || !mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1) ||
+            !mbar_wait(&full_v[st], (j / p.stages) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // keys 0-63 and 64-127 accumulate into two column blocks, alternately
+        const uint32_t d = tmem + 4 * NP + (j & 1) * 2 * NP;
+        const uint64_t a0 = sw128_desc_mn(rv_a + st * kTcSlot, kTcHalf);
+#pragma unroll
+        for (int i = 0; i < kTcKeys / 16; ++i) {
+          const int jj = i & 1, kk = i >> 1;   // page jj, 16-key step kk in it
+          umma_bf16(d + jj * NP, a0 + ((jj * 2 * kTcHalf + kk * 2048) >> 4),
+                    b0 + (((jj * 4 + kk) * 16 * (NP * 2)) >> 4), idesc_o, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&o_full[j & 1]);
+        umma_commit(&empty_v[st]);
+        umma_commit(p_empty);
+      }
+      if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
+      umma_commit(&drain[1]);
+      mbar_wait(&drain[1], 0);
     }
   } else if (fits) {
-    // -------------------------------------------- softmax / accumulate warps
+    // ------------------------ softmax / accumulate warps (0 .. kTcSoftWarps - 1)
     // warp w: TMEM lane quadrant w % 4 (keys of S, dims of O) and query
     // rows r0 .. r0 + 15 (TMEM columns), r0 = 16 * (w / 4)
     const int quad = warp & 3;
@@ -842,13 +913,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool fine = true;
     TcRange rg = tc_range(p, base);
     TcSeg sg;
-    while (tc_next(p, base, rg, sg)) {
+    bool have = tc_next(p, base, rg, sg);
+    // row positions are loaded one segment ahead (warp 0, lane = row)
+    int pr_cur = warp == 0 && have && lane < p.RG ? p.row_pos[sg.b * p.R + lane / p.G] : -1;
+    while (have) {
+      TcSeg nx;
+      const bool have_nx = tc_next(p, base, rg, nx);
+      const int pr_nx =
+          warp == 0 && have_nx && lane < p.RG ? p.row_pos[nx.b * p.R + lane / p.G] : -1;
       const int b = sg.b;
       const int k_lo = sg.t0 * kTcKeys;
       const int k_hi = min(kend[b], k_lo + sg.len * kTcKeys);
       const int n_tiles = sg.len;
       if (warp == 0) {
-        const int pr = lane < p.RG ? p.row_pos[b * p.R + lane / p.G] : -1;
+        const int pr = pr_cur;
         pos_sh[lane] = pr;
         m_sh[lane] = -INFINITY;
         int mn = lane < p.RG ? pr : INT_MAX;
@@ -870,11 +948,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after();
         float x[NR];
         {
-          uint32_t r16[16];
-          tmem_ld_32x32_x16(lane_base + sb * NP + r0, r16);
+          uint32_t ra[16], rb[16];
+          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + r0, ra);
+          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + NP + r0, rb);
           tmem_ld_wait();
 #pragma unroll
-          for (int r = 0; r < NR; ++r) x[r] = __uint_as_float(r16[r]);
+          for (int r = 0; r < NR; ++r) x[r] = __uint_as_float(ra[r]) + __uint_as_float(rb[r]);
         }
         tc_fence_before();
         __syncwarp();
@@ -949,15 +1028,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int j = tc - 1;
           fine = fine && mbar_wait(&o_full[j & 1], (j >> 1) & 1);
           tc_fence_after();
-          uint32_t r16[16];
-          tmem_ld_32x32_x16(lane_base + 2 * NP + (j & 1) * NP + r0, r16);
+          uint32_t ra[16], rb[16];
+          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0, ra);
+          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0, rb);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&o_empty[j & 1]);
 #pragma unroll
           for (int r = 0; r < NR; ++r)
-            o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] + __uint_as_float(r16[r]);
+            o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] +
+                   (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
         }
       }
       if (!fine) break;
@@ -965,15 +1046,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int j = tc - 1;
         fine = mbar_wait(&o_full[j & 1], (j >> 1) & 1);
         tc_fence_after();
-        uint32_t r16[16];
-        tmem_ld_32x32_x16(lane_base + 2 * NP + (j & 1) * NP + r0, r16);
+        uint32_t ra[16], rb[16];
+        tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0, ra);
+        tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0, rb);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&o_empty[j & 1]);
 #pragma unroll
         for (int r = 0; r < NR; ++r)
-          o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] + __uint_as_float(r16[r]);
+          o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] +
+                 (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
       }
       // ---- row sums over the 128 key lanes, then the partial output
       {
@@ -1002,6 +1085,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       named_bar_sync(2, kSoftThreads);   // row state is rewritten by the next segment
+      sg = nx;
+      have = have_nx;
+      pr_cur = pr_nx;
     }
     if (!fine && lane == 0) flag(p.status, ISD_DEV_TIMEOUT);
   }
@@ -1009,7 +1095,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 4 * NP);
+    tmem_dealloc(tmem, 8 * NP);
   }
 }
 
@@ -1071,13 +1157,13 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p
   const int g = blockIdx.x, b = blockIdx.y;
   __shared__ float w[kTcNP][kMaxSplits];
   const int* base = p.item_base;
-  const int64_t T = static_cast<int64_t>(p.nkv) * base[p.B];
+  const int64_t U = tc_ubase(p, base, p.B);
   const int nt = base[b + 1] - base[b];
   int parts = 0;
-  if (nt > 0 && T > 0) {
-    const int C = static_cast<int>(i64max(1, i64min(C_grid, T / p.min_tiles)));
-    const int64_t first = static_cast<int64_t>(base[b]) * p.nkv + static_cast<int64_t>(g) * nt;
-    parts = tc_cta_of(first + nt - 1, T, C) - tc_cta_of(first, T, C) + 1;
+  if (nt > 0) {
+    const int C = tc_ctas(p, U, C_grid);
+    const int64_t first = tc_ubase(p, base, b) + static_cast<int64_t>(g) * (nt + kTcSegCost) + kTcSegCost;
+    parts = tc_cta_of(first + nt - 1, U, C) - tc_cta_of(first, U, C) + 1;
   }
   if (parts > p.max_parts || parts > kMaxSplits) {
     if (threadIdx.x == 0) flag(p.status, ISD_DEV_BAD_STATE);
@@ -1149,7 +1235,7 @@ Derived derive(const AttnShape& s) {
     d.max_items = s.batch * s.n_kv_heads * d.max_splits;
     d.MT = kTcNP / 16;
     d.NG = 1;
-    d.stages = 4;
+    d.stages = kTcMaxStages;
     while (d.stages > 2 && tc_smem(d.stages, s.batch) > 232448) --d.stages;
     d.smem = tc_smem(d.stages, s.batch);
     return d;
