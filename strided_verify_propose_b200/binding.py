@@ -430,17 +430,28 @@ def gemm_bf16_single(w, x, workspace=None, status=None):
     return y
 
 
+def attention_workspace(batch: int, rows_per_req: int, n_q: int, n_kv: int, head_dim: int,
+                        max_pages_per_req: int, page_size: int, device="cuda"):
+    """Workspace for isd_paged_attention at these sizes (scratch only: any
+    later launch that fits may reuse it)."""
+    import torch
+    n = int(lib().isd_attention_workspace_bytes(batch, rows_per_req, n_q, n_kv, head_dim,
+                                                max_pages_per_req, page_size))
+    return torch.empty(n, device=device, dtype=torch.uint8)
+
+
 def paged_attention(q, row_pos, k_pool, v_pool, page_table, rows_per_req: int, layer: int = 0,
-                    status=None):
-    """Attention of rows q [B*R, n_q, hd] over the paged pools (torch device tensors)."""
+                    status=None, workspace=None):
+    """Attention of rows q [B*R, n_q, hd] over the paged pools (torch device
+    tensors). workspace: from attention_workspace, else a fresh one."""
     import torch
     n_layers, num_pages, n_kv, page_size, hd = k_pool.shape
     rows, n_q, _ = q.shape
     B = rows // rows_per_req
     maxp = page_table.shape[1]
-    ws_bytes = int(lib().isd_attention_workspace_bytes(B, rows_per_req, n_q, n_kv, hd, maxp,
-                                                       page_size))
-    ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    ws = workspace if workspace is not None else attention_workspace(
+        B, rows_per_req, n_q, n_kv, hd, maxp, page_size, q.device)
+    ws_bytes = ws.numel()
     out = torch.empty(rows, n_q * hd, device=q.device, dtype=torch.bfloat16)
     st = status if status is not None else torch.zeros(1, device=q.device, dtype=torch.int32)
     check(lib().isd_paged_attention(_ptr(q), _ptr(row_pos), _ptr(k_pool), _ptr(v_pool),
