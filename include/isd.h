@@ -242,6 +242,31 @@ int isd_paged_attention(const void *q_dev, const int32_t *row_pos_dev, const voi
                         void *out_dev, void *workspace_dev, size_t workspace_bytes,
                         int32_t *status_dev, void *stream);
 
+/* Host-only query of the work split of the tcgen05 attention kernel (head_dim
+ * 128, 64-key pages, at most 32 query rows per KV head): no GPU work. The
+ * kernel runs one CTA per SM over the (request, KV head, 128-key tile)
+ * sequence; each CTA takes a contiguous range in which every (request, KV
+ * head) segment counts as 2 tiles besides its own tiles, and a pair cut
+ * between CTAs leaves one partial per CTA, merged in CTA order (paged
+ * attention on tensor cores, a block's queries against its request's paged
+ * prefix; Bud's Wiki "Introspective Diffusion Language Models", Method).
+ *  kend_host [batch]: keys visible to each request's last row (its largest
+ *  row position + 1; clipped to max_pages_per_req * page_size as the kernel
+ *  does). num_sms: CTAs of the launch.
+ *  seg_out [seg_capacity][ISD_ATTN_SEG_FIELDS]: per segment, in CTA order:
+ *  CTA, request, KV head, first tile, tiles, partial slot ((request * n_kv +
+ *  head) * max_parts + part; -1 if part >= max_parts, which a valid split
+ *  never produces). *n_segments: the segments (also when capacity is short);
+ *  *max_parts: the partial slots per (request, KV head).
+ * Returns ISD_OK, ISD_E_UNSUPPORTED for shapes the tcgen05 kernel does not
+ * serve, ISD_E_INVALID for bad arguments or a short seg_capacity. */
+#define ISD_ATTN_SEG_FIELDS 6
+int isd_attention_split(int32_t batch, int32_t rows_per_req, int32_t n_q_heads,
+                        int32_t n_kv_heads, int32_t head_dim, int32_t max_pages_per_req,
+                        int32_t page_size, const int32_t *kend_host, int32_t num_sms,
+                        int32_t *seg_out, int32_t seg_capacity, int32_t *n_segments,
+                        int32_t *max_parts);
+
 /* Verify / resample / propose from given block logits, then the length and
  * page bookkeeping: the tail of isd_step without the forward.
  *  logits_dev [B*(2N-1)][vocab] fp32; other arguments as in isd_step (kv

@@ -18,6 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libisd.so")
 
 ISD_OK = 0
+ISD_E_INVALID, ISD_E_UNSUPPORTED = -1, -2
 ISD_DEV_POOL_EXHAUSTED = 0x01
 ISD_DEV_TABLE_FULL = 0x02
 ISD_DEV_BAD_TOKEN = 0x04
@@ -34,7 +35,7 @@ EXPORTS = ("isd_init", "isd_load_gated_lora", "isd_step", "isd_prefill", "isd_la
            "isd_paged_attention", "isd_accept_workspace_bytes", "isd_accept_propose",
            "isd_profile_enable", "isd_profile_read", "isd_profile_class_name",
            "isd_accept_propose_noalloc", "isd_gemm_workspace_bytes", "isd_gemm_bf16_single",
-           "isd_gemm_plan")
+           "isd_gemm_plan", "isd_attention_split")
 PROF_CLASSES = 16
 
 
@@ -96,6 +97,8 @@ def lib():
     L.isd_gemm_workspace_bytes.restype = sz
     L.isd_gemm_bf16_single.argtypes = [vp, vp, vp, i32, i32, i32, vp, sz, vp, vp]
     L.isd_gemm_plan.argtypes = [i32, i32, i32, i32, i32, i32, C.POINTER(i32)]
+    L.isd_attention_split.argtypes = [i32] * 7 + [C.POINTER(i32), i32, C.POINTER(i32), i32,
+                                                  C.POINTER(i32), C.POINTER(i32)]
     L.isd_attention_workspace_bytes.argtypes = [i32] * 7
     L.isd_attention_workspace_bytes.restype = sz
     L.isd_paged_attention.argtypes = [vp, vp, vp, vp, vp] + [i32] * 10 + [vp, vp, sz, vp, vp]
@@ -408,6 +411,32 @@ def gemm_plan(m: int, n: int, k: int, single: bool = False, max_splits: int = 8,
     if lib().isd_gemm_plan(m, n, k, int(single), max_splits, num_sms, out) != 0:
         return None
     return dict(zip(GEMM_PLAN_FIELDS, list(out)))
+
+
+ATTN_SEG_FIELDS = ("cta", "request", "kv_head", "tile0", "tiles", "slot")
+
+
+def attention_split(batch: int, rows_per_req: int, n_q: int, n_kv: int, head_dim: int,
+                    max_pages_per_req: int, page_size: int, kend, num_sms: int = 148):
+    """The tcgen05 attention kernel's work split (host only): an int32 array
+    [segments][ATTN_SEG_FIELDS] in CTA order and the partial slots per
+    (request, KV head); None when that kernel does not serve the shape."""
+    import numpy as np
+    ke = np.ascontiguousarray(np.asarray(kend, dtype=np.int32))
+    if ke.shape != (batch,):
+        raise ValueError("kend needs one key count per request")
+    kp = ke.ctypes.data_as(C.POINTER(C.c_int32))
+    n, mp = C.c_int32(0), C.c_int32(0)
+    L = lib()
+    rc = L.isd_attention_split(batch, rows_per_req, n_q, n_kv, head_dim, max_pages_per_req,
+                               page_size, kp, num_sms, None, 0, C.byref(n), C.byref(mp))
+    if rc == ISD_E_UNSUPPORTED:
+        return None
+    seg = np.zeros((max(n.value, 1), len(ATTN_SEG_FIELDS)), np.int32)
+    check(L.isd_attention_split(batch, rows_per_req, n_q, n_kv, head_dim, max_pages_per_req,
+                                page_size, kp, num_sms, seg.ctypes.data_as(C.POINTER(C.c_int32)),
+                                seg.shape[0], C.byref(n), C.byref(mp)))
+    return seg[:n.value], mp.value
 
 
 def gemm_workspace(m: int, n: int, k: int, device="cuda"):

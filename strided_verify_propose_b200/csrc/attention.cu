@@ -18,6 +18,7 @@
 #include <algorithm>
 #include <cstdlib>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -601,37 +602,42 @@ struct TcSeg {
 
 struct TcRange {
   int64_t x, hi, U;
-  int C;
+  int C, c;   // working CTAs; this CTA
 };
 
-__device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
-__device__ __forceinline__ int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
+// The split functions serve the kernel and, unchanged, the host-side query
+// isd_attention_split.
+__host__ __device__ __forceinline__ int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
 
-__device__ __forceinline__ int tc_cta_of(int64_t x, int64_t U, int C) {
+__host__ __device__ __forceinline__ int tc_cta_of(int64_t x, int64_t U, int C) {
   return static_cast<int>(((x + 1) * C - 1) / U);
 }
 
 // First unit of request b (base[b] = 128-key tiles of the requests before b).
-__device__ __forceinline__ int64_t tc_ubase(const AttnParams& p, const int* base, int b) {
+__host__ __device__ __forceinline__ int64_t tc_ubase(const AttnParams& p, const int* base, int b) {
   return static_cast<int64_t>(p.nkv) * (base[b] + static_cast<int64_t>(kTcSegCost) * b);
 }
 
 // Working CTAs: each takes at least min_tiles units.
-__device__ __forceinline__ int tc_ctas(const AttnParams& p, int64_t U, int grid) {
+__host__ __device__ __forceinline__ int tc_ctas(const AttnParams& p, int64_t U, int grid) {
   return static_cast<int>(i64max(1, i64min(grid, U / p.min_tiles)));
 }
 
-__device__ __forceinline__ TcRange tc_range(const AttnParams& p, const int* base) {
+// The unit range of CTA c of a grid of `grid` CTAs.
+__host__ __device__ __forceinline__ TcRange tc_range(const AttnParams& p, const int* base, int grid,
+                                                     int c) {
   TcRange r;
   r.U = tc_ubase(p, base, p.B);
-  r.C = tc_ctas(p, r.U, gridDim.x);
-  const int c = blockIdx.x;
+  r.C = tc_ctas(p, r.U, grid);
+  r.c = c;
   r.x = c < r.C ? c * r.U / r.C : 0;
   r.hi = c < r.C ? (c + 1) * r.U / r.C : 0;
   return r;
 }
 
-__device__ __forceinline__ bool tc_next(const AttnParams& p, const int* base, TcRange& r, TcSeg& sg) {
+__host__ __device__ __forceinline__ bool tc_next(const AttnParams& p, const int* base, TcRange& r,
+                                                 TcSeg& sg) {
   while (r.x < r.hi) {
     int lo = 0, hi = p.B;
     while (hi - lo > 1) {
@@ -653,7 +659,7 @@ __device__ __forceinline__ bool tc_next(const AttnParams& p, const int* base, Tc
     sg.g = g;
     sg.t0 = off - kTcSegCost;
     sg.len = static_cast<int>(i64min(r.hi - r.x, nt - sg.t0));
-    const int part = static_cast<int>(blockIdx.x) - tc_cta_of(first, r.U, r.C);
+    const int part = r.c - tc_cta_of(first, r.U, r.C);
     sg.slot = part < p.max_parts ? (b * p.nkv + sg.g) * p.max_parts + part : -1;
     r.x += sg.len;
     return true;
@@ -743,7 +749,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0 && fits) {
       int tc = 0, it = 0, q_issued = 0, nk = 0;
       bool ok = true;
-      TcRange rg = tc_range(p, base);
+      TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
       TcSeg sg;
       for (; ok && tc_next(p, base, rg, sg); ++it) {
         const int b = sg.b, g = sg.g;
@@ -817,7 +823,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t rk_a = smem_u32(ring_k), q_a = smem_u32(qs);
       int tc = 0, it = 0;
       bool ok = true;
-      TcRange rg = tc_range(p, base);
+      TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
       TcSeg sg;
       for (; ok && tc_next(p, base, rg, sg); ++it) {
         const int n_tiles = sg.len;
@@ -866,7 +872,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t b0 = sw64_desc_mn(smem_u32(ps));
       int n_total = 0;
       {
-        TcRange rg = tc_range(p, base);
+        TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
         TcSeg sg;
         while (tc_next(p, base, rg, sg)) n_total += sg.len;
       }
@@ -911,7 +917,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float ls[NR];
     int tc = 0;
     bool fine = true;
-    TcRange rg = tc_range(p, base);
+    TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
     TcSeg sg;
     bool have = tc_next(p, base, rg, sg);
     // row positions are loaded one segment ahead (warp 0, lane = row)
@@ -1275,6 +1281,44 @@ Derived derive(const AttnShape& s) {
 }
 
 }  // namespace
+
+int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_t* seg,
+                    int seg_capacity, int* n_segments, int* max_parts) {
+  const Derived d = derive(s);
+  if (!d.tc) return -1;
+  AttnParams p{};
+  p.B = s.batch;
+  p.nkv = s.n_kv_heads;
+  p.min_tiles = d.min_tiles;
+  p.max_parts = d.max_splits;
+  // 128-key tile prefix, as the kernel builds it from the row positions
+  std::vector<int> base(static_cast<size_t>(s.batch) + 1, 0);
+  const int cap = s.max_pages_per_req * s.page_size;
+  for (int b = 0; b < s.batch; ++b) {
+    const int ke = std::min(std::max(kend[b], 0), cap);
+    base[b + 1] = base[b] + (ke + kTcKeys - 1) / kTcKeys;
+  }
+  int n = 0;
+  for (int c = 0; c < num_sms; ++c) {
+    TcRange r = tc_range(p, base.data(), num_sms, c);
+    TcSeg sg;
+    while (tc_next(p, base.data(), r, sg)) {
+      if (n < seg_capacity) {
+        int32_t* o = seg + static_cast<size_t>(n) * 6;
+        o[0] = c;
+        o[1] = sg.b;
+        o[2] = sg.g;
+        o[3] = sg.t0;
+        o[4] = sg.len;
+        o[5] = sg.slot;
+      }
+      ++n;
+    }
+  }
+  *n_segments = n;
+  *max_parts = d.max_splits;
+  return n <= seg_capacity ? 0 : -2;
+}
 
 size_t attention_workspace_bytes(const AttnShape& s) {
   const Derived d = derive(s);

@@ -964,6 +964,26 @@ int isd_gemm_plan(int32_t m, int32_t n, int32_t k, int32_t single, int32_t max_s
   return p.n_pad > 0 ? ISD_OK : fail(ISD_E_UNSUPPORTED, "no GEMM plan");
 }
 
+int isd_attention_split(int32_t batch, int32_t rows_per_req, int32_t n_q_heads,
+                        int32_t n_kv_heads, int32_t head_dim, int32_t max_pages_per_req,
+                        int32_t page_size, const int32_t* kend_host, int32_t num_sms,
+                        int32_t* seg_out, int32_t seg_capacity, int32_t* n_segments,
+                        int32_t* max_parts) {
+  if (!kend_host || !n_segments || !max_parts || (seg_capacity > 0 && !seg_out))
+    return fail(ISD_E_INVALID, "null argument");
+  if (batch < 1 || batch > 1024 || rows_per_req < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads ||
+      head_dim < 1 || max_pages_per_req < 1 || page_size < 1 || num_sms < 1 || seg_capacity < 0)
+    return fail(ISD_E_INVALID, "bad shape");
+  isd::AttnShape s{batch, rows_per_req, n_q_heads, n_kv_heads, head_dim, page_size, 1,
+                   max_pages_per_req, 1};
+  int n = 0, mp = 0;
+  const int rc = isd::attention_split(s, kend_host, num_sms, seg_out, seg_capacity, &n, &mp);
+  if (rc == -1) return fail(ISD_E_UNSUPPORTED, "shape not served by the tcgen05 attention kernel");
+  *n_segments = n;
+  *max_parts = mp;
+  return rc == 0 ? ISD_OK : fail(ISD_E_INVALID, "seg_capacity too small");
+}
+
 size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k) {
   if (m < 1 || m > 4096 || n < 128 || n % 128 || k < 64 || k % 64) return 0;
   return isd::gemm_streamk_workspace_bytes(isd::plan_gemm(m, n, k, 0, 1, num_sms(), true));

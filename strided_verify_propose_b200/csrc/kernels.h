@@ -74,6 +74,13 @@ struct AttnShape {
       max_pages_per_req, n_layers;
 };
 size_t attention_workspace_bytes(const AttnShape& s);
+// Host mirror of the tcgen05 attention kernel's work split over num_sms CTAs,
+// from the per-request key counts kend[batch]: one record {CTA, request, KV
+// head, first 128-key tile, tiles, partial slot} per segment, in CTA order.
+// Returns 0; -1 when the tcgen05 kernel does not serve the shape; -2 when
+// seg_capacity records are too few (n_segments holds the count needed).
+int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_t* seg,
+                    int seg_capacity, int* n_segments, int* max_parts);
 // k_map / v_map: tensor maps over the pools as [n_layers*num_pages*n_kv*page_size][head_dim]
 // with box_rows = page_size.
 cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map, const AttnShape& s,
