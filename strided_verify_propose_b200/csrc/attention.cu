@@ -1191,22 +1191,38 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p
     for (int s = 0; s < parts; ++s) w[qi][s] *= inv;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < p.RG * (HD / 4); i += blockDim.x) {
-    const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < parts; ++s) {
-      const float ws = w[qi][s];
-      const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * kTcNP + qi) * HD + d);
-      acc.x += ws * v.x;
-      acc.y += ws * v.y;
-      acc.z += ws * v.z;
-      acc.w += ws * v.w;
+  // part-major: every load of one part is in flight at once (one L2 round
+  // trip per part); each output still sums its parts in part order
+  constexpr int kVec = kTcNP * (HD / 4) / 128;   // float4 outputs per thread
+  float4 acc[kVec];
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < parts; ++s) {
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) {
+      const int i = threadIdx.x + j * 128;
+      if (i < p.RG * (HD / 4)) {
+        const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
+        const float ws = w[qi][s];
+        const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * kTcNP + qi) * HD + d);
+        acc[j].x += ws * v.x;
+        acc[j].y += ws * v.y;
+        acc[j].z += ws * v.z;
+        acc[j].w += ws * v.w;
+      }
     }
-    const int r = qi / p.G, h = qi % p.G;
-    __align__(8) __nv_bfloat16 o4[4] = {__float2bfloat16_rn(acc.x), __float2bfloat16_rn(acc.y),
-                                        __float2bfloat16_rn(acc.z), __float2bfloat16_rn(acc.w)};
-    *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b * p.R + r) * p.nq + g * p.G + h) * HD + d) =
-        *reinterpret_cast<const uint2*>(o4);
+  }
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int i = threadIdx.x + j * 128;
+    if (i < p.RG * (HD / 4)) {
+      const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
+      const int r = qi / p.G, h = qi % p.G;
+      __align__(8) __nv_bfloat16 o4[4] = {__float2bfloat16_rn(acc[j].x), __float2bfloat16_rn(acc[j].y),
+                                          __float2bfloat16_rn(acc[j].z), __float2bfloat16_rn(acc[j].w)};
+      *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(b * p.R + r) * p.nq + g * p.G + h) * HD + d) =
+          *reinterpret_cast<const uint2*>(o4);
+    }
   }
 }
 
