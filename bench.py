@@ -441,7 +441,7 @@ def roofline_entry(prof, shape, B, N, lens, steps, peaks):
         achieved = kv / avg_s / 1e9
         peak = peaks["hbm"]
         traffic = None
-        if top == "attention_split" and shape.head_dim == 128 and shape.page_size == 64:
+        if top == "attention" and shape.head_dim == 128 and shape.page_size == 64:
             traffic = ATTN_DRAM_PER_KV_BYTE * kv   # bytes per launch (scaled ncu capture)
         return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic,

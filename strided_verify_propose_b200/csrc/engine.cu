@@ -187,7 +187,7 @@ enum ProfClass {
   kPBookkeep, kPOther, kPCount
 };
 const char* kProfNames[ISD_PROF_CLASSES] = {
-    "assemble", "embed_norm", "gemm_qkv", "qkv_reduce_rope_kvwrite", "attention_split",
+    "assemble", "embed_norm", "gemm_qkv", "qkv_reduce_rope_kvwrite", "attention",
     "attention_combine", "gemm_o", "residual_norm", "gemm_gate_up_silu", "gemm_down",
     "gemm_lm_head", "accept_stats", "accept_decide", "bookkeep", "lora", "unused"};
 
