@@ -24,6 +24,10 @@ reading is listed in the docstring of the function that applies it.
 
 Parity status: the model forward is pinned to an independent Qwen3 decoder
 implementation (HF transformers) on tiny shapes; the accept / resample rule by
-exact enumeration; the ISD layout by the pages' TPF formula and by brute-force
-trajectory distributions; page bookkeeping by brute-force invariants.
+exact enumeration; the ISD layout by the pages' TPF formula, the TPF and
+efficiency values the pages print, and brute-force trajectory distributions;
+the gated LoRA by bitwise base-only verify rows and by a merged-weight model
+on the MASK rows; page bookkeeping by brute-force invariants. Parity
+unpinned: which MASK row proposes which draft position (reading R4 of
+isd.py), which no distribution-level test can see.
 """

@@ -46,7 +46,8 @@ R7 uniform slots per request (2N-1): [0, N-1) accept tests, [N-1] the new
    token, [N, 2N-1) sampled proposals.
 R8 greedy verify (temperature 0): accept iff d_j == argmax p_j; the new
    token is argmax of row A.
-R9 R-ISD: the gated LoRA delta is applied to MASK rows only.
+R9 R-ISD: the gated LoRA delta is applied to MASK rows only (restart padding
+   rows included); x* and the pending drafts run on the base weights.
 """
 from __future__ import annotations
 
