@@ -399,7 +399,7 @@ def run_cuda(args, ws, rank, local):
 
 
 # DRAM bytes (read + write) per byte of K + V of the tcgen05 attention kernel,
-# from the ncu capture summarised in profiles/attn_tc_kernel_qwen3_8b_b64.md
+# from one ncu capture of the kernel at this workload shape (one layer, batch 64)
 # (603.6 MB for a launch over 580.4 MB of K + V at the same workload shape);
 # the roofline's `traffic` scales it to this run's launch.
 ATTN_DRAM_PER_KV_BYTE = 603.6 / 580.4

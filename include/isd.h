@@ -290,9 +290,15 @@ int isd_accept_propose(const float *logits_dev, const isd_batch *batch, const is
  * batch * (2N-1) * ceil(vocab/8192) * 16 bytes of it (at most 4 MiB, e.g.
  * batch <= 1024 at N = 4 and vocab 151936) and returns ISD_E_UNSUPPORTED
  * above that. The first call on each device looks up the array's device
- * address with that device current; make that first call before any
- * stream capture. All calls share the array: calls that overlap on the GPU
- * race and must be serialised by the caller. No scratch needs clearing. */
+ * address with that device current. Under CUDA's lazy module loading (the
+ * default) that lookup is also what loads this part of the library onto the
+ * device and places the array there, so the first call on a device does
+ * allocate (the array and the module's code) and can fail with ISD_E_CUDA
+ * when the device is out of memory: make that first call at start-up,
+ * before a pool takes the GPU's memory and before any stream capture.
+ * Later calls allocate nothing. All calls share the array: calls that
+ * overlap on the GPU race and must be serialised by the caller. No scratch
+ * needs clearing. */
 int isd_accept_propose_noalloc(const float *logits_dev, const isd_batch *batch, const isd_kv *kv,
                                int32_t page_size, int32_t vocab, int32_t *pending_dev,
                                float *q_cache_dev, const float *uniforms_dev,

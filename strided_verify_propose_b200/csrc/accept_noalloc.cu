@@ -14,7 +14,11 @@
 // device (cudaGetSymbolAddress, with that device current) on the first call
 // made while that device is current; host code must not use the symbol's
 // name as a pointer, since in host code it only stands in for the device
-// object. Every call shares the array, so calls whose work overlaps on the
+// object. With lazy module loading (CUDA's default) that first lookup also
+// loads this translation unit's module onto the device, which places the
+// array: the first call on a device allocates and can fail when the device
+// is full, so callers make it at start-up; later calls allocate nothing.
+// Every call shares the array, so calls whose work overlaps on the
 // GPU (different streams, or devices sharing nothing but this library) race
 // on it; callers must serialise them. The kernels write every scratch entry
 // before they read it, so nothing needs clearing between calls.

@@ -30,7 +30,10 @@ TINY_LOGIT_STD = 0.32  # logit standard deviation of the tiny decoder (N(0, 0.02
 
 def logit_tolerance(oracle_logits: np.ndarray) -> float:
     """2e-2 at the tiny decoder's logit spread, scaled with the spread of
-    wider models (bf16 activation rounding grows with it)."""
+    wider models: the bf16 rounding of every GEMM input grows with the
+    activations, which grow with the logit spread (an fp64 emulation of the
+    kernels' rounding points gives 5.5e-2 at Qwen3-8B widths after two
+    layers, against 8e-2 here)."""
     return LOGIT_TOL * max(1.0, float(np.std(oracle_logits)) / TINY_LOGIT_STD)
 
 

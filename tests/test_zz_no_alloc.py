@@ -77,3 +77,27 @@ def test_noalloc_rejects_batches_beyond_its_scratch(cuda_lib):
     u = torch.zeros(Bn, 2 * N - 1, device="cuda")
     with pytest.raises(RuntimeError, match="fixed array holds"):
         B.accept_propose_noalloc(logits, st, kv, 16, u, 0)
+
+
+def test_noalloc_calls_after_the_first_allocate_nothing(cuda_lib):
+    """The property the entry point is named for: once the first call on the
+    device has placed the library's array, further calls leave both the
+    device's free memory and PyTorch's allocator untouched."""
+    from strided_verify_propose_b200 import binding as B
+    Bn, N, V = 64, 4, 151936
+    c = _accept_case(Bn, N, V, oi.ARGMAX, oi.STOCHASTIC, seed=777, boost=7.5)
+    logits = torch.from_numpy(c["logits"]).cuda()
+    u = torch.from_numpy(c["u"]).cuda()
+    st, kv = _state(c, Bn, N, V)
+    B.accept_propose_noalloc(logits, st, kv, c["P"], u, 0)      # first call: may load the module
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0, reserved0 = torch.cuda.memory_allocated(), torch.cuda.memory_reserved()
+    for _ in range(5):
+        B.accept_propose_noalloc(logits, st, kv, c["P"], u, 0)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert int(st.status.item()) & ~B.ISD_DEV_POOL_EXHAUSTED == 0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.memory_reserved() == reserved0
+    assert free1 == free0, (free0, free1)
