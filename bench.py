@@ -64,8 +64,12 @@ WORKLOADS = {
     # R-ISD: Qwen3-8B shape + rank-128 gated LoRA on MASK rows, batch 32, N=4, prompts 2048
     "risd_8b_b32": dict(shape=synth.QWEN3_8B, batch=32, stride=4, len_lo=2048, len_hi=2048,
                         lora_rank=128),
+    # Qwen3-32B shape (64 layers, hidden 5120, 64/8 heads), batch 64, N=4, prompts U[1024, 8192]
+    "qwen3_32b_b64": dict(shape=synth.QWEN3_32B, batch=64, stride=4, len_lo=1024, len_hi=8192),
 }
 ACCEPT_RATE = 0.9
+MODEL_NAMES = {synth.QWEN3_8B: "qwen3-8b-shape (random init)",
+               synth.QWEN3_32B: "qwen3-32b-shape (random init)"}
 
 
 def load_peaks():
@@ -151,10 +155,15 @@ def setup_dist():
 
 # ------------------------------------------------------------ algorithmic ---
 
+def step_w_params(shape):
+    """Weights a step streams: every layer's projections and the LM head."""
+    return shape.n_layers * shape.params_per_layer() + shape.vocab * shape.hidden
+
+
 def step_bytes_flops(shape, lens_now, B, N):
     """Algorithmic bytes / flops of one step (weights once, KV once, logits once)."""
     R = 2 * N - 1
-    w_params = shape.n_layers * shape.params_per_layer() + shape.vocab * shape.hidden
+    w_params = step_w_params(shape)
     kv = sum(int(L) + R for L in lens_now) * shape.kv_bytes_per_token()
     logits = B * R * shape.vocab * 4
     flops = 2.0 * B * R * w_params
@@ -333,6 +342,12 @@ def run_cuda(args, ws, rank, local):
     e2e_ms = x_start.elapsed_time(x_stop)
     e2e_committed = int((pin_acc.long() + 1).sum().item())
 
+    # ---- the other single-GPU configurations of the same model (one GPU only)
+    extras = None
+    if ws == 1 and not args.no_extras and shape is synth.QWEN3_8B and not lora_rank \
+            and not wl.get("sample"):
+        extras = extra_configs(model, shape, args, seed)
+
     # ---- reduce over ranks: max time, summed tokens
     (ms, e2e_ms, nat_ms, eager_ms_all), (committed, e2e_committed, nat_committed, eager_committed) = \
         reduce_over_ranks([ms, e2e_ms, nat_ms, eager_ms or 0.0],
@@ -361,13 +376,14 @@ def run_cuda(args, ws, rank, local):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (random-init weights, uniform random prompts, seeded)",
-            "config": {"workload": args.workload, "model": "qwen3-8b-shape (random init)"
-                       if shape is synth.QWEN3_8B else "tiny", "batch_per_gpu": B,
+            "config": {"workload": args.workload, "model": MODEL_NAMES.get(shape, "tiny"),
+                       "batch_per_gpu": B,
                        "global_batch": B * ws, "stride_n": N, "rows_per_step": B * R,
                        "prompt_len": [wl["len_lo"], wl["len_hi"]], "page_size": P,
                        "parallelism": f"replicas x{ws} (request-sharded, no collective)",
                        "uniforms": f"acceptance-controlled a={ACCEPT_RATE}",
-                       "l2": "inputs larger than L2 (weights 16 GB + KV > 126 MB)"},
+                       "l2": f"inputs larger than L2 (weights {2 * step_w_params(shape) / 1e9:.0f} GB "
+                             "+ KV > 126 MB)"},
             "tokens_per_forward": committed / (args.steps * B * ws),
             "hbm_roofline_fraction_step": hbm_frac_step,
             "hbm_roofline_ceiling_step": ceiling,
@@ -391,11 +407,89 @@ def run_cuda(args, ws, rank, local):
                     "h2d_bytes_per_step": B * R * 4, "d2h_bytes_per_step": B * 4 + B * N * 4},
             "peaks": peaks,
         }
+        if extras is not None:
+            ex = dict(extras)
+            b1 = ex["qwen3_8b_b1"]
+            b1["hbm_roofline_fraction"] = b1["step_bytes"] / (b1["ms_per_step"] * 1e-3) / (
+                peaks["hbm"] * 1e9)
+            result["other_configs"] = ex
+            result["risd_overhead_alpha"] = ex["risd_8b_b32"]["alpha"]
     del model
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def extra_configs(model, shape, args, seed):
+    """The model's two other single-GPU configurations, on the same weights:
+    batch 1 with a 2048-token prompt, and R-ISD (a rank-128 gated LoRA,
+    A, B ~ N(0, 0.01), on the MASK rows) at batch 32 with 2048-token
+    prompts, timed against the same steps without the adapter. Each runs
+    args.warmup eager steps, then args.steps steps between CUDA events
+    (acceptance-controlled uniforms, inputs resident)."""
+    import torch
+    from strided_verify_propose_b200 import binding as Bd
+    N = 4
+    R, P, V = 2 * N - 1, shape.page_size, shape.vocab
+    stream = torch.cuda.current_stream()
+    out = {}
+
+    def make(B, plen, s0):
+        lens = np.full(B, plen, np.int64)
+        prompts = synth.prompts(shape, lens, s0)
+        steps = args.warmup + 3 * args.steps + 2
+        maxp = -(-(plen + steps * N + R + 1) // P) + 1
+        need = [-(-(plen - 1 + R) // P)] * B
+        num_pages = int(sum(need)) + B * (-(-steps * N // P) + 2)
+        table, free = synth.page_layout(need, num_pages, maxp, s0)
+        kv = Bd.KVCache(shape, num_pages, table, free)
+        st = Bd.StepState(B, N, V, sample=False)
+        Bd.prefill(model, kv, st, prompts)
+        torch.cuda.synchronize()
+        if int(st.status.item()) != 0:
+            raise RuntimeError("prefill status")
+        return kv, st
+
+    def timed(kv, st, B, flags, s0, first):
+        for i in range(args.warmup):
+            Bd.step(model, kv, st, torch.from_numpy(
+                synth.controlled_uniforms(B, N, ACCEPT_RATE, s0, first + i)).cuda(), flags)
+        u = torch.from_numpy(np.stack([synth.controlled_uniforms(B, N, ACCEPT_RATE, s0, first + 100 + i)
+                                       for i in range(args.steps)])).cuda()
+        acc = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
+        lens0 = st.seq_len.cpu().numpy().copy()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            Bd.step(model, kv, st, u[i], flags)
+            acc[i].copy_(st.accepted)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if int(st.status.item()) != 0:
+            raise RuntimeError("step status")
+        return e0.elapsed_time(e1), int((acc.long() + 1).sum().item()), lens0
+
+    # batch 1, prompt 2048: every projection streams its weights for 7 rows
+    kv, st = make(1, 2048, seed + 11)
+    ms1, com1, lens1 = timed(kv, st, 1, 0, seed + 11, 0)
+    w, kvb, _, _ = step_bytes_flops(shape, lens1, 1, N)
+    out["qwen3_8b_b1"] = {"ms_per_step": ms1 / args.steps, "value": com1 / (ms1 * 1e-3),
+                          "unit": "tokens/s", "step_bytes": w + kvb, "steps": args.steps}
+    del kv, st
+    # R-ISD at batch 32: the same steps with and without the adapter
+    model.load_lora(Bd.random_device_lora(shape, 128, seed=seed, std=0.01), rank=128)
+    kv, st = make(32, 2048, seed + 12)
+    ms_b, _, _ = timed(kv, st, 32, 0, seed + 12, 0)
+    ms_l, com_l, _ = timed(kv, st, 32, Bd.USE_LORA, seed + 12, 1000)
+    out["risd_8b_b32"] = {"ms_per_step": ms_l / args.steps, "value": com_l / (ms_l * 1e-3),
+                          "unit": "tokens/s", "base_ms_per_step": ms_b / args.steps,
+                          "alpha": ms_l / ms_b, "steps": args.steps,
+                          "adapter": "rank 128, A, B ~ N(0, 0.01), q/k/v/o/gate/up/down"}
+    del kv, st
+    torch.cuda.synchronize()
+    return out
 
 
 # DRAM bytes (read + write) per byte of K + V of the tcgen05 attention kernel,
@@ -616,6 +710,8 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="qwen3_8b_b64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the batch-1 and R-ISD runs reported beside the headline")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the steps launched one by one instead of replaying a CUDA graph")
     ap.add_argument("--component", default=None,

@@ -188,6 +188,17 @@ const char *isd_profile_class_name(int cls);
 const char *isd_last_error(void);
 void isd_destroy(isd_ctx *ctx);
 
+/* Cycle limit of every bounded device wait (an mbarrier phase, a stream-K
+ * partner's flag) on the current device; 0 restores the default of 4e9
+ * cycles (about 2 s). A wait that runs out sets ISD_DEV_TIMEOUT and its
+ * kernel returns without writing the affected results, so a context stays
+ * usable. For tests of failure handling: a short limit lets a test make a
+ * wait run out quickly. Synchronous (not during stream capture); affects
+ * every context on the device. No counterpart on the pages: the status word
+ * is this library's own failure reporting. Returns ISD_E_INVALID for a limit
+ * below 1000 cycles, ISD_E_CUDA if the copy fails. */
+int isd_set_wait_limit(long long cycles);
+
 /* ---- component entry points (used by the tests; same kernels as a step) -- */
 
 /* Y = X W^T on the tcgen05 tensor cores, fp32 accumulate.

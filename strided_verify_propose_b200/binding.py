@@ -35,7 +35,7 @@ EXPORTS = ("isd_init", "isd_load_gated_lora", "isd_step", "isd_prefill", "isd_la
            "isd_paged_attention", "isd_accept_workspace_bytes", "isd_accept_propose",
            "isd_profile_enable", "isd_profile_read", "isd_profile_class_name",
            "isd_accept_propose_noalloc", "isd_gemm_workspace_bytes", "isd_gemm_bf16_single",
-           "isd_gemm_plan", "isd_attention_split")
+           "isd_gemm_plan", "isd_attention_split", "isd_set_wait_limit")
 PROF_CLASSES = 16
 
 
@@ -108,6 +108,7 @@ def lib():
                                      vp, vp, vp, sz, vp, vp]
     L.isd_accept_propose_noalloc.argtypes = [vp, C.POINTER(Batch), C.POINTER(KV), i32, i32, vp,
                                              vp, vp, vp, vp, vp, vp]
+    L.isd_set_wait_limit.argtypes = [C.c_longlong]
     L.isd_profile_enable.argtypes = [vp, C.c_int]
     L.isd_profile_read.argtypes = [vp, C.POINTER(C.c_double), C.POINTER(i32)]
     L.isd_profile_class_name.argtypes = [C.c_int]
@@ -388,6 +389,11 @@ def prefill(model: Model, kv: KVCache, st: StepState, prompts: List[np.ndarray])
 
 
 # ------------------------------------------------------ component calls ---
+
+def set_wait_limit(cycles: int) -> None:
+    """Cycle limit of the library's bounded device waits (0: the default)."""
+    check(lib().isd_set_wait_limit(int(cycles)))
+
 
 def gemm_bf16(w, x, split_k: int = 1, status=None):
     """Y[split][m][n] partial sums of X W^T (torch bf16 device tensors)."""

@@ -1336,6 +1336,8 @@ int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_
   return n <= seg_capacity ? 0 : -2;
 }
 
+cudaError_t set_wait_limit_attention(long long cycles) { return set_wait_limit_here(cycles); }
+
 size_t attention_workspace_bytes(const AttnShape& s) {
   const Derived d = derive(s);
   const size_t rows = static_cast<size_t>(d.MT) * 16;

@@ -16,6 +16,16 @@ namespace isd {
 // B200's clocks) and reports ISD_DEV_TIMEOUT instead of hanging the GPU.
 constexpr long long kWaitCycles = 4000000000LL;
 
+// The limit the waits of this translation unit use (each .cu file holds its
+// own copy; isd_set_wait_limit sets all of them). Read only once a wait has
+// not completed at its first poll.
+static __device__ long long g_wait_limit = kWaitCycles;
+
+// Set this translation unit's wait limit on the current device (synchronous).
+static inline cudaError_t set_wait_limit_here(long long cycles) {
+  return cudaMemcpyToSymbol(g_wait_limit, &cycles, sizeof(cycles));
+}
+
 __device__ __forceinline__ void flag(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
 }
@@ -71,8 +81,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

@@ -1053,6 +1053,14 @@ int isd_paged_attention(const void* q_dev, const int32_t* row_pos_dev, const voi
   return ISD_OK;
 }
 
+int isd_set_wait_limit(long long cycles) {
+  if (cycles != 0 && cycles < 1000) return fail(ISD_E_INVALID, "wait limit below 1000 cycles");
+  const long long c = cycles == 0 ? 4000000000LL : cycles;
+  ISD_CUDA(isd::set_wait_limit_gemm(c));
+  ISD_CUDA(isd::set_wait_limit_attention(c));
+  return ISD_OK;
+}
+
 size_t isd_accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab) {
   return isd::accept_workspace_bytes(batch, stride_n, vocab);
 }

@@ -333,8 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (m_ == 2) {
             // the first part's CTA is in its epilogue: wait for its flag
             const long long t0 = clock64();
+            const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
             while (ld_acquire_gpu(&sync[1]) == 0) {
-              if (clock64() - t0 > kWaitCycles) {
+              if (clock64() - t0 > limit) {
                 flag(p.status, ISD_DEV_TIMEOUT);
                 m_ = 3;
                 break;
@@ -546,6 +547,8 @@ size_t gemm_streamk_workspace_bytes(const GemmPlan& plan) {
 }
 
 size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }
+
+cudaError_t set_wait_limit_gemm(long long cycles) { return set_wait_limit_here(cycles); }
 
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,

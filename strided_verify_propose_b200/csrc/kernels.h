@@ -13,6 +13,11 @@ namespace isd {
 // Record msg as the calling thread's last error (see isd_last_error); returns code.
 int set_error(int code, const char* msg);
 
+// Cycle limit of the bounded device waits of the GEMM and attention kernels
+// on the current device (synchronous copies to each file's limit).
+cudaError_t set_wait_limit_gemm(long long cycles);
+cudaError_t set_wait_limit_attention(long long cycles);
+
 // --------------------------------------------------------------- tensor maps
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix, box
 // {64 columns (128 B), box_rows}, 128-byte swizzle, zero fill out of bounds.

@@ -71,6 +71,8 @@ QWEN3_8B_2L = dataclasses.replace(QWEN3_8B, n_layers=2)
 # Qwen3-32B widths.
 QWEN3_32B = ModelShape(n_layers=64, hidden=5120, n_q_heads=64, n_kv_heads=8, head_dim=128,
                        intermediate=25600, vocab=151936, page_size=64)
+# Qwen3-32B widths, two layers.
+QWEN3_32B_2L = dataclasses.replace(QWEN3_32B, n_layers=2)
 
 
 # --------------------------------------------------------------- streams ---

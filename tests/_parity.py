@@ -44,8 +44,12 @@ def _softmax(z):
 
 
 def _cdf_draw(w, u):
-    """(index, relative margin) of the inverse-CDF draw of weights w at u."""
+    """(index, relative margin) of the inverse-CDF draw of weights w at u.
+    u = 0 picks the first token of nonzero weight in any precision: no
+    rounding can move that draw (margin inf)."""
     w = np.asarray(w, dtype=np.float64)
+    if u == 0.0:
+        return int(np.flatnonzero(w > 0)[0]), np.inf
     c = np.cumsum(w)
     total = c[-1]
     t = u * total
@@ -82,15 +86,66 @@ def _argmax(z):
     return int(np.flatnonzero(z == z.max())[0])
 
 
+# decision kinds the near cases are counted by
+KINDS = ("accept", "argmax", "draw")
+
+
 class Outcome:
+    """What the comparison of one request-step found: per decision kind, the
+    decisions examined and how many of them fell inside the error band."""
+
     def __init__(self):
         self.clear = True          # every decision clear of the error band
         self.accept_clear = True   # the accept tests were (A compared exactly)
         self.notes = []
+        self.decisions = {k: 0 for k in KINDS}
+        self.near_kinds = {k: 0 for k in KINDS}
 
-    def near(self, what):
+    def seen(self, kind):
+        self.decisions[kind] += 1
+
+    def near(self, kind, what):
         self.clear = False
+        self.near_kinds[kind] += 1
         self.notes.append(what)
+
+
+class Report:
+    """Counts over a whole run: request-steps compared and compared exactly,
+    requests that left the comparison after a near decision went the other
+    way, and per decision kind the decisions examined and the near ones."""
+
+    def __init__(self, label):
+        self.label = label
+        self.request_steps = 0
+        self.exact = 0
+        self.dropped = 0
+        self.decisions = {k: 0 for k in KINDS}
+        self.near = {k: 0 for k in KINDS}
+        self.max_dz = 0.0
+        self.tol = 0.0
+
+    def add(self, out):
+        self.request_steps += 1
+        self.exact += 1 if out.clear else 0
+        for k in KINDS:
+            self.decisions[k] += out.decisions[k]
+            self.near[k] += out.near_kinds[k]
+
+    def near_fraction(self, kind):
+        return self.near[kind] / self.decisions[kind] if self.decisions[kind] else 0.0
+
+    def line(self):
+        parts = [f"{k} {self.near[k]}/{self.decisions[k]} near" for k in KINDS]
+        return (f"parity[{self.label}]: {self.exact}/{self.request_steps} request-steps exact, "
+                f"{self.dropped} requests parted; " + ", ".join(parts) +
+                f"; max |dz| {self.max_dz:.3g} (bar {self.tol:.3g})")
+
+    def check(self, max_near, min_request_steps=1):
+        """Upper bounds on the near fraction of each decision kind."""
+        assert self.request_steps >= min_request_steps, self.line()
+        for k, bound in max_near.items():
+            assert self.near_fraction(k) <= bound, (k, self.line())
 
 
 def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u, N, propose,
@@ -111,10 +166,11 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
     for j in range(n):
         d = drafts[j]
         if greedy:
+            out.seen("argmax")
             ok_o = d == _argmax(lo[j])
             ok_g = d == _argmax(lg[j])
             if ok_o != ok_g:
-                out.near(f"greedy test {j}")
+                out.near("argmax", f"greedy test {j}")
                 A_g_expected = None
                 break
         else:
@@ -124,8 +180,9 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
             r_o = p_o / qd_o if qd_o > 0 else np.inf
             r_g = p_g / qd_g if qd_g > 0 else np.inf
             ok_o, ok_g = u[j] < r_o, u[j] < r_g
+            out.seen("accept")
             if abs(u[j] - r_o) < ACCEPT_BAR or ok_o != ok_g or abs(u[j] - r_g) < FP32_REL * max(r_g, 1e-30):
-                out.near(f"accept test {j}")
+                out.near("accept", f"accept test {j}")
                 break
         if not ok_o:
             break
@@ -136,16 +193,18 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
     A = dec.accepted
     # ---- the new token from row A
     if greedy:
+        out.seen("argmax")
         t_o, t_g = _argmax(lo[A]), _argmax(lg[A])
         assert gpu_new == t_g, "greedy new token is not the argmax of the kernel's logits"
         if t_o == t_g:
             assert gpu_new == dec.new_token
         else:
-            out.near("greedy new token")
+            out.near("argmax", "greedy new token")
     else:
         exc = drafts[A] if (A < n and not sample_prop) else -1
         w_o = _weights(lo[A], q_o[A] if (A < n and sample_prop) else None, exc)
         w_g = _weights(lg[A], q_g[A] if (A < n and sample_prop) else None, exc)
+        out.seen("draw")
         t_o, m_o = _cdf_draw(w_o, u[N - 1])
         t_g, m_g = _cdf_draw(w_g, u[N - 1])
         assert t_o == dec.new_token
@@ -156,19 +215,21 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
         if t_o == t_g and m_g >= FP32_REL:
             assert gpu_new == dec.new_token
         else:
-            out.near("new-token draw")
+            out.near("draw", "new-token draw")
     # ---- proposals (rows n+1..n+N-1), only after no rejection
     if A == n:
         for i in range(1, N):
             r = n + i
             if not sample_prop:
+                out.seen("argmax")
                 a_o, a_g = _argmax(lo[r]), _argmax(lg[r])
                 assert gpu_props[i - 1] == a_g, "argmax proposal is not the kernel logits' argmax"
                 if a_o == a_g:
                     assert gpu_props[i - 1] == dec.proposals[i - 1]
                 else:
-                    out.near(f"argmax proposal {i}")
+                    out.near("argmax", f"argmax proposal {i}")
             else:
+                out.seen("draw")
                 t_o, _ = _cdf_draw(_softmax(lo[r]), u[N + i - 1])
                 t_g, m_g = _cdf_draw(_softmax(lg[r]), u[N + i - 1])
                 if m_g >= FP32_REL:
@@ -178,5 +239,5 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
                 if t_o == t_g and m_g >= FP32_REL:
                     assert gpu_props[i - 1] == dec.proposals[i - 1]
                 else:
-                    out.near(f"sampled proposal {i}")
+                    out.near("draw", f"sampled proposal {i}")
     return out

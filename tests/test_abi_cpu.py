@@ -58,3 +58,84 @@ def test_gate_up_packing_interleaves_blocks_of_16():
     qkv = packed["layers"][0]["w_qkv"].float().numpy()
     assert np.array_equal(qkv[:shape.q_dim], w["layers"][0]["wq"])
     assert np.array_equal(qkv[shape.q_dim + shape.kv_dim:], w["layers"][0]["wv"])
+
+
+# ------------------------------------------------ host argument validation --
+# Every call below is refused by the library's host-side checks before it
+# touches a device, so they run without a GPU.
+
+def _cfg(**kw):
+    base = dict(n_layers=2, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=64, intermediate=704,
+                vocab=1024, rope_theta=1e6, rms_eps=1e-6, mask_token_id=1023, page_size=16,
+                max_batch=4, max_rows=64, max_position=512)
+    base.update(kw)
+    return binding.ModelCfg(*[base[f] for f, _ in binding.ModelCfg._fields_])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), binding.ISD_E_UNSUPPORTED),
+    (dict(page_size=48), binding.ISD_E_UNSUPPORTED),
+    (dict(n_q_heads=6, n_kv_heads=2), binding.ISD_E_UNSUPPORTED),    # group of 3
+    (dict(hidden=200), binding.ISD_E_UNSUPPORTED),
+    (dict(vocab=1000, mask_token_id=999), binding.ISD_E_UNSUPPORTED),
+    (dict(max_rows=8192), binding.ISD_E_UNSUPPORTED),
+    (dict(max_batch=2048), binding.ISD_E_UNSUPPORTED),
+    (dict(mask_token_id=1024), binding.ISD_E_INVALID),
+    (dict(hidden=0), binding.ISD_E_INVALID),
+])
+def test_init_refuses_bad_configs(kw, code):
+    lib = binding.lib()
+    h = ctypes.c_void_p()
+    assert lib.isd_init(ctypes.byref(_cfg(**kw)), None, ctypes.byref(h)) == code
+    assert not h.value
+    assert lib.isd_last_error()
+
+
+def test_entry_points_refuse_null_arguments():
+    lib = binding.lib()
+    h = ctypes.c_void_p()
+    assert lib.isd_init(None, None, ctypes.byref(h)) == binding.ISD_E_INVALID
+    b = binding.Batch(4, 3, 0, 1, 1, None)
+    kv = binding.KV(1, 1, 1, 1, 1, 8, 4, 8)
+    assert lib.isd_step(None, ctypes.byref(b), ctypes.byref(kv), 1, None, 1, 1, None, 1,
+                        None) == binding.ISD_E_INVALID
+    assert lib.isd_prefill(None, ctypes.byref(kv), 1, 8, None, 1, 3, 1, 1, 1, 1,
+                           None) == binding.ISD_E_INVALID
+    assert lib.isd_load_gated_lora(None, None) == binding.ISD_E_INVALID
+    assert lib.isd_accept_propose(None, ctypes.byref(b), ctypes.byref(kv), 16, 1024, 1, None, 1,
+                                  1, None, 1, 1 << 20, 1, None) == binding.ISD_E_INVALID
+    assert lib.isd_gemm_bf16(None, 1, 1, 64, 128, 64, 1, None, None) == binding.ISD_E_INVALID
+    assert lib.isd_profile_enable(None, 1) == binding.ISD_E_INVALID
+
+
+def test_accept_refuses_out_of_range_sizes():
+    lib = binding.lib()
+    kv = binding.KV(1, 1, 1, 1, 1, 8, 4, 8)
+    for batch, n, vocab, code in [(0, 3, 1024, binding.ISD_E_INVALID),
+                                  (4, 9, 1024, binding.ISD_E_INVALID),
+                                  (4, 3, 1022, binding.ISD_E_UNSUPPORTED)]:
+        b = binding.Batch(batch, n, 0, 1, 1, None)
+        assert lib.isd_accept_propose(1, ctypes.byref(b), ctypes.byref(kv), 16, vocab, 1, None, 1,
+                                      1, None, 1, 1 << 20, 1, None) == code, (batch, n, vocab)
+    # the fixed-scratch variant refuses a batch its array cannot hold
+    b = binding.Batch(1024, 8, 0, 1, 1, None)
+    assert lib.isd_accept_propose_noalloc(1, ctypes.byref(b), ctypes.byref(kv), 16, 151936, 1,
+                                          None, 1, 1, None, 1, None) == binding.ISD_E_UNSUPPORTED
+    assert b"fixed array holds" in lib.isd_last_error()
+
+
+def test_component_calls_refuse_unsupported_shapes():
+    lib = binding.lib()
+    # GEMM: n not a multiple of 128, k not of 64, too many splits
+    assert lib.isd_gemm_bf16(1, 1, 1, 64, 100, 64, 1, None, None) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_gemm_bf16(1, 1, 1, 64, 128, 96, 1, None, None) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_gemm_bf16(1, 1, 1, 64, 128, 128, 3, None, None) == binding.ISD_E_UNSUPPORTED
+    # attention: head_dim 96, a group of 3 query heads, 9 rows x 8 heads > 64
+    args = [1, 1, 1, 1, 1]
+    assert lib.isd_paged_attention(*args, 4, 7, 8, 8, 96, 64, 10, 4, 1, 0, 1, 1, 1 << 20, None,
+                                   None) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_paged_attention(*args, 4, 7, 6, 2, 128, 64, 10, 4, 1, 0, 1, 1, 1 << 20, None,
+                                   None) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_paged_attention(*args, 4, 9, 64, 8, 128, 64, 10, 4, 1, 0, 1, 1, 1 << 20, None,
+                                   None) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_set_wait_limit(10) == binding.ISD_E_INVALID
