@@ -72,6 +72,18 @@ MODEL_NAMES = {synth.QWEN3_8B: "qwen3-8b-shape (random init)",
                synth.QWEN3_32B: "qwen3-32b-shape (random init)"}
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU baseline."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -624,7 +636,8 @@ def run_reference(args, ws, rank):
             "data": "synthetic", "config": {"workload": args.workload, "batch_per_gpu": wl["batch"],
                                              "stride_n": wl["stride"]},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": sample, "wall_s": time.time() - t0},
+                             "sample": sample, "wall_s": time.time() - t0,
+                             "cpu_model": cpu_model(), "host_cpus": os.cpu_count()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -733,7 +746,8 @@ def main():
         if ws == 1 and not args.no_cpu_baseline:
             v, threads, sample, _ = oracle_sample(args, 2, args.workload)
             res["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                   "sample": sample}
+                                   "sample": sample, "cpu_model": cpu_model(),
+                                   "host_cpus": os.cpu_count()}
         print(json.dumps(res), flush=True)
 
 

@@ -157,6 +157,9 @@ struct isd_ctx {
   std::map<std::tuple<int, int, int, int>, GemmPlan> plans;
   void* sk_ws = nullptr;            // stream-K partials + sync words (sync words zeroed)
   size_t sk_ws_bytes = 0;
+  int32_t* red_cnt = nullptr;       // arrival / departure counters of in-kernel split-K reduction
+  int32_t red_cnt_n = 0;
+  std::map<std::tuple<int, int, int, int>, int> coresident;   // per plan: CTAs resident at once
   int launches = 0;
 
   // gated LoRA (R-ISD): packed adapters per layer + their workspace
@@ -251,10 +254,16 @@ struct AugSpec {
   int k2;
 };
 
+// With reduce_out, a split-K plan whose whole grid fits on the device at
+// once reduces its splits inside the kernel: the partials go to the front of
+// out and the single output slice behind them; *reduce_out points at the
+// slices the next kernel reads (the reduced slice with *splits_used = 1, or
+// out itself with the plan's split count).
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
-         const AugSpec* aug = nullptr) {
+         const AugSpec* aug = nullptr, float** reduce_out = nullptr,
+         const isd::QkvReduceArgs* qkv = nullptr, bool* qkv_fused = nullptr) {
   if (epi == isd::kEpiF32 && out_elems > 0) {
     // large prefill chunks: no more splits than the partial buffer holds
     const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
@@ -279,11 +288,32 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
     if (rc) return rc;
     ga = isd::GemmAugment{aug->tw2, tx2, aug->k2};
   }
+  isd::GemmReduce red{};
+  bool reduced = false;
+  float* result = out;
+  if (reduce_out && epi == isd::kEpiF32 && plan.splits > 1 && !plan.streamk) {
+    const size_t rf = isd::gemm_reduce_floats(plan, n);
+    if (rf + static_cast<size_t>(m) * n <= out_elems &&
+        isd::gemm_reduce_counters(plan, n) <= c->red_cnt_n) {
+      auto key = std::make_tuple(plan.pair, plan.n_mma, static_cast<int>(plan.smem_bytes), 0);
+      auto it = c->coresident.find(key);
+      if (it == c->coresident.end()) it = c->coresident.emplace(key, isd::gemm_coresident_ctas(plan)).first;
+      const int64_t ctas = static_cast<int64_t>(n / 128) * plan.n_chunks * plan.splits;
+      if (ctas <= it->second) {
+        red = isd::GemmReduce{out, rf, c->red_cnt, c->red_cnt_n, it->second};
+        reduced = true;
+        result = out + rf;
+      }
+    }
+  }
   cudaEvent_t e0 = prof_mark(c, st);
-  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, aug ? &ga : nullptr));
+  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, result, act, status, st, c->sk_ws,
+                            c->sk_ws_bytes, aug ? &ga : nullptr, reduced ? &red : nullptr,
+                            reduced ? qkv : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
-  if (splits_used) *splits_used = plan.splits;
+  if (qkv_fused) *qkv_fused = reduced && qkv != nullptr;
+  if (splits_used) *splits_used = reduced ? 1 : plan.splits;
+  if (reduce_out) *reduce_out = result;
   c->launches += 1;
   return ISD_OK;
 }
@@ -406,12 +436,9 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_qkv, c->hn, M, H, 3 * r, status, st);
       if (rc) return rc;
     }
-    rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr);
-    if (rc) return rc;
     isd::QkvReduceArgs qa;
-    qa.part = c->part;
-    qa.splits = s;
+    qa.part = nullptr;
+    qa.splits = 0;
     qa.rows = M;
     qa.rows_per_req = rows_per_req;
     qa.n_q = g.n_q_heads;
@@ -432,11 +459,24 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
     qa.status = status;
-    cudaEvent_t a0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_qkv_reduce(qa, st));
-    c->launches += 1;
+    // the QKV projection; when its split-K reduction runs in the kernel the
+    // kernel also finishes QK-norm, RoPE and the q / KV writes
+    float* slices = nullptr;
+    bool fused = false;
+    rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr,
+              &slices, &qa, &fused);
+    if (rc) return rc;
     cudaEvent_t a1 = prof_mark(c, st);
-    prof_add(c, kPQkvReduce, a0, a1);
+    if (!fused) {
+      qa.part = slices;
+      qa.splits = s;
+      cudaEvent_t a0 = a1;
+      ISD_CUDA(isd::launch_qkv_reduce(qa, st));
+      c->launches += 1;
+      a1 = prof_mark(c, st);
+      prof_add(c, kPQkvReduce, a0, a1);
+    }
     cudaEvent_t amid = prof_event(c);
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid));
@@ -449,10 +489,10 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
-              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
+              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr, &slices);
     if (rc) return rc;
     cudaEvent_t r0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
+    ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
     prof_add(c, kPResNorm, r0, prof_mark(c, st));
     c->launches += 1;
     // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
@@ -471,11 +511,11 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr, &slices);
     if (rc) return rc;
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
     cudaEvent_t r1 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
+    ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
     prof_add(c, kPResNorm, r1, prof_mark(c, st));
     c->launches += 1;
   }
@@ -535,6 +575,7 @@ int alloc_workspace(isd_ctx* c) {
       static_cast<size_t>(g.max_batch) * 4,
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
+      static_cast<size_t>(2 * (wide / 128) * 8) * 4,      // split-K reduction counters
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -564,8 +605,11 @@ int alloc_workspace(isd_ctx* c) {
   c->prefill_lens = reinterpret_cast<int32_t*>(b + off[i++]);
   c->sk_ws = b + off[i++];
   c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
-  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
-    return fail(ISD_E_CUDA, "stream-K workspace clear failed");
+  c->red_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
+  c->red_cnt_n = static_cast<int32_t>(2 * (wide / 128) * 8);
+  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
+      cudaMemset(c->red_cnt, 0, static_cast<size_t>(c->red_cnt_n) * 4) != cudaSuccess)
+    return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;
   std::vector<float2> tab(static_cast<size_t>(g.max_position) * half);

@@ -64,14 +64,40 @@ struct GemmAugment {
   int32_t k;
 };
 
+// Split-K reduced inside the kernel (a plan with splits > 1 and no
+// stream-K): the splits park fp32 partials in red (gemm_reduce_floats), wait
+// for each other on counters (gemm_reduce_counters ints, zero before the
+// first launch; each launch leaves them zero) and write one output slice.
+// The splits wait for each other, so the whole grid must be resident at
+// once: coresident is gemm_coresident_ctas(plan), and the launch is refused
+// when the grid has more CTAs.
+struct GemmReduce {
+  float* red;
+  size_t red_floats;
+  int32_t* counters;
+  int32_t n_counters;
+  int32_t coresident;
+};
+size_t gemm_reduce_floats(const GemmPlan& plan, int32_t n_out);
+int gemm_reduce_counters(const GemmPlan& plan, int32_t n_out);
+// CTAs of this plan's kernel that can be resident on the device at once.
+int gemm_coresident_ctas(const GemmPlan& plan);
+
+struct QkvReduceArgs;
+
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
-// kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
-// with W's rows interleaved in blocks of 16 (gate rows then up rows).
+// kEpiF32: out_f32[split][m][n_out] (one slice when reduced); kEpiSiluMul:
+// out_act[m][n_out / 2] bf16 with W's rows interleaved in blocks of 16
+// (gate rows then up rows).
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmAugment* augment = nullptr);
+                        const GemmAugment* augment = nullptr, const GemmReduce* reduce = nullptr,
+                        const QkvReduceArgs* qkv = nullptr);
+// (qkv with reduce: the reduced output is the fused QKV projection and the
+// kernel finishes it as launch_qkv_reduce would, writing no output slice;
+// qkv->part and qkv->splits are ignored.)
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {
