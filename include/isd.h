@@ -254,7 +254,7 @@ int isd_paged_attention(const void *q_dev, const int32_t *row_pos_dev, const voi
                         int32_t *status_dev, void *stream);
 
 /* Host-only query of the work split of the tcgen05 attention kernel (head_dim
- * 128, 64-key pages, at most 32 query rows per KV head): no GPU work. The
+ * 128, 64-key pages, at most 64 query rows per KV head): no GPU work. The
  * kernel runs one CTA per SM over the (request, KV head, 128-key tile)
  * sequence; each CTA takes a contiguous range in which every (request, KV
  * head) segment counts as 2 tiles besides its own tiles, and a pair cut

@@ -49,6 +49,7 @@ struct AttnParams {
   // tcgen05 kernel: balanced contiguous tile ranges
   int32_t max_parts;           // partial slots per (request, KV head)
   int32_t min_tiles;           // fewest tiles per CTA (fewer CTAs for small work)
+  int32_t kstages, vstages;    // K and V ring slots
   int32_t* status;
 };
 
@@ -472,10 +473,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
-// tcgen05 variant (head_dim 128, 64-key pages, at most 32 query rows per KV
-// head): the contractions run on the 5th-generation tensor cores with fp32
-// accumulators in tensor memory, so the tile math no longer competes with
-// the HBM stream.
+// tcgen05 variant (head_dim 128, 64-key pages, at most 64 query rows per KV
+// head, in tiles of NP = 32 or 64 rows): the contractions run on the
+// 5th-generation tensor cores with fp32 accumulators in tensor memory, so the
+// tile math no longer competes with the HBM stream. At NP = 64 (Qwen3-32B's
+// 56 rows; prefill passes) S and O take all 512 TMEM columns, P^T rows are
+// 128 bytes (128-byte swizzle) and the V ring is one slot shorter.
 //
 // Per 128-key tile (two pages) of a work item:
 //   S^T[key][row] = K Q^T     UMMA M = 128 keys, N = 32 rows, K = 128 dims
@@ -501,19 +504,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // The work split and the partial-sum format are shared with the mma.sync
 // kernel; the same combine kernel finishes.
 constexpr int kTcKeys = 128;                 // keys per tile (two 64-key pages)
-constexpr int kTcNP = 32;                    // query rows per tile (UMMA N)
+constexpr int kTcMaxNP = 64;                 // most query rows per tile (UMMA N: 32 or 64)
 constexpr int kTcSoftWarps = 8;              // two per TMEM lane quadrant
-constexpr int kTcRows = kTcNP / 2;           // query rows per softmax warp
 constexpr int kTcThreads = (kTcSoftWarps + 3) * 32;
 constexpr int kTcSlot = kTcKeys * 128 * 2;        // one K or V tile, 32 KB
-constexpr int kTcStage = 2 * kTcSlot;             // a K slot and a V slot, 64 KB
 constexpr int kTcHalf = 64 * 128;                 // one [64 keys][64 dims] box, 8 KB
-constexpr int kTcQBuf = 2 * kTcNP * 128;          // Q: two 64-dim halves of NP rows, 8 KB
-constexpr int kTcPBuf = kTcKeys * kTcNP * 2;      // P^T: [128 keys][NP rows] bf16, 8 KB
-constexpr int kTcMisc = 2048;                     // reduction scratch, row state
 constexpr int kTcBars = 256;
 constexpr int kTcMinTiles = 2;                    // fewest tiles per working CTA
-constexpr int kTcMaxStages = (kTcBars / 8 - 16) / 4;   // barriers: 4 per stage + 16
+constexpr int kTcMaxStages = 3;                   // slots per ring (barriers: 2 per slot + 16)
+// Per NP (query rows of a tile: 32, or 64 for groups of up to 64 rows):
+// Q: two 64-dim halves of NP rows; P^T: [128 keys][NP rows] bf16; reduction
+// scratch and row state
+__host__ __device__ constexpr int tc_qbuf(int np) { return 2 * np * 128; }
+__host__ __device__ constexpr int tc_pbuf(int np) { return kTcKeys * np * 2; }
+__host__ __device__ constexpr int tc_misc(int np) { return np <= 32 ? 2048 : 3072; }
 
 // Max or sum of v[0..15] over the 32 lanes, reduce-scatter style: after 16
 // shuffles lanes 2i and 2i+1 both hold the reduction of value i.
@@ -667,33 +671,37 @@ __host__ __device__ __forceinline__ bool tc_next(const AttnParams& p, const int*
   return false;
 }
 
+template <int NP>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                    const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
-  constexpr int NP = kTcNP;
-  constexpr int NR = kTcRows;
+  constexpr int NR = NP / 2;                 // query rows per softmax warp
+  constexpr int kQBuf = tc_qbuf(NP);
+  constexpr int kPBuf = tc_pbuf(NP);
+  constexpr int kRowWarps = NP / 32;         // warps that keep the per-row state
   constexpr int kSoftThreads = kTcSoftWarps * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* ring_k = smem;                                 // stages x K tile
-  uint8_t* ring_v = ring_k + p.stages * kTcSlot;          // stages x V tile
-  uint8_t* qs = ring_v + p.stages * kTcSlot;              // 2 x Q
-  uint8_t* ps = qs + 2 * kTcQBuf;                         // P^T
-  float* red = reinterpret_cast<float*>(ps + kTcPBuf);    // [4 quadrants][NP]
+  const int KS = p.kstages, VS = p.vstages;
+  uint8_t* ring_k = smem;                                 // KS x K tile
+  uint8_t* ring_v = ring_k + KS * kTcSlot;                // VS x V tile
+  uint8_t* qs = ring_v + VS * kTcSlot;                    // 2 x Q
+  uint8_t* ps = qs + 2 * kQBuf;                           // P^T
+  float* red = reinterpret_cast<float*>(ps + kPBuf);      // [4 quadrants][NP]
   float* m_sh = red + 4 * NP;                             // running max per row (log2 units)
   float* alpha_sh = m_sh + NP;                            // [2][NP] per-tile rescale
   float* l_sh = alpha_sh + 2 * NP;                        // row sums at item end
   float* mu_sh = l_sh + NP;                               // exponent offset (m, 0 while m = -inf)
   int* pos_sh = reinterpret_cast<int*>(mu_sh + NP);       // row positions of the item
-  int* minpos_sh = pos_sh + NP;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kTcMisc);
-  uint64_t* full_k = bars;                 // [stages] each
-  uint64_t* empty_k = full_k + p.stages;
-  uint64_t* full_v = empty_k + p.stages;
-  uint64_t* empty_v = full_v + p.stages;
-  uint64_t* q_full = empty_v + p.stages;   // [2]
+  int* minpos_sh = pos_sh + NP;                           // [kRowWarps]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + tc_misc(NP));
+  uint64_t* full_k = bars;                 // [KS] each
+  uint64_t* empty_k = full_k + KS;
+  uint64_t* full_v = empty_k + KS;         // [VS] each
+  uint64_t* empty_v = full_v + VS;
+  uint64_t* q_full = empty_v + VS;         // [2]
   uint64_t* q_empty = q_full + 2;          // [2]
   uint64_t* s_full = q_empty + 2;          // [2]
   uint64_t* s_empty = s_full + 2;          // [2]
@@ -707,9 +715,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* base = kend + p.B;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.stages; ++i) {
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&full_k[i], 1);
       mbar_init(&empty_k[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
       mbar_init(&full_v[i], 1);
       mbar_init(&empty_v[i], 1);
     }
@@ -728,7 +738,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_barrier_init();
   }
   // query rows past the tile's RG rows are never loaded: keep them zero
-  for (int i = threadIdx.x; i < 2 * kTcQBuf / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < 2 * kQBuf / 16; i += blockDim.x)
     reinterpret_cast<int4*>(qs)[i] = make_int4(0, 0, 0, 0);
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 0) {
@@ -763,13 +773,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         mbar_arrive_expect_tx(&q_full[qb], 2 * p.RG * 128);
         for (int hh = 0; hh < 2; ++hh)
-          tma_load_3d(qs + qb * kTcQBuf + hh * (NP * 128), &qmap, &q_full[qb], hh * 64, g * p.G,
+          tma_load_3d(qs + qb * kQBuf + hh * (NP * 128), &qmap, &q_full[qb], hh * 64, g * p.G,
                       b * p.R);
         ++q_issued;
         const int32_t* pt = p.page_table + static_cast<int64_t>(b) * p.maxp;
         for (int t = 0; t < n_tiles; ++t, ++tc) {
-          const int st = tc % p.stages;
-          const uint32_t ph = ((tc / p.stages) & 1) ^ 1;
+          const int st = tc % KS, sv = tc % VS;
+          const uint32_t ph = ((tc / KS) & 1) ^ 1, phv = ((tc / VS) & 1) ^ 1;
           int rows[2];
           for (int j = 0; j < 2; ++j) {
             const int key0 = k_lo + t * kTcKeys + j * 64;
@@ -796,24 +806,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ++nk;
           // V as [page][dim half]: each page is 16 keys per MMA k-step, dim
           // halves LBO apart
-          if (!mbar_wait(&empty_v[st], ph)) {
+          if (!mbar_wait(&empty_v[sv], phv)) {
             ok = false;
             break;
           }
-          uint8_t* vs = ring_v + st * kTcSlot;
-          mbar_arrive_expect_tx(&full_v[st], kTcSlot);
+          uint8_t* vs = ring_v + sv * kTcSlot;
+          mbar_arrive_expect_tx(&full_v[sv], kTcSlot);
           for (int j = 0; j < 2; ++j)
             for (int hh = 0; hh < 2; ++hh)
-              tma_load_2d(vs + j * 2 * kTcHalf + hh * kTcHalf, &vmap, &full_v[st], hh * 64, rows[j]);
+              tma_load_2d(vs + j * 2 * kTcHalf + hh * kTcHalf, &vmap, &full_v[sv], hh * 64, rows[j]);
         }
       }
       if (!ok) flag(p.status, ISD_DEV_TIMEOUT);
       // copies in flight land before the CTA exits (after a timeout the last
       // K load may have no V load beside it)
-      for (int j = max(0, nk - p.stages); j < nk; ++j)
-        if (!mbar_wait(&full_k[j % p.stages], (j / p.stages) & 1)) break;
-      for (int j = max(0, tc - p.stages); j < tc; ++j)
-        if (!mbar_wait(&full_v[j % p.stages], (j / p.stages) & 1)) break;
+      for (int j = max(0, nk - KS); j < nk; ++j)
+        if (!mbar_wait(&full_k[j % KS], (j / KS) & 1)) break;
+      for (int j = max(0, tc - VS); j < tc; ++j)
+        if (!mbar_wait(&full_v[j % VS], (j / VS) & 1)) break;
       if (q_issued > 0) mbar_wait(&q_full[(q_issued - 1) & 1], ((q_issued - 1) >> 1) & 1);
     }
   } else if (warp == kTcSoftWarps + 1) {
@@ -832,10 +842,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
-        const uint64_t b0 = sw128_desc(q_a + qb * kTcQBuf);
+        const uint64_t b0 = sw128_desc(q_a + qb * kQBuf);
         for (int t = 0; t < n_tiles; ++t, ++tc) {
-          const int st = tc % p.stages;
-          if (!mbar_wait(&full_k[st], (tc / p.stages) & 1) ||
+          const int st = tc % KS;
+          if (!mbar_wait(&full_k[st], (tc / KS) & 1) ||
               !mbar_wait(&s_empty[tc & 1], ((tc >> 1) & 1) ^ 1)) {
             ok = false;
             break;
@@ -869,7 +879,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // A (V^T) and B (P^T) both MN-major
       const uint32_t idesc_o = idesc_bf16(128, NP) | (1u << 15) | (1u << 16);
       const uint32_t rv_a = smem_u32(ring_v);
-      const uint64_t b0 = sw64_desc_mn(smem_u32(ps));
+      // P^T rows of NP bf16: 64 bytes (64-byte swizzle) or 128 bytes (128-byte swizzle)
+      const uint64_t b0 = NP == 32 ? sw64_desc_mn(smem_u32(ps)) : sw128_desc_mn(smem_u32(ps), 8192);
       int n_total = 0;
       {
         TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
@@ -878,9 +889,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       bool ok = true;
       for (int j = 0; j < n_total; ++j) {
-        const int st = j % p.stages;
+        const int st = j % VS;
         if (!mbar_wait(p_full, j & 1) || !mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1) ||
-            !mbar_wait(&full_v[st], (j / p.stages) & 1)) {
+            !mbar_wait(&full_v[st], (j / VS) & 1)) {
           ok = false;
           break;
         }
@@ -910,9 +921,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r0 = (warp >> 2) * NR;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const int kl = quad * 32 + lane;           // key within the tile; dim for O
-    // P^T row of this thread's key: 64 bytes, 16-byte chunks swizzled by key
+    // P^T row of this thread's key: NP bf16 (64 or 128 bytes), 16-byte chunks
+    // swizzled by key (64- or 128-byte swizzle)
     uint8_t* p_row = ps + kl * (NP * 2);
-    const int p_sw = (kl >> 1) & 3;
+    const int p_sw = NP == 32 ? (kl >> 1) & 3 : kl & 7;
+    const int my_row = warp * 32 + lane;       // the row whose state this thread keeps (warps < kRowWarps)
     float o[NR];
     float ls[NR];
     int tc = 0;
@@ -920,25 +933,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
     TcSeg sg;
     bool have = tc_next(p, base, rg, sg);
-    // row positions are loaded one segment ahead (warp 0, lane = row)
-    int pr_cur = warp == 0 && have && lane < p.RG ? p.row_pos[sg.b * p.R + lane / p.G] : -1;
+    // row positions are loaded one segment ahead (warps < kRowWarps, one row per thread)
+    int pr_cur = warp < kRowWarps && have && my_row < p.RG ? p.row_pos[sg.b * p.R + my_row / p.G] : -1;
     while (have) {
       TcSeg nx;
       const bool have_nx = tc_next(p, base, rg, nx);
       const int pr_nx =
-          warp == 0 && have_nx && lane < p.RG ? p.row_pos[nx.b * p.R + lane / p.G] : -1;
+          warp < kRowWarps && have_nx && my_row < p.RG ? p.row_pos[nx.b * p.R + my_row / p.G] : -1;
       const int b = sg.b;
       const int k_lo = sg.t0 * kTcKeys;
       const int k_hi = min(kend[b], k_lo + sg.len * kTcKeys);
       const int n_tiles = sg.len;
-      if (warp == 0) {
+      if (warp < kRowWarps) {
         const int pr = pr_cur;
-        pos_sh[lane] = pr;
-        m_sh[lane] = -INFINITY;
-        int mn = lane < p.RG ? pr : INT_MAX;
+        pos_sh[my_row] = pr;
+        m_sh[my_row] = -INFINITY;
+        int mn = my_row < p.RG ? pr : INT_MAX;
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o2));
-        if (lane == 0) *minpos_sh = mn;
+        if (lane == 0) minpos_sh[warp] = mn;
       }
 #pragma unroll
       for (int r = 0; r < NR; ++r) {
@@ -946,20 +959,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ls[r] = 0.f;
       }
       named_bar_sync(2, kSoftThreads);
-      const int minpos = *minpos_sh;
+      int minpos = minpos_sh[0];
+#pragma unroll
+      for (int w2 = 1; w2 < kRowWarps; ++w2) minpos = min(minpos, minpos_sh[w2]);
       for (int t = 0; t < n_tiles; ++t, ++tc) {
         const int sb = tc & 1;
         // ---- S tile -> registers
         fine = fine && mbar_wait(&s_full[sb], (tc >> 1) & 1);
         tc_fence_after();
         float x[NR];
-        {
+#pragma unroll
+        for (int gq = 0; gq < NR / 16; ++gq) {
           uint32_t ra[16], rb[16];
-          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + r0, ra);
-          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + NP + r0, rb);
+          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + r0 + gq * 16, ra);
+          tmem_ld_32x32_x16(lane_base + sb * 2 * NP + NP + r0 + gq * 16, rb);
           tmem_ld_wait();
 #pragma unroll
-          for (int r = 0; r < NR; ++r) x[r] = __uint_as_float(ra[r]) + __uint_as_float(rb[r]);
+          for (int r = 0; r < 16; ++r)
+            x[gq * 16 + r] = __uint_as_float(ra[r]) + __uint_as_float(rb[r]);
         }
         tc_fence_before();
         __syncwarp();
@@ -989,14 +1006,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           fine = false;
           break;
         }
-        if (warp == 0) {
-          const float m_old = m_sh[lane];
-          const float mt = fmaxf(fmaxf(red[lane], red[NP + lane]), fmaxf(red[2 * NP + lane], red[3 * NP + lane]));
+        if (warp < kRowWarps) {
+          const int q = my_row;
+          const float m_old = m_sh[q];
+          const float mt = fmaxf(fmaxf(red[q], red[NP + q]), fmaxf(red[2 * NP + q], red[3 * NP + q]));
           const float m_new = fmaxf(m_old, mt * p.scale_log2);
-          alpha_sh[sb * NP + lane] = m_new == -INFINITY ? 1.f : ex2(m_old - m_new);
-          m_sh[lane] = m_new;
+          alpha_sh[sb * NP + q] = m_new == -INFINITY ? 1.f : ex2(m_old - m_new);
+          m_sh[q] = m_new;
           // a row with no key yet: every x is -inf and 2^(x - 0) = 0
-          mu_sh[lane] = m_new == -INFINITY ? 0.f : m_new;
+          mu_sh[q] = m_new == -INFINITY ? 0.f : m_new;
         }
         named_bar_sync(2, kSoftThreads);
         // ---- P = 2^(x scale - m), partial row sums, P^T to shared memory
@@ -1017,14 +1035,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fine = fine && mbar_wait(p_empty, (tc & 1) ^ 1);
         {
-          // rows r0 .. r0 + 7 and r0 + 8 .. r0 + 15: 16-byte chunks r0/8 and r0/8 + 1
-          const uint4 c0 = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]),
-                                      pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          const uint4 c1 = make_uint4(pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]),
-                                      pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
+          // rows r0 + 8 cc .. r0 + 8 cc + 7: 16-byte chunk r0 / 8 + cc of the key's row
           const int ch = r0 >> 3;
-          *reinterpret_cast<uint4*>(p_row + ((ch ^ p_sw) << 4)) = c0;
-          *reinterpret_cast<uint4*>(p_row + (((ch + 1) ^ p_sw) << 4)) = c1;
+#pragma unroll
+          for (int cc = 0; cc < NR / 8; ++cc) {
+            const uint4 cv = make_uint4(pack_bf16(x[8 * cc], x[8 * cc + 1]),
+                                        pack_bf16(x[8 * cc + 2], x[8 * cc + 3]),
+                                        pack_bf16(x[8 * cc + 4], x[8 * cc + 5]),
+                                        pack_bf16(x[8 * cc + 6], x[8 * cc + 7]));
+            *reinterpret_cast<uint4*>(p_row + (((ch + cc) ^ p_sw) << 4)) = cv;
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
@@ -1034,17 +1054,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int j = tc - 1;
           fine = fine && mbar_wait(&o_full[j & 1], (j >> 1) & 1);
           tc_fence_after();
-          uint32_t ra[16], rb[16];
-          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0, ra);
-          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0, rb);
-          tmem_ld_wait();
+#pragma unroll
+          for (int gq = 0; gq < NR / 16; ++gq) {
+            uint32_t ra[16], rb[16];
+            tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0 + gq * 16, ra);
+            tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0 + gq * 16, rb);
+            tmem_ld_wait();
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+              o[gq * 16 + r] = o[gq * 16 + r] * alpha_sh[(j & 1) * NP + r0 + gq * 16 + r] +
+                               (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&o_empty[j & 1]);
-#pragma unroll
-          for (int r = 0; r < NR; ++r)
-            o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] +
-                   (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
         }
       }
       if (!fine) break;
@@ -1052,33 +1075,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int j = tc - 1;
         fine = mbar_wait(&o_full[j & 1], (j >> 1) & 1);
         tc_fence_after();
-        uint32_t ra[16], rb[16];
-        tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0, ra);
-        tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0, rb);
-        tmem_ld_wait();
+#pragma unroll
+        for (int gq = 0; gq < NR / 16; ++gq) {
+          uint32_t ra[16], rb[16];
+          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + r0 + gq * 16, ra);
+          tmem_ld_32x32_x16(lane_base + 4 * NP + (j & 1) * 2 * NP + NP + r0 + gq * 16, rb);
+          tmem_ld_wait();
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+            o[gq * 16 + r] = o[gq * 16 + r] * alpha_sh[(j & 1) * NP + r0 + gq * 16 + r] +
+                             (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&o_empty[j & 1]);
-#pragma unroll
-        for (int r = 0; r < NR; ++r)
-          o[r] = o[r] * alpha_sh[(j & 1) * NP + r0 + r] +
-                 (__uint_as_float(ra[r]) + __uint_as_float(rb[r]));
       }
       // ---- row sums over the 128 key lanes, then the partial output
-      {
-        const float sm = lane_reduce16<false>(ls, lane);
-        if ((lane & 1) == 0) red[quad * NP + r0 + (lane >> 1)] = sm;
+#pragma unroll
+      for (int gq = 0; gq < NR / 16; ++gq) {
+        float l16[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) l16[r] = ls[gq * 16 + r];
+        const float sm = lane_reduce16<false>(l16, lane);
+        if ((lane & 1) == 0) red[quad * NP + r0 + gq * 16 + (lane >> 1)] = sm;
       }
       if (!named_bar_and(2, kSoftThreads, fine)) {
         fine = false;
         break;
       }
-      if (warp == 0) {
-        const float L = (red[lane] + red[NP + lane]) + (red[2 * NP + lane] + red[3 * NP + lane]);
-        l_sh[lane] = L;
+      if (warp < kRowWarps) {
+        const int q = my_row;
+        const float L = (red[q] + red[NP + q]) + (red[2 * NP + q] + red[3 * NP + q]);
+        l_sh[q] = L;
         if (sg.slot >= 0)
-          p.part_ml[static_cast<int64_t>(sg.slot) * NP + lane] = make_float2(m_sh[lane], L);
-        else if (lane == 0)
+          p.part_ml[static_cast<int64_t>(sg.slot) * NP + q] = make_float2(m_sh[q], L);
+        else if (q == 0)
           flag(p.status, ISD_DEV_BAD_STATE);
       }
       named_bar_sync(2, kSoftThreads);
@@ -1157,11 +1188,12 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p, _
 // Combine for the tcgen05 kernel's balanced ranges: (request b, KV head g)
 // has parts from CTAs c(first tile) .. c(last tile), in slots
 // (b * nkv + g) * max_parts + 0 .. parts - 1. Same merge as above.
+template <int NP>
 __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p, int C_grid,
                                                               __nv_bfloat16* out) {
   constexpr int HD = 128;
   const int g = blockIdx.x, b = blockIdx.y;
-  __shared__ float w[kTcNP][kMaxSplits];
+  __shared__ float w[NP][kMaxSplits];
   const int* base = p.item_base;
   const int64_t U = tc_ubase(p, base, p.B);
   const int nt = base[b + 1] - base[b];
@@ -1178,11 +1210,11 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p
   const int64_t slot0 = static_cast<int64_t>(b * p.nkv + g) * p.max_parts;
   for (int qi = threadIdx.x; qi < p.RG; qi += blockDim.x) {
     float M = -INFINITY;
-    for (int s = 0; s < parts; ++s) M = fmaxf(M, p.part_ml[(slot0 + s) * kTcNP + qi].x);
+    for (int s = 0; s < parts; ++s) M = fmaxf(M, p.part_ml[(slot0 + s) * NP + qi].x);
     const float Rm = M == -INFINITY ? 0.f : M;
     float L = 0.f;
     for (int s = 0; s < parts; ++s) {
-      const float2 ml = p.part_ml[(slot0 + s) * kTcNP + qi];
+      const float2 ml = p.part_ml[(slot0 + s) * NP + qi];
       const float ws = ml.y * exp2f(ml.x - Rm);
       w[qi][s] = ws;
       L += ws;
@@ -1193,7 +1225,7 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p
   __syncthreads();
   // part-major: every load of one part is in flight at once (one L2 round
   // trip per part); each output still sums its parts in part order
-  constexpr int kVec = kTcNP * (HD / 4) / 128;   // float4 outputs per thread
+  constexpr int kVec = NP * (HD / 4) / 128;   // float4 outputs per thread
   float4 acc[kVec];
 #pragma unroll
   for (int j = 0; j < kVec; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1204,7 +1236,7 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p
       if (i < p.RG * (HD / 4)) {
         const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
         const float ws = w[qi][s];
-        const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * kTcNP + qi) * HD + d);
+        const float4 v = *reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * NP + qi) * HD + d);
         acc[j].x += ws * v.x;
         acc[j].y += ws * v.y;
         acc[j].z += ws * v.z;
@@ -1230,12 +1262,15 @@ struct Derived {
   int RG, MT, NG, split_keys, max_splits, stages, max_items;
   int min_tiles = 1;
   bool tc;        // the tcgen05 kernel serves this shape
+  int np = 32;    // its query rows per tile
+  int kstages = 0, vstages = 0;
   size_t smem;
 };
 
 // Shared memory of the tcgen05 kernel for a batch of B requests.
-size_t tc_smem(int stages, int B) {
-  return 1024 + static_cast<size_t>(stages) * kTcStage + 2 * kTcQBuf + kTcPBuf + kTcMisc + kTcBars +
+size_t tc_smem(int np, int kstages, int vstages, int B) {
+  return 1024 + static_cast<size_t>(kstages + vstages) * kTcSlot + 2 * tc_qbuf(np) + tc_pbuf(np) +
+         tc_misc(np) + kTcBars +
          16 + (2 * static_cast<size_t>(B) + 1) * sizeof(int);
 }
 
@@ -1243,7 +1278,9 @@ Derived derive(const AttnShape& s) {
   Derived d;
   const int G = s.n_q_heads / s.n_kv_heads;
   d.RG = s.rows_per_req * G;
-  d.tc = s.head_dim == 128 && s.page_size == 64 && d.RG <= kTcNP && tc_smem(2, s.batch) <= 232448;
+  d.np = d.RG <= 32 ? 32 : 64;
+  d.tc = s.head_dim == 128 && s.page_size == 64 && d.RG <= kTcMaxNP &&
+         tc_smem(d.np, 2, 2, s.batch) <= 232448;
   if (d.tc) {
     // one CTA per SM, equal contiguous tile ranges of at least kTcMinTiles
     // tiles; a (request, head) run of n tiles then spans at most
@@ -1255,11 +1292,16 @@ Derived derive(const AttnShape& s) {
         std::max<int64_t>(kTcMinTiles, (max_tiles + kMaxSplits - 2) / (kMaxSplits - 1)));
     d.max_splits = static_cast<int>((max_tiles + d.min_tiles - 1) / d.min_tiles + 1);
     d.max_items = s.batch * s.n_kv_heads * d.max_splits;
-    d.MT = kTcNP / 16;
+    d.MT = d.np / 16;
     d.NG = 1;
-    d.stages = kTcMaxStages;
-    while (d.stages > 2 && tc_smem(d.stages, s.batch) > 232448) --d.stages;
-    d.smem = tc_smem(d.stages, s.batch);
+    // the deepest rings that fit, the K ring first (a K slot frees as soon as
+    // S is computed, a V slot only after the softmax and PV)
+    d.kstages = kTcMaxStages;
+    d.vstages = kTcMaxStages;
+    while (d.vstages > 2 && tc_smem(d.np, d.kstages, d.vstages, s.batch) > 232448) --d.vstages;
+    while (d.kstages > 2 && tc_smem(d.np, d.kstages, d.vstages, s.batch) > 232448) --d.kstages;
+    d.stages = d.kstages;
+    d.smem = tc_smem(d.np, d.kstages, d.vstages, s.batch);
     return d;
   }
   d.MT = (d.RG + 15) / 16;
@@ -1416,18 +1458,29 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
   if (d.tc) {
     static bool tc_attr = false;
     if (!tc_attr) {
-      const cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel),
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<32>),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(reinterpret_cast<const void*>(attn_tc_kernel<64>),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
       if (e != cudaSuccess) return e;
       tc_attr = true;
     }
     p.max_parts = d.max_splits;
     p.min_tiles = d.min_tiles;
-    attn_tc_kernel<<<sms, kTcThreads, d.smem, stream>>>(k_map, v_map, qmap, p);
+    p.kstages = d.kstages;
+    p.vstages = d.vstages;
+    if (d.np == 32)
+      attn_tc_kernel<32><<<sms, kTcThreads, d.smem, stream>>>(k_map, v_map, qmap, p);
+    else
+      attn_tc_kernel<64><<<sms, kTcThreads, d.smem, stream>>>(k_map, v_map, qmap, p);
     const cudaError_t le = cudaGetLastError();
     if (le != cudaSuccess) return le;   // the combine reads what this kernel writes
     if (between) cudaEventRecord(between, stream);
-    attn_combine_tc_kernel<<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
+    if (d.np == 32)
+      attn_combine_tc_kernel<32><<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
+    else
+      attn_combine_tc_kernel<64><<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
     if (launches) *launches += 2;
     return cudaGetLastError();
   }

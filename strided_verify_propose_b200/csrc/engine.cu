@@ -159,6 +159,9 @@ struct isd_ctx {
   size_t sk_ws_bytes = 0;
   int32_t* red_cnt = nullptr;       // arrival / departure counters of in-kernel split-K reduction
   int32_t red_cnt_n = 0;
+  float* rn_ss = nullptr;           // [hidden / 128][rn_ss_stride] per-tile row sums of squares
+  int32_t rn_ss_stride = 0;         // rows (the step rows: batch x (2N - 1) at most)
+  int32_t* rn_cnt = nullptr;        // [2] grid barrier of the fused residual + RMSNorm
   std::map<std::tuple<int, int, int, int>, int> coresident;   // per plan: CTAs resident at once
   int launches = 0;
 
@@ -263,7 +266,8 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
          const AugSpec* aug = nullptr, float** reduce_out = nullptr,
-         const isd::QkvReduceArgs* qkv = nullptr, bool* qkv_fused = nullptr) {
+         const isd::QkvReduceArgs* qkv = nullptr, bool* qkv_fused = nullptr,
+         const isd::ResNormArgs* rn = nullptr) {
   if (epi == isd::kEpiF32 && out_elems > 0) {
     // large prefill chunks: no more splits than the partial buffer holds
     const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
@@ -309,9 +313,9 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, result, act, status, st, c->sk_ws,
                             c->sk_ws_bytes, aug ? &ga : nullptr, reduced ? &red : nullptr,
-                            reduced ? qkv : nullptr));
+                            reduced ? qkv : nullptr, reduced ? rn : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
-  if (qkv_fused) *qkv_fused = reduced && qkv != nullptr;
+  if (qkv_fused) *qkv_fused = reduced && (qkv != nullptr || rn != nullptr);
   if (splits_used) *splits_used = reduced ? 1 : plan.splits;
   if (reduce_out) *reduce_out = result;
   c->launches += 1;
@@ -488,13 +492,20 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_o, c->attn, M, c->q_dim, r, status, st);
       if (rc) return rc;
     }
+    // the O projection; a reduced split-K GEMM also adds the residual and
+    // applies the MLP's RMSNorm
+    isd::ResNormArgs rn_o{c->x, c->mlp_norm[l], g.rms_eps, c->hn, c->rn_ss, c->rn_ss_stride,
+                          c->rn_cnt};
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
-              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr, &slices);
+              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr, &slices, nullptr,
+              &fused, M <= c->rn_ss_stride ? &rn_o : nullptr);
     if (rc) return rc;
-    cudaEvent_t r0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
-    prof_add(c, kPResNorm, r0, prof_mark(c, st));
-    c->launches += 1;
+    if (!fused) {
+      cudaEvent_t r0 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
+      prof_add(c, kPResNorm, r0, prof_mark(c, st));
+      c->launches += 1;
+    }
     // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
     // K-blocks follow each tile's base K-blocks (stream-K cuts unchanged)
     AugSpec aug_gu{ll ? &ll->tb_gu : nullptr, c->lora_xa, 2 * r};
@@ -510,14 +521,18 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_d, c->act, M, g.intermediate, r, status, st);
       if (rc) return rc;
     }
-    rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr, &slices);
-    if (rc) return rc;
     const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
-    cudaEvent_t r1 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
-    prof_add(c, kPResNorm, r1, prof_mark(c, st));
-    c->launches += 1;
+    isd::ResNormArgs rn_d{c->x, next_norm, g.rms_eps, c->hn, c->rn_ss, c->rn_ss_stride, c->rn_cnt};
+    rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr, &slices,
+              nullptr, &fused, M <= c->rn_ss_stride ? &rn_d : nullptr);
+    if (rc) return rc;
+    if (!fused) {
+      cudaEvent_t r1 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
+      prof_add(c, kPResNorm, r1, prof_mark(c, st));
+      c->launches += 1;
+    }
   }
   return ISD_OK;
 }
@@ -576,6 +591,8 @@ int alloc_workspace(isd_ctx* c) {
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
       static_cast<size_t>(2 * (wide / 128) * 8) * 4,      // split-K reduction counters
+      static_cast<size_t>(g.hidden / 128) * step_rows * 4,  // residual + norm: tile sums
+      256,                                                  // residual + norm: grid barrier
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -607,8 +624,12 @@ int alloc_workspace(isd_ctx* c) {
   c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
   c->red_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
   c->red_cnt_n = static_cast<int32_t>(2 * (wide / 128) * 8);
+  c->rn_ss = reinterpret_cast<float*>(b + off[i++]);
+  c->rn_ss_stride = static_cast<int32_t>(step_rows);
+  c->rn_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
   if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
-      cudaMemset(c->red_cnt, 0, static_cast<size_t>(c->red_cnt_n) * 4) != cudaSuccess)
+      cudaMemset(c->red_cnt, 0, static_cast<size_t>(c->red_cnt_n) * 4) != cudaSuccess ||
+      cudaMemset(c->rn_cnt, 0, 256) != cudaSuccess)
     return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;

@@ -42,6 +42,9 @@ constexpr int kTileK = 64;                  // K elements per stage (128 bytes)
 constexpr int kStageA = kTileM * kTileK * 2;  // 16 KB
 constexpr size_t kMaxSmem = 231424;         // 226 KB dynamic (+ a few static bytes <= 227 KB)
 constexpr int kEpiWarps = 8;                // epilogue warps (two per TMEM quadrant)
+constexpr int kMaxChunksPerWarp = 8;        // 32-token chunks per epilogue warp (512 tokens / 32 / 2)
+constexpr int kRedRows = 2;                 // rows per warp per round of the in-kernel split-K sum
+constexpr int kRedSplits = 4;               // splits whose loads are unrolled (more take a loop)
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 struct GemmParams {
@@ -73,6 +76,9 @@ struct GemmParams {
   // reduce == 2: the reduced output is the fused QKV projection; instead of
   // writing it, apply QK-norm and RoPE and write q and the K/V page slots
   QkvReduceArgs qkv;
+  // reduce == 3: the reduced output is added to the residual stream and the
+  // next RMSNorm follows (after a barrier over the whole grid)
+  ResNormArgs rn;
 };
 
 // QK-norm + NeoX RoPE + q / KV-page writes for one token row of one
@@ -436,7 +442,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       // TMEM loads run one chunk ahead of the chunk being written out
       uint32_t r[32];
       if (half < nchunk) tmem_ld_32x32_async(lane_addr + half * 32, r);
-      for (int c = half; c < nchunk; c += 2) {
+      // SwiGLU tiles: the bf16 results stay in registers until every chunk is
+      // read, then the accumulator is released and the stores follow, so the
+      // next tile's MMAs run while this tile's results leave
+      const bool staged = p.epi == kEpiSiluMul && (mode == 0 || mode == 2);
+      bool released = false;
+      if (staged) {
+        const bool hi = lane >= 16;
+        uint32_t ov[kMaxChunksPerWarp * 8];   // [chunk][8]: token pairs (2k, 2k + 1) of 16 results
+#pragma unroll
+        for (int ci = 0; ci < kMaxChunksPerWarp; ++ci) {
+          const int c = half + 2 * ci;
+          if (c < nchunk) {
+            float v[32];
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (c + 2 < nchunk) tmem_ld_32x32_async(lane_addr + (c + 2) * 32, r);
+            if (mode == 2) {
+              const float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += __ldcg(pp + j * kTileM);
+            }
+            // gate and up rows of a feature sit 16 lanes apart: low lanes
+            // finish even tokens, high lanes odd ones
+#pragma unroll
+            for (int k = 0; k < 16; k += 2) {
+              float o2[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = 2 * (k + e);
+                const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
+                const float x_j1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 16);
+                const float g = hi ? x_j1 : v[j];
+                const float u = hi ? v[j + 1] : x_j;
+                o2[e] = silu_mul(g, u);
+              }
+              __nv_bfloat162 pk = __floats2bfloat162_rn(o2[0], o2[1]);
+              ov[ci * 8 + k / 2] = *reinterpret_cast<uint32_t*>(&pk);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair)
+            mbar_arrive_cluster(empty_addr);
+          else
+            mbar_arrive(tmem_empty);
+        }
+        released = true;
+        const int half_n = p.n_out / 2;
+        const int f = mt * 64 + quad * 16 + (lane & 15);
+#pragma unroll
+        for (int ci = 0; ci < kMaxChunksPerWarp; ++ci) {
+          const int c = half + 2 * ci;
+          if (c < nchunk) {
+            const int t0 = tok0 + c * 32;
+            const bool full_chunk = c * 32 + 32 <= p.n_pad && t0 + 32 <= p.m;
+            __nv_bfloat16* rowp =
+                p.out_act + static_cast<int64_t>(t0 + (hi ? 1 : 0)) * half_n + f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int jj = 2 * k + (hi ? 1 : 0);
+              const uint32_t w = ov[ci * 8 + k / 2];
+              const uint16_t bits = (k & 1) ? static_cast<uint16_t>(w >> 16) : static_cast<uint16_t>(w);
+              if (full_chunk || (c * 32 + jj < p.n_pad && t0 + jj < p.m))
+                *reinterpret_cast<uint16_t*>(rowp) = bits;
+              rowp += 2 * half_n;
+            }
+          }
+        }
+      }
+      for (int c = half; !staged && c < nchunk; c += 2) {
         float v[32];
         tmem_ld_wait();
 #pragma unroll
@@ -499,13 +577,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // accumulators read: release them to the MMA issuer (of the pair)
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (kPair)
-          mbar_arrive_cluster(empty_addr);
-        else
-          mbar_arrive(tmem_empty);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (kPair)
+            mbar_arrive_cluster(empty_addr);
+          else
+            mbar_arrive(tmem_empty);
+        }
       }
       if (mode == 1) {
         // partial parked: publish it
@@ -539,23 +619,134 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t_lo = c_lo * 32, t_hi = min(c_hi * 32, p.n_pad);
           const int64_t sstride = static_cast<int64_t>(nchunk) * 32 * kTileM;
           const float* base = p.red + static_cast<int64_t>(red_tile) * S * sstride;
-          // warp ew takes token rows t_lo + ew, + 8, ...; lane l features 4l..4l+3
+          // warp ew takes token rows t_lo + ew, + 8, ...; lane l features
+          // 4l..4l+3. Rows go kRedRows at a time with every split's load of
+          // them (and the residual's) in flight together; the sum still runs
+          // in split order.
           const int t_end = min(t_hi, p.m - tok0);
-          for (int t = t_lo + ew; t < t_end; t += kEpiWarps) {
-            const float* q = base + static_cast<int64_t>(t) * kTileM + lane * 4;
-            float4 acc = __ldcg(reinterpret_cast<const float4*>(q));
-            for (int s2 = 1; s2 < S; ++s2) {
-              const float4 d = __ldcg(reinterpret_cast<const float4*>(q + s2 * sstride));
-              acc.x += d.x;
-              acc.y += d.y;
-              acc.z += d.z;
-              acc.w += d.w;
+          for (int t = t_lo + ew; t < t_end; t += kEpiWarps * kRedRows) {
+            float4 part4[kRedSplits][kRedRows];
+            float4 xo[kRedRows];
+#pragma unroll
+            for (int rr = 0; rr < kRedRows; ++rr) {
+              const int tr = t + rr * kEpiWarps;
+              const float* q = base + static_cast<int64_t>(tr) * kTileM + lane * 4;
+#pragma unroll
+              for (int s2 = 0; s2 < kRedSplits; ++s2)
+                part4[s2][rr] = (tr < t_end && s2 < S)
+                                    ? __ldcg(reinterpret_cast<const float4*>(q + s2 * sstride))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+              xo[rr] = (p.reduce == 3 && tr < t_end)
+                           ? *reinterpret_cast<const float4*>(
+                                 p.rn.x + static_cast<int64_t>(tok0 + tr) * p.n_out + mt * kTileM + lane * 4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            if (p.reduce == 2)
-              qkv_row_epilogue(p.qkv, acc, tok0 + t, mt, lane);
-            else
-              *reinterpret_cast<float4*>(p.out + static_cast<int64_t>(tok0 + t) * p.n_out +
-                                         mt * kTileM + lane * 4) = acc;
+#pragma unroll
+            for (int rr = 0; rr < kRedRows; ++rr) {
+              const int tr = t + rr * kEpiWarps;
+              if (tr >= t_end) continue;   // uniform across the warp
+              float4 acc = part4[0][rr];
+#pragma unroll
+              for (int s2 = 1; s2 < kRedSplits; ++s2) {
+                if (s2 < S) {
+                  acc.x += part4[s2][rr].x;
+                  acc.y += part4[s2][rr].y;
+                  acc.z += part4[s2][rr].z;
+                  acc.w += part4[s2][rr].w;
+                }
+              }
+              // more splits than the unrolled loads cover
+              for (int s2 = kRedSplits; s2 < S; ++s2) {
+                const float4 d = __ldcg(reinterpret_cast<const float4*>(
+                    base + s2 * sstride + static_cast<int64_t>(tr) * kTileM + lane * 4));
+                acc.x += d.x;
+                acc.y += d.y;
+                acc.z += d.z;
+                acc.w += d.w;
+              }
+              if (p.reduce == 2) {
+                qkv_row_epilogue(p.qkv, acc, tok0 + tr, mt, lane);
+              } else if (p.reduce == 3) {
+                // x += the projection; this tile's share of the row's sum of squares
+                float4 x4 = xo[rr];
+                x4.x += acc.x;
+                x4.y += acc.y;
+                x4.z += acc.z;
+                x4.w += acc.w;
+                *reinterpret_cast<float4*>(p.rn.x + static_cast<int64_t>(tok0 + tr) * p.n_out +
+                                           mt * kTileM + lane * 4) = x4;
+                const float ss = warp_sum(x4.x * x4.x + x4.y * x4.y + x4.z * x4.z + x4.w * x4.w);
+                if (lane == 0) p.rn.ss[static_cast<int64_t>(mt) * p.rn.ss_stride + tok0 + tr] = ss;
+              } else {
+                *reinterpret_cast<float4*>(p.out + static_cast<int64_t>(tok0 + tr) * p.n_out +
+                                           mt * kTileM + lane * 4) = acc;
+              }
+            }
+          }
+        }
+        if (p.reduce == 3) {
+          // every row's residual and tile sums are written once every CTA of
+          // the grid has passed here; then this split normalises its rows
+          const int total = static_cast<int>(gridDim.x * gridDim.y * gridDim.z);
+          __threadfence();
+          named_bar_sync(1, 32 * kEpiWarps);
+          if (ew == 0 && lane == 0) {
+            atomicAdd(&p.rn.grid_cnt[0], 1);
+            int ok_ = epi_mode;
+            const long long t0 = clock64();
+            const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
+            while (ld_acquire_gpu(&p.rn.grid_cnt[0]) < total) {
+              if (clock64() - t0 > limit) {
+                flag(p.status, ISD_DEV_TIMEOUT);
+                ok_ = 0;
+                break;
+              }
+            }
+            epi_mode = ok_;
+          }
+          named_bar_sync(1, 32 * kEpiWarps);
+          if (epi_mode) {
+            const int c_lo = split * nchunk / S, c_hi = (split + 1) * nchunk / S;
+            const int t_lo = c_lo * 32, t_end = min(min(c_hi * 32, p.n_pad), p.m - tok0);
+            const int tiles = p.n_out / kTileM;
+            const float4 w4 = *reinterpret_cast<const float4*>(p.rn.norm_w + mt * kTileM + lane * 4);
+            // kRedRows rows per round, their loads in flight together; the
+            // tile sums of a row are added lane by lane in tile order, then
+            // across lanes by the fixed butterfly
+            for (int t = t_lo + ew; t < t_end; t += kEpiWarps * kRedRows) {
+              float tot[kRedRows];
+              float4 xo[kRedRows];
+#pragma unroll
+              for (int rr = 0; rr < kRedRows; ++rr) {
+                const int tr = t + rr * kEpiWarps;
+                tot[rr] = 0.f;
+                xo[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (tr < t_end) {
+                  const int row = tok0 + tr;
+                  for (int i = lane; i < tiles; i += 32)
+                    tot[rr] += __ldcg(p.rn.ss + static_cast<int64_t>(i) * p.rn.ss_stride + row);
+                  xo[rr] = *reinterpret_cast<const float4*>(
+                      p.rn.x + static_cast<int64_t>(row) * p.n_out + mt * kTileM + lane * 4);
+                }
+              }
+#pragma unroll
+              for (int rr = 0; rr < kRedRows; ++rr) {
+                const int tr = t + rr * kEpiWarps;
+                if (tr >= t_end) continue;   // uniform across the warp
+                const int row = tok0 + tr;
+                const float rstd = rsqrtf(warp_sum(tot[rr]) / p.n_out + p.rn.eps);
+                __align__(8) __nv_bfloat16 o4[4] = {
+                    __float2bfloat16_rn(xo[rr].x * rstd * w4.x), __float2bfloat16_rn(xo[rr].y * rstd * w4.y),
+                    __float2bfloat16_rn(xo[rr].z * rstd * w4.z), __float2bfloat16_rn(xo[rr].w * rstd * w4.w)};
+                *reinterpret_cast<uint2*>(p.rn.hn + static_cast<int64_t>(row) * p.n_out + mt * kTileM +
+                                          lane * 4) = *reinterpret_cast<const uint2*>(o4);
+              }
+            }
+          }
+          named_bar_sync(1, 32 * kEpiWarps);
+          if (ew == 0 && lane == 0 && atomicAdd(&p.rn.grid_cnt[1], 1) == total - 1) {
+            p.rn.grid_cnt[0] = 0;
+            p.rn.grid_cnt[1] = 0;
           }
         }
         named_bar_sync(1, 32 * kEpiWarps);
@@ -734,7 +925,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace, size_t sk_workspace_bytes,
                         const GemmAugment* augment, const GemmReduce* reduce,
-                        const QkvReduceArgs* qkv) {
+                        const QkvReduceArgs* qkv, const ResNormArgs* rn) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -795,6 +986,12 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
         return cudaErrorInvalidValue;
       p.reduce = 2;
       p.qkv = *qkv;
+    } else if (rn != nullptr) {
+      if (rn->x == nullptr || rn->norm_w == nullptr || rn->hn == nullptr || rn->ss == nullptr ||
+          rn->grid_cnt == nullptr || rn->ss_stride < m)
+        return cudaErrorInvalidValue;
+      p.reduce = 3;
+      p.rn = *rn;
     }
   }
   const CUtensorMap* tw2 = &tmap_w;

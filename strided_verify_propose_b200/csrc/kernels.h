@@ -85,6 +85,19 @@ int gemm_coresident_ctas(const GemmPlan& plan);
 
 struct QkvReduceArgs;
 
+// The residual add and the next RMSNorm, finished by a reduced split-K GEMM:
+// x[row] += Y[row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w), the row's sum
+// of squares gathered from per-tile shares after a barrier over the grid.
+struct ResNormArgs {
+  float* x;               // [m][n_out] fp32 residual stream (updated)
+  const float* norm_w;    // [n_out]
+  float eps;
+  __nv_bfloat16* hn;      // [m][n_out] bf16 normalised output
+  float* ss;              // [n_out / 128][ss_stride] per-tile sums of squares (scratch)
+  int32_t ss_stride;      // >= m
+  int32_t* grid_cnt;      // [2] zero before the first launch; each launch leaves them zero
+};
+
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out] (one slice when reduced); kEpiSiluMul:
 // out_act[m][n_out / 2] bf16 with W's rows interleaved in blocks of 16
@@ -94,7 +107,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
                         const GemmAugment* augment = nullptr, const GemmReduce* reduce = nullptr,
-                        const QkvReduceArgs* qkv = nullptr);
+                        const QkvReduceArgs* qkv = nullptr, const ResNormArgs* rn = nullptr);
 // (qkv with reduce: the reduced output is the fused QKV projection and the
 // kernel finishes it as launch_qkv_reduce would, writing no output slice;
 // qkv->part and qkv->splits are ignored.)

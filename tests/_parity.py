@@ -13,7 +13,8 @@ inverse-CDF draw, argmax) is classified before it is compared:
   correct decision for its own logits (validity), and the trajectories may
   part there;
 * accept tests within 1e-3 of the ratio p/q are always "near" (the
-  tolerance the method's accuracy statement sets).
+  tolerance the method's accuracy statement sets), except u = 0, which
+  accepts any draft of nonzero probability whatever the rounding.
 
 Logits are compared element-wise against LOGIT_TOL scaled by the logit
 spread (logit_tolerance below).
@@ -181,7 +182,11 @@ def compare_decision(dec, gpu_A, gpu_new, gpu_props, lo, lg, drafts, q_o, q_g, u
             r_g = p_g / qd_g if qd_g > 0 else np.inf
             ok_o, ok_g = u[j] < r_o, u[j] < r_g
             out.seen("accept")
-            if abs(u[j] - r_o) < ACCEPT_BAR or ok_o != ok_g or abs(u[j] - r_g) < FP32_REL * max(r_g, 1e-30):
+            # u = 0 accepts any draft of nonzero probability in any precision
+            # (u q < p is 0 < p): no rounding can move that decision
+            certain = u[j] == 0.0 and p_o > 0 and p_g > 0
+            if not certain and (abs(u[j] - r_o) < ACCEPT_BAR or ok_o != ok_g
+                                or abs(u[j] - r_g) < FP32_REL * max(r_g, 1e-30)):
                 out.near("accept", f"accept test {j}")
                 break
         if not ok_o:

@@ -102,9 +102,13 @@ def test_random_shapes(seed):
 
 
 def test_shapes_not_on_tensor_cores():
-    # head_dim 64 and more than 32 query rows per KV head go to the other kernel
+    # head_dim 64, 32-key pages and more than 64 query rows per KV head go to
+    # the other kernel; 33..64 rows (Qwen3-32B's 8 heads x 7 rows) stay
     assert B.attention_split(4, 7, 32, 8, 64, 10, 64, [100] * 4) is None
-    assert B.attention_split(4, 16, 32, 8, 128, 10, 64, [100] * 4) is None
+    assert B.attention_split(4, 7, 32, 8, 128, 10, 32, [100] * 4) is None
+    assert B.attention_split(4, 17, 32, 8, 128, 10, 64, [100] * 4) is None
+    assert B.attention_split(4, 7, 64, 8, 128, 10, 64, [100] * 4) is not None
+    assert B.attention_split(4, 16, 32, 8, 128, 10, 64, [100] * 4) is not None
 
 
 def test_bad_arguments():

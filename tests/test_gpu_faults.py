@@ -158,7 +158,9 @@ def test_bounded_wait_runs_out_and_the_context_stays_usable():
 
 
 def _state_buffers(kv, st):
-    return [kv.k_pool, kv.v_pool, kv.page_table, kv.free_head, st.seq_len, st.n_draft, st.pending]
+    # bf16 pools as their 16-bit patterns (numpy has no bfloat16)
+    return [kv.k_pool.view(torch.int16), kv.v_pool.view(torch.int16), kv.page_table, kv.free_head,
+            st.seq_len, st.n_draft, st.pending]
 
 
 @pytest.mark.parametrize("shape_name,Bn", [("TINY", 4), ("QWEN3_8B_2L", 8)])

@@ -200,7 +200,7 @@ def test_tiny_config_sample_mode():
 
 # Upper bounds on the near fraction per decision kind. Tiny decoder: logits
 # within 5e-3 of the oracle's, vocabulary 1024.
-TINY_NEAR = {"accept": 0.05, "argmax": 0.1, "draw": 0.25}
+TINY_NEAR = {"accept": 0.02, "argmax": 0.08, "draw": 0.12}
 
 
 @pytest.mark.parametrize("N,propose,verify", [
@@ -217,7 +217,7 @@ def test_tiny_batch(N, propose, verify):
 
 # Qwen3-8B widths: argmax decisions flip only where the oracle's top-2 logit
 # gap is below the kernels' logit error (a few hundredths).
-WIDE_NEAR = {"accept": 0.01, "argmax": 0.1}
+WIDE_NEAR = {"accept": 0.01, "argmax": 0.05}
 
 
 def test_qwen3_8b_widths_two_layers():
