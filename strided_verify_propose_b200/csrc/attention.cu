@@ -692,7 +692,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* red = reinterpret_cast<float*>(ps + kPBuf);      // [4 quadrants][NP]
   float* m_sh = red + 4 * NP;                             // running max per row (log2 units)
   float* alpha_sh = m_sh + NP;                            // [2][NP] per-tile rescale
-  float* l_sh = alpha_sh + 2 * NP;                        // row sums at item end
+  float* l_sh = alpha_sh + 2 * NP;                        // 1 / row sum at item end
   float* mu_sh = l_sh + NP;                               // exponent offset (m, 0 while m = -inf)
   int* pos_sh = reinterpret_cast<int*>(mu_sh + NP);       // row positions of the item
   int* minpos_sh = pos_sh + NP;                           // [kRowWarps]
@@ -1106,7 +1106,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (warp < kRowWarps) {
         const int q = my_row;
         const float L = (red[q] + red[NP + q]) + (red[2 * NP + q] + red[3 * NP + q]);
-        l_sh[q] = L;
+        l_sh[q] = L > 0.f ? 1.f / L : 0.f;   // one reciprocal per row
         if (sg.slot >= 0)
           p.part_ml[static_cast<int64_t>(sg.slot) * NP + q] = make_float2(m_sh[q], L);
         else if (q == 0)
@@ -1116,10 +1116,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (sg.slot >= 0) {
         float* po = p.part_o + (static_cast<int64_t>(sg.slot) * NP + r0) * 128 + kl;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const float L = l_sh[r0 + r];
-          po[r * 128] = L > 0.f ? o[r] / L : 0.f;
-        }
+        for (int r = 0; r < NR; ++r) po[r * 128] = o[r] * l_sh[r0 + r];
       }
       named_bar_sync(2, kSoftThreads);   // row state is rewritten by the next segment
       sg = nx;

@@ -152,17 +152,13 @@ struct isd_ctx {
   void* acc_ws = nullptr;
   size_t acc_ws_bytes = 0;
   int32_t* prefill_lens = nullptr;  // [max_batch]
+  int32_t* prefill_order = nullptr; // [max_batch] requests by descending prompt length
+  int32_t* prefill_ptab = nullptr;  // [max_batch][max pages] page table rows in that order
 
   std::map<std::tuple<const void*, int, int, int>, CUtensorMap> act_maps;
   std::map<std::tuple<int, int, int, int>, GemmPlan> plans;
   void* sk_ws = nullptr;            // stream-K partials + sync words (sync words zeroed)
   size_t sk_ws_bytes = 0;
-  int32_t* red_cnt = nullptr;       // arrival / departure counters of in-kernel split-K reduction
-  int32_t red_cnt_n = 0;
-  float* rn_ss = nullptr;           // [hidden / 128][rn_ss_stride] per-tile row sums of squares
-  int32_t rn_ss_stride = 0;         // rows (the step rows: batch x (2N - 1) at most)
-  int32_t* rn_cnt = nullptr;        // [2] grid barrier of the fused residual + RMSNorm
-  std::map<std::tuple<int, int, int, int>, int> coresident;   // per plan: CTAs resident at once
   int launches = 0;
 
   // gated LoRA (R-ISD): packed adapters per layer + their workspace
@@ -257,17 +253,10 @@ struct AugSpec {
   int k2;
 };
 
-// With reduce_out, a split-K plan whose whole grid fits on the device at
-// once reduces its splits inside the kernel: the partials go to the front of
-// out and the single output slice behind them; *reduce_out points at the
-// slices the next kernel reads (the reduced slice with *splits_used = 1, or
-// out itself with the plan's split count).
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
-         const AugSpec* aug = nullptr, float** reduce_out = nullptr,
-         const isd::QkvReduceArgs* qkv = nullptr, bool* qkv_fused = nullptr,
-         const isd::ResNormArgs* rn = nullptr) {
+         const AugSpec* aug = nullptr) {
   if (epi == isd::kEpiF32 && out_elems > 0) {
     // large prefill chunks: no more splits than the partial buffer holds
     const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
@@ -292,32 +281,11 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
     if (rc) return rc;
     ga = isd::GemmAugment{aug->tw2, tx2, aug->k2};
   }
-  isd::GemmReduce red{};
-  bool reduced = false;
-  float* result = out;
-  if (reduce_out && epi == isd::kEpiF32 && plan.splits > 1 && !plan.streamk) {
-    const size_t rf = isd::gemm_reduce_floats(plan, n);
-    if (rf + static_cast<size_t>(m) * n <= out_elems &&
-        isd::gemm_reduce_counters(plan, n) <= c->red_cnt_n) {
-      auto key = std::make_tuple(plan.pair, plan.n_mma, static_cast<int>(plan.smem_bytes), 0);
-      auto it = c->coresident.find(key);
-      if (it == c->coresident.end()) it = c->coresident.emplace(key, isd::gemm_coresident_ctas(plan)).first;
-      const int64_t ctas = static_cast<int64_t>(n / 128) * plan.n_chunks * plan.splits;
-      if (ctas <= it->second) {
-        red = isd::GemmReduce{out, rf, c->red_cnt, c->red_cnt_n, it->second};
-        reduced = true;
-        result = out + rf;
-      }
-    }
-  }
   cudaEvent_t e0 = prof_mark(c, st);
-  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, result, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, aug ? &ga : nullptr, reduced ? &red : nullptr,
-                            reduced ? qkv : nullptr, reduced ? rn : nullptr));
+  ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
+                            c->sk_ws_bytes, aug ? &ga : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
-  if (qkv_fused) *qkv_fused = reduced && (qkv != nullptr || rn != nullptr);
-  if (splits_used) *splits_used = reduced ? 1 : plan.splits;
-  if (reduce_out) *reduce_out = result;
+  if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
   return ISD_OK;
 }
@@ -440,9 +408,12 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_qkv, c->hn, M, H, 3 * r, status, st);
       if (rc) return rc;
     }
+    rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr);
+    if (rc) return rc;
     isd::QkvReduceArgs qa;
-    qa.part = nullptr;
-    qa.splits = 0;
+    qa.part = c->part;
+    qa.splits = s;
     qa.rows = M;
     qa.rows_per_req = rows_per_req;
     qa.n_q = g.n_q_heads;
@@ -463,24 +434,11 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
     qa.status = status;
-    // the QKV projection; when its split-K reduction runs in the kernel the
-    // kernel also finishes QK-norm, RoPE and the q / KV writes
-    float* slices = nullptr;
-    bool fused = false;
-    rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr,
-              &slices, &qa, &fused);
-    if (rc) return rc;
+    cudaEvent_t a0 = prof_mark(c, st);
+    ISD_CUDA(isd::launch_qkv_reduce(qa, st));
+    c->launches += 1;
     cudaEvent_t a1 = prof_mark(c, st);
-    if (!fused) {
-      qa.part = slices;
-      qa.splits = s;
-      cudaEvent_t a0 = a1;
-      ISD_CUDA(isd::launch_qkv_reduce(qa, st));
-      c->launches += 1;
-      a1 = prof_mark(c, st);
-      prof_add(c, kPQkvReduce, a0, a1);
-    }
+    prof_add(c, kPQkvReduce, a0, a1);
     cudaEvent_t amid = prof_event(c);
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid));
@@ -492,20 +450,13 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_o, c->attn, M, c->q_dim, r, status, st);
       if (rc) return rc;
     }
-    // the O projection; a reduced split-K GEMM also adds the residual and
-    // applies the MLP's RMSNorm
-    isd::ResNormArgs rn_o{c->x, c->mlp_norm[l], g.rms_eps, c->hn, c->rn_ss, c->rn_ss_stride,
-                          c->rn_cnt};
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
-              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr, &slices, nullptr,
-              &fused, M <= c->rn_ss_stride ? &rn_o : nullptr);
+              c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
     if (rc) return rc;
-    if (!fused) {
-      cudaEvent_t r0 = prof_mark(c, st);
-      ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
-      prof_add(c, kPResNorm, r0, prof_mark(c, st));
-      c->launches += 1;
-    }
+    cudaEvent_t r0 = prof_mark(c, st);
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
+    prof_add(c, kPResNorm, r0, prof_mark(c, st));
+    c->launches += 1;
     // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
     // K-blocks follow each tile's base K-blocks (stream-K cuts unchanged)
     AugSpec aug_gu{ll ? &ll->tb_gu : nullptr, c->lora_xa, 2 * r};
@@ -521,18 +472,14 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       rc = lora_xa(c, ll->ta_d, c->act, M, g.intermediate, r, status, st);
       if (rc) return rc;
     }
-    const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
-    isd::ResNormArgs rn_d{c->x, next_norm, g.rms_eps, c->hn, c->rn_ss, c->rn_ss_stride, c->rn_cnt};
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr, &slices,
-              nullptr, &fused, M <= c->rn_ss_stride ? &rn_d : nullptr);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr);
     if (rc) return rc;
-    if (!fused) {
-      cudaEvent_t r1 = prof_mark(c, st);
-      ISD_CUDA(isd::launch_residual_norm(slices, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
-      prof_add(c, kPResNorm, r1, prof_mark(c, st));
-      c->launches += 1;
-    }
+    const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
+    cudaEvent_t r1 = prof_mark(c, st);
+    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
+    prof_add(c, kPResNorm, r1, prof_mark(c, st));
+    c->launches += 1;
   }
   return ISD_OK;
 }
@@ -590,9 +537,8 @@ int alloc_workspace(isd_ctx* c) {
       static_cast<size_t>(g.max_batch) * 4,
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
-      static_cast<size_t>(2 * (wide / 128) * 8) * 4,      // split-K reduction counters
-      static_cast<size_t>(g.hidden / 128) * step_rows * 4,  // residual + norm: tile sums
-      256,                                                  // residual + norm: grid barrier
+      static_cast<size_t>(g.max_batch) * 4,                                    // prefill order
+      static_cast<size_t>(g.max_batch) * max_pages * 4,                        // prefill page rows
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -622,15 +568,10 @@ int alloc_workspace(isd_ctx* c) {
   c->prefill_lens = reinterpret_cast<int32_t*>(b + off[i++]);
   c->sk_ws = b + off[i++];
   c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
-  c->red_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
-  c->red_cnt_n = static_cast<int32_t>(2 * (wide / 128) * 8);
-  c->rn_ss = reinterpret_cast<float*>(b + off[i++]);
-  c->rn_ss_stride = static_cast<int32_t>(step_rows);
-  c->rn_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
-  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
-      cudaMemset(c->red_cnt, 0, static_cast<size_t>(c->red_cnt_n) * 4) != cudaSuccess ||
-      cudaMemset(c->rn_cnt, 0, 256) != cudaSuccess)
-    return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
+  c->prefill_order = reinterpret_cast<int32_t*>(b + off[i++]);
+  c->prefill_ptab = reinterpret_cast<int32_t*>(b + off[i++]);
+  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
+    return fail(ISD_E_CUDA, "stream-K workspace clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;
   std::vector<float2> tab(static_cast<size_t>(g.max_position) * half);
@@ -962,22 +903,34 @@ int isd_prefill(isd_ctx* ctx, const isd_kv* kv, const int32_t* tokens_dev, int32
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ctx->launches = 0;
+  // requests by descending prompt length: the requests a pass still has rows
+  // for are then a prefix of this order, and a pass runs only those
+  std::vector<int32_t> order(batch);
+  for (int b = 0; b < batch; ++b) order[b] = b;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int b) { return lens_host[a] > lens_host[b]; });
   ISD_CUDA(cudaMemcpyAsync(ctx->prefill_lens, lens_host, sizeof(int32_t) * batch,
                            cudaMemcpyHostToDevice, st));
-  if (sub > 1) {
-    // the page table with every request's row repeated once per sub-request
-    const size_t row_bytes = static_cast<size_t>(kv->max_pages_per_req) * sizeof(int32_t);
-    for (int j = 0; j < sub; ++j)
-      ISD_CUDA(cudaMemcpy2DAsync(ctx->prefill_table + static_cast<size_t>(j) * kv->max_pages_per_req,
-                                 row_bytes * sub, kv->page_table_dev, row_bytes, row_bytes, batch,
-                                 cudaMemcpyDeviceToDevice, st));
-  }
+  ISD_CUDA(cudaMemcpyAsync(ctx->prefill_order, order.data(), sizeof(int32_t) * batch,
+                           cudaMemcpyHostToDevice, st));
+  // the page table in that order, and again with every row repeated once per
+  // attention sub-request
+  ISD_CUDA(isd::launch_gather_rows(kv->page_table_dev, ctx->prefill_order, batch,
+                                   kv->max_pages_per_req, 1, ctx->prefill_ptab, st));
+  ISD_CUDA(isd::launch_gather_rows(kv->page_table_dev, ctx->prefill_order, batch,
+                                   kv->max_pages_per_req, sub, ctx->prefill_table, st));
+  ctx->launches += 2;
+  isd_kv kv_sorted = *kv;
+  kv_sorted.page_table_dev = ctx->prefill_ptab;
   isd::RowMeta meta{ctx->meta_tok, ctx->meta_pos, ctx->meta_flags};
+  int active = batch;
   for (int start = 0; start < longest - 1; start += chunk) {
-    ISD_CUDA(isd::launch_assemble_prefill(tokens_dev, max_len, ctx->prefill_lens, batch, chunk,
-                                          start, meta, st));
+    while (active > 0 && lens_host[order[active - 1]] - 1 <= start) --active;
+    ISD_CUDA(isd::launch_assemble_prefill(tokens_dev, max_len, ctx->prefill_lens, ctx->prefill_order,
+                                          active, chunk, start, meta, st));
     ctx->launches += 1;
-    rc = forward_layers(ctx, kv, batch, chunk, status_dev, st, false, sub, ctx->prefill_table);
+    rc = forward_layers(ctx, &kv_sorted, active, chunk, status_dev, st, false, sub,
+                        ctx->prefill_table);
     if (rc) return rc;
   }
   // starting state: L = len - 1, x* = last prompt token, no drafts

@@ -42,9 +42,6 @@ constexpr int kTileK = 64;                  // K elements per stage (128 bytes)
 constexpr int kStageA = kTileM * kTileK * 2;  // 16 KB
 constexpr size_t kMaxSmem = 231424;         // 226 KB dynamic (+ a few static bytes <= 227 KB)
 constexpr int kEpiWarps = 8;                // epilogue warps (two per TMEM quadrant)
-constexpr int kMaxChunksPerWarp = 8;        // 32-token chunks per epilogue warp (512 tokens / 32 / 2)
-constexpr int kRedRows = 2;                 // rows per warp per round of the in-kernel split-K sum
-constexpr int kRedSplits = 4;               // splits whose loads are unrolled (more take a loop)
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 struct GemmParams {
@@ -65,91 +62,7 @@ struct GemmParams {
   // continues over aug_kb K-blocks of a second operand pair (tmap_w2,
   // tmap_x2), accumulating into the same result
   int32_t aug_kb;
-  // split-K reduced in the kernel: every split parks its fp32 partial in
-  // red[(tile * n_chunks + chunk) * splits + split][tokens][128], then each
-  // split sums its share of the tile's token chunks over all splits in split
-  // order and writes one output slice; red_cnt[2 * (tile * n_chunks + chunk)]
-  // counts arrivals, [.. + 1] departures (the last departure zeroes both)
-  int32_t reduce;
-  float* red;
-  int32_t* red_cnt;
-  // reduce == 2: the reduced output is the fused QKV projection; instead of
-  // writing it, apply QK-norm and RoPE and write q and the K/V page slots
-  QkvReduceArgs qkv;
-  // reduce == 3: the reduced output is added to the residual stream and the
-  // next RMSNorm follows (after a barrier over the whole grid)
-  ResNormArgs rn;
 };
-
-// QK-norm + NeoX RoPE + q / KV-page writes for one token row of one
-// 128-feature tile of the fused QKV projection, reduced over the splits:
-// lane l holds features 4l..4l+3 of the tile (heads of a.head_dim features,
-// 128 / head_dim per tile). Per head: RMSNorm over head_dim for q and k,
-// rotate-half pairs (i, i + head_dim/2) at the row's absolute position, q to
-// the attention input, k and v into the row's page slot.
-__device__ __forceinline__ void qkv_row_epilogue(const QkvReduceArgs& a, float4 v, int row, int mt,
-                                                 int lane) {
-  const int HD = a.head_dim;
-  const int f = mt * kTileM + lane * 4;          // first feature of this lane
-  const int hd = f / HD, d = f % HD;             // head and its first dim
-  const int flags = a.meta.flags[row];
-  int pos = a.meta.pos[row];
-  const bool write_kv = (flags & kRowWriteKV) && pos >= 0;
-  if (pos >= a.max_position) {
-    if (lane == 0 && mt == 0) flag(a.status, ISD_DEV_BAD_STATE);
-    pos = a.max_position - 1;
-  }
-  const int rpos = pos < 0 ? 0 : pos;
-  float x[4] = {v.x, v.y, v.z, v.w};
-  if (hd < a.n_q + a.n_kv) {
-    // every lane of the warp holds the same head kind (a tile never mixes
-    // q / k with v: q and k widths are multiples of 128)
-    const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
-    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
-    // sum over the head's lanes: head_dim / 4 lanes (32 or 16)
-    for (int o = HD / 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rstd = rsqrtf(ss / HD + a.eps);
-    const float4 w4 = *reinterpret_cast<const float4*>(nw + d);
-    x[0] *= rstd * w4.x;
-    x[1] *= rstd * w4.y;
-    x[2] *= rstd * w4.z;
-    x[3] *= rstd * w4.w;
-    // the partner dims d +- head_dim/2 sit head_dim/8 lanes away
-    float y[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) y[j] = __shfl_xor_sync(0xffffffffu, x[j], HD / 8);
-    const bool lower = d < HD / 2;
-    const int i0 = lower ? d : d - HD / 2;
-    const float2* cs = a.rope + static_cast<int64_t>(rpos) * (HD / 2) + i0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 c = cs[j];
-      x[j] = lower ? x[j] * c.x - y[j] * c.y : x[j] * c.x + y[j] * c.y;
-    }
-  }
-  __align__(8) __nv_bfloat16 o4[4] = {__float2bfloat16_rn(x[0]), __float2bfloat16_rn(x[1]),
-                                       __float2bfloat16_rn(x[2]), __float2bfloat16_rn(x[3])};
-  if (hd < a.n_q) {
-    __nv_bfloat16* qo = a.q_out + (static_cast<int64_t>(row) * a.n_q + hd) * HD + d;
-    *reinterpret_cast<uint2*>(qo) = *reinterpret_cast<const uint2*>(o4);
-  } else if (write_kv) {
-    const int b = row / a.rows_per_req;
-    const int pidx = pos / a.page_size;
-    const int page = pidx < a.max_pages_per_req
-                         ? a.page_table[static_cast<int64_t>(b) * a.max_pages_per_req + pidx]
-                         : -1;
-    if (page < 0 || page >= a.num_pages) {
-      if ((lane & (HD / 4 - 1)) == 0) flag(a.status, ISD_DEV_BAD_PAGE);
-      return;
-    }
-    const int64_t slot_base = (static_cast<int64_t>(a.layer) * a.num_pages + page) * a.n_kv;
-    const bool is_k = hd < a.n_q + a.n_kv;
-    const int g = is_k ? hd - a.n_q : hd - a.n_q - a.n_kv;
-    __nv_bfloat16* dst = (is_k ? a.k_pool : a.v_pool) +
-                         (((slot_base + g) * a.page_size) + pos % a.page_size) * HD + d;
-    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(o4);
-  }
-}
 
 // One contiguous run of K-blocks of one tile, processed by one CTA (pair).
 struct Segment {
@@ -407,16 +320,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
       // cut tile: 1 = first part to finish (park the partial), 2 = second
       // (add the parked partial, then the normal epilogue), 3 = second after
-      // a timeout (status flagged, nothing written); 4 = a split of an
-      // in-kernel reduced split-K tile (park the partial, then reduce)
+      // a timeout (status flagged, nothing written)
       int mode = 0;
       float* part = nullptr;
       int32_t* sync = nullptr;
-      const int red_tile = mt * static_cast<int>(gridDim.y) + static_cast<int>(blockIdx.y);
-      if (p.reduce) {
-        mode = 4;
-        part = p.red + (static_cast<int64_t>(red_tile) * gridDim.z + split) * nchunk * 32 * kTileM;
-      } else if (!sg.whole) {
+      if (!sg.whole) {
         const int slot = sg.slot * (kPair ? 2 : 1) + static_cast<int>(rank);
         part = p.sk_part + static_cast<int64_t>(slot) * nchunk * 32 * kTileM;
         sync = p.sk_sync + 2 * slot;
@@ -442,79 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // TMEM loads run one chunk ahead of the chunk being written out
       uint32_t r[32];
       if (half < nchunk) tmem_ld_32x32_async(lane_addr + half * 32, r);
-      // SwiGLU tiles: the bf16 results stay in registers until every chunk is
-      // read, then the accumulator is released and the stores follow, so the
-      // next tile's MMAs run while this tile's results leave
-      const bool staged = p.epi == kEpiSiluMul && (mode == 0 || mode == 2);
-      bool released = false;
-      if (staged) {
-        const bool hi = lane >= 16;
-        uint32_t ov[kMaxChunksPerWarp * 8];   // [chunk][8]: token pairs (2k, 2k + 1) of 16 results
-#pragma unroll
-        for (int ci = 0; ci < kMaxChunksPerWarp; ++ci) {
-          const int c = half + 2 * ci;
-          if (c < nchunk) {
-            float v[32];
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            if (c + 2 < nchunk) tmem_ld_32x32_async(lane_addr + (c + 2) * 32, r);
-            if (mode == 2) {
-              const float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] += __ldcg(pp + j * kTileM);
-            }
-            // gate and up rows of a feature sit 16 lanes apart: low lanes
-            // finish even tokens, high lanes odd ones
-#pragma unroll
-            for (int k = 0; k < 16; k += 2) {
-              float o2[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int j = 2 * (k + e);
-                const float x_j = __shfl_xor_sync(0xffffffffu, v[j], 16);
-                const float x_j1 = __shfl_xor_sync(0xffffffffu, v[j + 1], 16);
-                const float g = hi ? x_j1 : v[j];
-                const float u = hi ? v[j + 1] : x_j;
-                o2[e] = silu_mul(g, u);
-              }
-              __nv_bfloat162 pk = __floats2bfloat162_rn(o2[0], o2[1]);
-              ov[ci * 8 + k / 2] = *reinterpret_cast<uint32_t*>(&pk);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (kPair)
-            mbar_arrive_cluster(empty_addr);
-          else
-            mbar_arrive(tmem_empty);
-        }
-        released = true;
-        const int half_n = p.n_out / 2;
-        const int f = mt * 64 + quad * 16 + (lane & 15);
-#pragma unroll
-        for (int ci = 0; ci < kMaxChunksPerWarp; ++ci) {
-          const int c = half + 2 * ci;
-          if (c < nchunk) {
-            const int t0 = tok0 + c * 32;
-            const bool full_chunk = c * 32 + 32 <= p.n_pad && t0 + 32 <= p.m;
-            __nv_bfloat16* rowp =
-                p.out_act + static_cast<int64_t>(t0 + (hi ? 1 : 0)) * half_n + f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const int jj = 2 * k + (hi ? 1 : 0);
-              const uint32_t w = ov[ci * 8 + k / 2];
-              const uint16_t bits = (k & 1) ? static_cast<uint16_t>(w >> 16) : static_cast<uint16_t>(w);
-              if (full_chunk || (c * 32 + jj < p.n_pad && t0 + jj < p.m))
-                *reinterpret_cast<uint16_t*>(rowp) = bits;
-              rowp += 2 * half_n;
-            }
-          }
-        }
-      }
-      for (int c = half; !staged && c < nchunk; c += 2) {
+      for (int c = half; c < nchunk; c += 2) {
         float v[32];
         tmem_ld_wait();
 #pragma unroll
@@ -522,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c + 2 < nchunk) tmem_ld_32x32_async(lane_addr + (c + 2) * 32, r);
         const int t0 = tok0 + c * 32;
         // partial slot: rows of 128 fp32, tokens 0 .. 32 * nchunk - 1
-        if (mode == 1 || mode == 4) {
+        if (mode == 1) {
           float* pp = part + static_cast<int64_t>(c * 32) * kTileM + quad * 32 + lane;
 #pragma unroll
           for (int j = 0; j < 32; ++j) pp[j * kTileM] = v[j];
@@ -577,183 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // accumulators read: release them to the MMA issuer (of the pair)
-      if (!released) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (kPair)
-            mbar_arrive_cluster(empty_addr);
-          else
-            mbar_arrive(tmem_empty);
-        }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (kPair)
+          mbar_arrive_cluster(empty_addr);
+        else
+          mbar_arrive(tmem_empty);
       }
       if (mode == 1) {
         // partial parked: publish it
         __threadfence();
         named_bar_sync(1, 32 * kEpiWarps);
         if (ew == 0 && lane == 0) st_release_gpu(&sync[1], 1);
-      } else if (mode == 4) {
-        // every split of the tile parks its partial; then this split sums
-        // its share of the token chunks over the splits, in split order
-        __threadfence();
-        named_bar_sync(1, 32 * kEpiWarps);
-        const int S = static_cast<int>(gridDim.z);
-        int32_t* cnt = p.red_cnt + 2 * red_tile;
-        if (ew == 0 && lane == 0) {
-          atomicAdd(&cnt[0], 1);
-          int ok_ = 1;
-          const long long t0 = clock64();
-          const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
-          while (ld_acquire_gpu(&cnt[0]) < S) {
-            if (clock64() - t0 > limit) {
-              flag(p.status, ISD_DEV_TIMEOUT);
-              ok_ = 0;
-              break;
-            }
-          }
-          epi_mode = ok_;
-        }
-        named_bar_sync(1, 32 * kEpiWarps);
-        if (epi_mode) {
-          const int c_lo = split * nchunk / S, c_hi = (split + 1) * nchunk / S;
-          const int t_lo = c_lo * 32, t_hi = min(c_hi * 32, p.n_pad);
-          const int64_t sstride = static_cast<int64_t>(nchunk) * 32 * kTileM;
-          const float* base = p.red + static_cast<int64_t>(red_tile) * S * sstride;
-          // warp ew takes token rows t_lo + ew, + 8, ...; lane l features
-          // 4l..4l+3. Rows go kRedRows at a time with every split's load of
-          // them (and the residual's) in flight together; the sum still runs
-          // in split order.
-          const int t_end = min(t_hi, p.m - tok0);
-          for (int t = t_lo + ew; t < t_end; t += kEpiWarps * kRedRows) {
-            float4 part4[kRedSplits][kRedRows];
-            float4 xo[kRedRows];
-#pragma unroll
-            for (int rr = 0; rr < kRedRows; ++rr) {
-              const int tr = t + rr * kEpiWarps;
-              const float* q = base + static_cast<int64_t>(tr) * kTileM + lane * 4;
-#pragma unroll
-              for (int s2 = 0; s2 < kRedSplits; ++s2)
-                part4[s2][rr] = (tr < t_end && s2 < S)
-                                    ? __ldcg(reinterpret_cast<const float4*>(q + s2 * sstride))
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-              xo[rr] = (p.reduce == 3 && tr < t_end)
-                           ? *reinterpret_cast<const float4*>(
-                                 p.rn.x + static_cast<int64_t>(tok0 + tr) * p.n_out + mt * kTileM + lane * 4)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int rr = 0; rr < kRedRows; ++rr) {
-              const int tr = t + rr * kEpiWarps;
-              if (tr >= t_end) continue;   // uniform across the warp
-              float4 acc = part4[0][rr];
-#pragma unroll
-              for (int s2 = 1; s2 < kRedSplits; ++s2) {
-                if (s2 < S) {
-                  acc.x += part4[s2][rr].x;
-                  acc.y += part4[s2][rr].y;
-                  acc.z += part4[s2][rr].z;
-                  acc.w += part4[s2][rr].w;
-                }
-              }
-              // more splits than the unrolled loads cover
-              for (int s2 = kRedSplits; s2 < S; ++s2) {
-                const float4 d = __ldcg(reinterpret_cast<const float4*>(
-                    base + s2 * sstride + static_cast<int64_t>(tr) * kTileM + lane * 4));
-                acc.x += d.x;
-                acc.y += d.y;
-                acc.z += d.z;
-                acc.w += d.w;
-              }
-              if (p.reduce == 2) {
-                qkv_row_epilogue(p.qkv, acc, tok0 + tr, mt, lane);
-              } else if (p.reduce == 3) {
-                // x += the projection; this tile's share of the row's sum of squares
-                float4 x4 = xo[rr];
-                x4.x += acc.x;
-                x4.y += acc.y;
-                x4.z += acc.z;
-                x4.w += acc.w;
-                *reinterpret_cast<float4*>(p.rn.x + static_cast<int64_t>(tok0 + tr) * p.n_out +
-                                           mt * kTileM + lane * 4) = x4;
-                const float ss = warp_sum(x4.x * x4.x + x4.y * x4.y + x4.z * x4.z + x4.w * x4.w);
-                if (lane == 0) p.rn.ss[static_cast<int64_t>(mt) * p.rn.ss_stride + tok0 + tr] = ss;
-              } else {
-                *reinterpret_cast<float4*>(p.out + static_cast<int64_t>(tok0 + tr) * p.n_out +
-                                           mt * kTileM + lane * 4) = acc;
-              }
-            }
-          }
-        }
-        if (p.reduce == 3) {
-          // every row's residual and tile sums are written once every CTA of
-          // the grid has passed here; then this split normalises its rows
-          const int total = static_cast<int>(gridDim.x * gridDim.y * gridDim.z);
-          __threadfence();
-          named_bar_sync(1, 32 * kEpiWarps);
-          if (ew == 0 && lane == 0) {
-            atomicAdd(&p.rn.grid_cnt[0], 1);
-            int ok_ = epi_mode;
-            const long long t0 = clock64();
-            const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
-            while (ld_acquire_gpu(&p.rn.grid_cnt[0]) < total) {
-              if (clock64() - t0 > limit) {
-                flag(p.status, ISD_DEV_TIMEOUT);
-                ok_ = 0;
-                break;
-              }
-            }
-            epi_mode = ok_;
-          }
-          named_bar_sync(1, 32 * kEpiWarps);
-          if (epi_mode) {
-            const int c_lo = split * nchunk / S, c_hi = (split + 1) * nchunk / S;
-            const int t_lo = c_lo * 32, t_end = min(min(c_hi * 32, p.n_pad), p.m - tok0);
-            const int tiles = p.n_out / kTileM;
-            const float4 w4 = *reinterpret_cast<const float4*>(p.rn.norm_w + mt * kTileM + lane * 4);
-            // kRedRows rows per round, their loads in flight together; the
-            // tile sums of a row are added lane by lane in tile order, then
-            // across lanes by the fixed butterfly
-            for (int t = t_lo + ew; t < t_end; t += kEpiWarps * kRedRows) {
-              float tot[kRedRows];
-              float4 xo[kRedRows];
-#pragma unroll
-              for (int rr = 0; rr < kRedRows; ++rr) {
-                const int tr = t + rr * kEpiWarps;
-                tot[rr] = 0.f;
-                xo[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (tr < t_end) {
-                  const int row = tok0 + tr;
-                  for (int i = lane; i < tiles; i += 32)
-                    tot[rr] += __ldcg(p.rn.ss + static_cast<int64_t>(i) * p.rn.ss_stride + row);
-                  xo[rr] = *reinterpret_cast<const float4*>(
-                      p.rn.x + static_cast<int64_t>(row) * p.n_out + mt * kTileM + lane * 4);
-                }
-              }
-#pragma unroll
-              for (int rr = 0; rr < kRedRows; ++rr) {
-                const int tr = t + rr * kEpiWarps;
-                if (tr >= t_end) continue;   // uniform across the warp
-                const int row = tok0 + tr;
-                const float rstd = rsqrtf(warp_sum(tot[rr]) / p.n_out + p.rn.eps);
-                __align__(8) __nv_bfloat16 o4[4] = {
-                    __float2bfloat16_rn(xo[rr].x * rstd * w4.x), __float2bfloat16_rn(xo[rr].y * rstd * w4.y),
-                    __float2bfloat16_rn(xo[rr].z * rstd * w4.z), __float2bfloat16_rn(xo[rr].w * rstd * w4.w)};
-                *reinterpret_cast<uint2*>(p.rn.hn + static_cast<int64_t>(row) * p.n_out + mt * kTileM +
-                                          lane * 4) = *reinterpret_cast<const uint2*>(o4);
-              }
-            }
-          }
-          named_bar_sync(1, 32 * kEpiWarps);
-          if (ew == 0 && lane == 0 && atomicAdd(&p.rn.grid_cnt[1], 1) == total - 1) {
-            p.rn.grid_cnt[0] = 0;
-            p.rn.grid_cnt[1] = 0;
-          }
-        }
-        named_bar_sync(1, 32 * kEpiWarps);
-        if (ew == 0 && lane == 0 && atomicAdd(&cnt[1], 1) == S - 1) {
-          cnt[0] = 0;
-          cnt[1] = 0;
-        }
       } else if (mode >= 2) {
         // every read of the parked partial is done: reset the slot
         named_bar_sync(1, 32 * kEpiWarps);
@@ -878,54 +550,11 @@ size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }
 
 cudaError_t set_wait_limit_gemm(long long cycles) { return set_wait_limit_here(cycles); }
 
-size_t gemm_reduce_floats(const GemmPlan& plan, int32_t n_out) {
-  if (plan.splits < 2 || plan.streamk) return 0;
-  const size_t rows = (static_cast<size_t>(plan.n_pad) + 31) / 32 * 32;
-  return static_cast<size_t>(n_out) * plan.n_chunks * plan.splits * rows;
-}
-
-int gemm_reduce_counters(const GemmPlan& plan, int32_t n_out) {
-  return 2 * (n_out / kTileM) * plan.n_chunks;
-}
-
-int gemm_coresident_ctas(const GemmPlan& plan) {
-  auto kernel = plan.pair
-                    ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
-                    : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kMaxSmem)) != cudaSuccess)
-    return 0;
-  if (!plan.pair) {
-    int per_sm = 0, dev = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads,
-                                                      plan.smem_bytes) != cudaSuccess ||
-        cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return 0;
-    return per_sm * sms;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = plan.smem_bytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) return 0;
-  return 2 * clusters;
-}
-
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace, size_t sk_workspace_bytes,
-                        const GemmAugment* augment, const GemmReduce* reduce,
-                        const QkvReduceArgs* qkv, const ResNormArgs* rn) {
+                        const GemmAugment* augment) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -963,37 +592,6 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.sk_part = nullptr;
   p.sk_sync = nullptr;
   p.aug_kb = 0;
-  p.reduce = 0;
-  p.red = nullptr;
-  p.red_cnt = nullptr;
-  if (reduce != nullptr) {
-    // every CTA of the grid must be resident at once (the splits of a tile
-    // wait for each other), one slice of fp32 output, partials and counters
-    // in the caller's buffers
-    const int64_t ctas = static_cast<int64_t>(n_out / kTileM) * plan.n_chunks * plan.splits;
-    if (epi != kEpiF32 || plan.streamk || plan.splits < 2 || reduce->red == nullptr ||
-        reduce->counters == nullptr || reduce->red_floats < gemm_reduce_floats(plan, n_out) ||
-        reduce->n_counters < gemm_reduce_counters(plan, n_out) || ctas > reduce->coresident)
-      return cudaErrorInvalidValue;
-    p.reduce = 1;
-    p.red = reduce->red;
-    p.red_cnt = reduce->counters;
-    if (qkv != nullptr) {
-      // q / k widths are whole tiles, so a tile never mixes v with q or k
-      const int hd = qkv->head_dim;
-      if ((hd != 64 && hd != 128) || (qkv->n_q * hd) % kTileM || (qkv->n_kv * hd) % kTileM ||
-          (qkv->n_q + 2 * qkv->n_kv) * hd != n_out || qkv->rows_per_req < 1)
-        return cudaErrorInvalidValue;
-      p.reduce = 2;
-      p.qkv = *qkv;
-    } else if (rn != nullptr) {
-      if (rn->x == nullptr || rn->norm_w == nullptr || rn->hn == nullptr || rn->ss == nullptr ||
-          rn->grid_cnt == nullptr || rn->ss_stride < m)
-        return cudaErrorInvalidValue;
-      p.reduce = 3;
-      p.rn = *rn;
-    }
-  }
   const CUtensorMap* tw2 = &tmap_w;
   const CUtensorMap* tx2 = &tmap_x;
   if (augment != nullptr && augment->k > 0) {

@@ -64,53 +64,14 @@ struct GemmAugment {
   int32_t k;
 };
 
-// Split-K reduced inside the kernel (a plan with splits > 1 and no
-// stream-K): the splits park fp32 partials in red (gemm_reduce_floats), wait
-// for each other on counters (gemm_reduce_counters ints, zero before the
-// first launch; each launch leaves them zero) and write one output slice.
-// The splits wait for each other, so the whole grid must be resident at
-// once: coresident is gemm_coresident_ctas(plan), and the launch is refused
-// when the grid has more CTAs.
-struct GemmReduce {
-  float* red;
-  size_t red_floats;
-  int32_t* counters;
-  int32_t n_counters;
-  int32_t coresident;
-};
-size_t gemm_reduce_floats(const GemmPlan& plan, int32_t n_out);
-int gemm_reduce_counters(const GemmPlan& plan, int32_t n_out);
-// CTAs of this plan's kernel that can be resident on the device at once.
-int gemm_coresident_ctas(const GemmPlan& plan);
-
-struct QkvReduceArgs;
-
-// The residual add and the next RMSNorm, finished by a reduced split-K GEMM:
-// x[row] += Y[row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w), the row's sum
-// of squares gathered from per-tile shares after a barrier over the grid.
-struct ResNormArgs {
-  float* x;               // [m][n_out] fp32 residual stream (updated)
-  const float* norm_w;    // [n_out]
-  float eps;
-  __nv_bfloat16* hn;      // [m][n_out] bf16 normalised output
-  float* ss;              // [n_out / 128][ss_stride] per-tile sums of squares (scratch)
-  int32_t ss_stride;      // >= m
-  int32_t* grid_cnt;      // [2] zero before the first launch; each launch leaves them zero
-};
-
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
-// kEpiF32: out_f32[split][m][n_out] (one slice when reduced); kEpiSiluMul:
-// out_act[m][n_out / 2] bf16 with W's rows interleaved in blocks of 16
-// (gate rows then up rows).
+// kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
+// with W's rows interleaved in blocks of 16 (gate rows then up rows).
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmAugment* augment = nullptr, const GemmReduce* reduce = nullptr,
-                        const QkvReduceArgs* qkv = nullptr, const ResNormArgs* rn = nullptr);
-// (qkv with reduce: the reduced output is the fused QKV projection and the
-// kernel finishes it as launch_qkv_reduce would, writing no output slice;
-// qkv->part and qkv->splits are ignored.)
+                        const GemmAugment* augment = nullptr);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {
@@ -146,9 +107,14 @@ cudaError_t launch_assemble_step(const int32_t* pending, const int32_t* n_draft,
                                  const int32_t* seq_len, int32_t batch, int32_t stride_n,
                                  int32_t mask_token, RowMeta meta, int32_t* status,
                                  cudaStream_t stream);
+// rows of `batch` requests, request order[i] (or i when order is null) in
+// block i of `chunk` rows
 cudaError_t launch_assemble_prefill(const int32_t* tokens, int32_t max_len, const int32_t* lens,
-                                    int32_t batch, int32_t chunk, int32_t start, RowMeta meta,
-                                    cudaStream_t stream);
+                                    const int32_t* order, int32_t batch, int32_t chunk,
+                                    int32_t start, RowMeta meta, cudaStream_t stream);
+// dst row (i * repeat + j) = src row order[i] for i < rows, j < repeat (int rows of row_len).
+cudaError_t launch_gather_rows(const int32_t* src, const int32_t* order, int32_t rows,
+                               int32_t row_len, int32_t repeat, int32_t* dst, cudaStream_t stream);
 cudaError_t launch_embed_norm(const __nv_bfloat16* embed, const float* norm_w, RowMeta meta,
                               int32_t rows, int32_t hidden, int32_t vocab, float eps, float* x,
                               __nv_bfloat16* hn, int32_t* status, cudaStream_t stream);

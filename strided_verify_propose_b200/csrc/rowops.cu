@@ -55,13 +55,16 @@ __global__ void assemble_step_kernel(const int32_t* pending, const int32_t* n_dr
   meta.flags[row] = (L < 0 ? 0 : kRowWriteKV) | (r > n ? kRowMask : 0);
 }
 
-// Prefill chunk: rows [start, start+chunk) of every prompt; positions past
-// len-2 are padding rows that see the prompt's keys but write nothing.
+// Prefill chunk: rows [start, start+chunk) of the prompt of request
+// order[i] (i = block); positions past len-2 are padding rows that see the
+// prompt's keys but write nothing.
 __global__ void assemble_prefill_kernel(const int32_t* tokens, int32_t max_len, const int32_t* lens,
-                                        int32_t chunk, int32_t start, RowMeta meta) {
-  const int b = blockIdx.x, r = threadIdx.x;
+                                        const int32_t* order, int32_t chunk, int32_t start,
+                                        RowMeta meta) {
+  const int i = blockIdx.x, r = threadIdx.x;
   if (r >= chunk) return;
-  const int row = b * chunk + r;
+  const int b = order ? order[i] : i;
+  const int row = i * chunk + r;
   const int len = lens[b];
   const int q = start + r;
   if (q < len - 1) {
@@ -270,9 +273,29 @@ cudaError_t launch_assemble_step(const int32_t* pending, const int32_t* n_draft,
 }
 
 cudaError_t launch_assemble_prefill(const int32_t* tokens, int32_t max_len, const int32_t* lens,
-                                    int32_t batch, int32_t chunk, int32_t start, RowMeta meta,
-                                    cudaStream_t stream) {
-  assemble_prefill_kernel<<<batch, 64, 0, stream>>>(tokens, max_len, lens, chunk, start, meta);
+                                    const int32_t* order, int32_t batch, int32_t chunk,
+                                    int32_t start, RowMeta meta, cudaStream_t stream) {
+  if (batch < 1) return cudaSuccess;
+  assemble_prefill_kernel<<<batch, 64, 0, stream>>>(tokens, max_len, lens, order, chunk, start,
+                                                    meta);
+  return cudaGetLastError();
+}
+
+// dst row (i * repeat + j) = src row order[i], rows of row_len ints.
+__global__ void gather_rows_kernel(const int32_t* src, const int32_t* order, int32_t row_len,
+                                   int32_t repeat, int32_t* dst) {
+  const int i = blockIdx.x;
+  const int32_t* s = src + static_cast<int64_t>(order[i]) * row_len;
+  for (int j = 0; j < repeat; ++j) {
+    int32_t* d = dst + (static_cast<int64_t>(i) * repeat + j) * row_len;
+    for (int k = threadIdx.x; k < row_len; k += blockDim.x) d[k] = s[k];
+  }
+}
+
+cudaError_t launch_gather_rows(const int32_t* src, const int32_t* order, int32_t rows,
+                               int32_t row_len, int32_t repeat, int32_t* dst, cudaStream_t stream) {
+  if (rows < 1) return cudaSuccess;
+  gather_rows_kernel<<<rows, 128, 0, stream>>>(src, order, row_len, repeat, dst);
   return cudaGetLastError();
 }
 
