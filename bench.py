@@ -301,12 +301,18 @@ def run_cuda(args, ws, rank, local):
         eager_ms = h_start.elapsed_time(h_stop)
         eager_committed = int((eager_hist.long() + 1).sum().item())
 
-    # ---- profiled region: same steps with per-kernel-class CUDA events
+    lens_after_timed = st.seq_len.cpu().numpy().copy()   # (after the eager steps too)
+
+    # ---- profiled region: same steps with per-kernel-class CUDA events; the
+    # lengths each profiled step starts from price its attention bytes
+    lens_prof = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
     model.profile(True)
     for i in range(args.steps):
+        lens_prof[i].copy_(st.seq_len)
         one(unif_d[step_i]); step_i += 1
     prof = model.profile_read()
     model.profile(False)
+    lens_prof = lens_prof.cpu().numpy()
 
     # ---- the same steps without the adapter: R-ISD overhead alpha
     base_ms = None
@@ -369,13 +375,17 @@ def run_cuda(args, ws, rank, local):
     if rank == 0:
         peaks = load_peaks()
         ms_step = ms / args.steps
-        wbytes, kvbytes, lbytes, flops = step_bytes_flops(shape, lens_before, B, N)
+        # the timed steps start from lens_before and grow by about a step's
+        # commit each: price them at the mean length of the timed region
+        lens_timed = lens_before + (lens_after_timed - lens_before) * (
+            0.5 * args.steps / (2 * args.steps if eager_ms is not None else args.steps))
+        wbytes, kvbytes, lbytes, flops = step_bytes_flops(shape, lens_timed, B, N)
         step_bytes = wbytes + kvbytes
         hbm_frac_step = (step_bytes / (ms_step * 1e-3)) / (peaks["hbm"] * 1e9)
         # ceiling: GEMMs at the tensor peak plus attention KV at HBM peak
         t_floor = flops / (peaks["bf16"] * 1e12) + kvbytes / (peaks["hbm"] * 1e9)
         ceiling = (step_bytes / (peaks["hbm"] * 1e9)) / t_floor
-        roof = roofline_entry(prof, shape, B, N, lens_before, args.steps, peaks)
+        roof = roofline_entry(prof, shape, B, N, lens_prof, args.steps, peaks)
         result = {
             "metric": "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
             if args.workload == "qwen3_8b_b64" else f"committed tokens/s ({args.workload})",
@@ -421,9 +431,10 @@ def run_cuda(args, ws, rank, local):
         }
         if extras is not None:
             ex = dict(extras)
-            b1 = ex["qwen3_8b_b1"]
-            b1["hbm_roofline_fraction"] = b1["step_bytes"] / (b1["ms_per_step"] * 1e-3) / (
-                peaks["hbm"] * 1e9)
+            for key in ("qwen3_8b_b1", "qwen3_8b_b64_sample"):
+                e = ex[key]
+                e["hbm_roofline_fraction"] = e["step_bytes"] / (e["ms_per_step"] * 1e-3) / (
+                    peaks["hbm"] * 1e9)
             result["other_configs"] = ex
             result["risd_overhead_alpha"] = ex["risd_8b_b32"]["alpha"]
     del model
@@ -434,12 +445,13 @@ def run_cuda(args, ws, rank, local):
 
 
 def extra_configs(model, shape, args, seed):
-    """The model's two other single-GPU configurations, on the same weights:
-    batch 1 with a 2048-token prompt, and R-ISD (a rank-128 gated LoRA,
-    A, B ~ N(0, 0.01), on the MASK rows) at batch 32 with 2048-token
-    prompts, timed against the same steps without the adapter. Each runs
-    args.warmup eager steps, then args.steps steps between CUDA events
-    (acceptance-controlled uniforms, inputs resident)."""
+    """The model's other single-GPU configurations, on the same weights:
+    batch 1 with a 2048-token prompt; the headline batch (64, prompts
+    U[512, 4096]) with sampled proposals and full q rows; and R-ISD (a
+    rank-128 gated LoRA, A, B ~ N(0, 0.01), on the MASK rows) at batch 32
+    with 2048-token prompts, timed against the same steps without the
+    adapter. Each runs args.warmup eager steps, then args.steps steps
+    between CUDA events (acceptance-controlled uniforms, inputs resident)."""
     import torch
     from strided_verify_propose_b200 import binding as Bd
     N = 4
@@ -447,16 +459,16 @@ def extra_configs(model, shape, args, seed):
     stream = torch.cuda.current_stream()
     out = {}
 
-    def make(B, plen, s0):
-        lens = np.full(B, plen, np.int64)
+    def make(B, plen, s0, sample=False, lens=None):
+        lens = np.full(B, plen, np.int64) if lens is None else lens
         prompts = synth.prompts(shape, lens, s0)
         steps = args.warmup + 3 * args.steps + 2
-        maxp = -(-(plen + steps * N + R + 1) // P) + 1
-        need = [-(-(plen - 1 + R) // P)] * B
+        maxp = -(-(int(lens.max()) + steps * N + R + 1) // P) + 1
+        need = [-(-(int(L) - 1 + R) // P) for L in lens]
         num_pages = int(sum(need)) + B * (-(-steps * N // P) + 2)
         table, free = synth.page_layout(need, num_pages, maxp, s0)
         kv = Bd.KVCache(shape, num_pages, table, free)
-        st = Bd.StepState(B, N, V, sample=False)
+        st = Bd.StepState(B, N, V, sample=sample)
         Bd.prefill(model, kv, st, prompts)
         torch.cuda.synchronize()
         if int(st.status.item()) != 0:
@@ -490,6 +502,17 @@ def extra_configs(model, shape, args, seed):
     out["qwen3_8b_b1"] = {"ms_per_step": ms1 / args.steps, "value": com1 / (ms1 * 1e-3),
                           "unit": "tokens/s", "step_bytes": w + kvb, "steps": args.steps}
     del kv, st
+    # the headline batch with sampled proposals: every step writes the next
+    # drafts' full q rows and the accept tests read them
+    lens64 = synth.prompt_lengths(64, 512, 4096, seed)     # the headline workload's lengths
+    kv, st = make(64, 0, seed + 13, sample=True, lens=lens64)
+    ms_s, com_s, lens_s = timed(kv, st, 64, Bd.PROPOSE_SAMPLE, seed + 13, 2000)
+    w, kvb, _, _ = step_bytes_flops(shape, lens_s, 64, N)
+    qbytes = 2 * 64 * (N - 1) * V * 4        # q rows read and written per step
+    out["qwen3_8b_b64_sample"] = {"ms_per_step": ms_s / args.steps, "value": com_s / (ms_s * 1e-3),
+                                  "unit": "tokens/s", "step_bytes": w + kvb + qbytes,
+                                  "steps": args.steps, "q_rows": "fp32, [64][3][151936]"}
+    del kv, st
     # R-ISD at batch 32: the same steps with and without the adapter
     model.load_lora(Bd.random_device_lora(shape, 128, seed=seed, std=0.01), rank=128)
     kv, st = make(32, 2048, seed + 12)
@@ -511,8 +534,9 @@ def extra_configs(model, shape, args, seed):
 ATTN_DRAM_PER_KV_BYTE = 603.6 / 580.4
 
 
-def roofline_entry(prof, shape, B, N, lens, steps, peaks):
-    """Roofline of the kernel class with the largest device time."""
+def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
+    """Roofline of the kernel class with the largest device time (lens_steps:
+    the request lengths each profiled step started from, [steps][B])."""
     if not prof:
         return None
     R = 2 * N - 1
@@ -543,7 +567,8 @@ def roofline_entry(prof, shape, B, N, lens, steps, peaks):
                 "peak_kind": f"{peaks['source']} sustained bf16",
                 "avg_launch_ms": avg_s * 1e3, "launches": cnt}
     if top.startswith("attention"):
-        kv = sum(int(L) + R for L in lens) * shape.kv_dim * 2 * 2   # one layer's K+V
+        # one layer's K+V, averaged over the profiled steps
+        kv = float(np.mean([sum(int(L) + R for L in ls) for ls in lens_steps])) * shape.kv_dim * 2 * 2
         achieved = kv / avg_s / 1e9
         peak = peaks["hbm"]
         traffic = None

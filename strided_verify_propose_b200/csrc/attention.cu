@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "qkv_row.cuh"
 
 namespace isd {
 
@@ -51,6 +52,11 @@ struct AttnParams {
   int32_t min_tiles;           // fewest tiles per CTA (fewer CTAs for small work)
   int32_t kstages, vstages;    // K and V ring slots
   int32_t* status;
+  // tcgen05 kernel prologue: this layer's QKV reduction (QK-norm, RoPE, q and
+  // the block's K/V page writes) done by every CTA before any load
+  int32_t qkv_on;
+  QkvReduceArgs qkv;
+  int32_t* pro_cnt;            // [2] arrivals / departures (zero between launches)
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -747,6 +753,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
   }
   build_items(p, kend, base);     // ends with __syncthreads
+  if (p.qkv_on) {
+    // this layer's QKV reduction, (row, head) items spread over every warp of
+    // the grid, four per warp at a time with all their loads in flight; the
+    // producer issues no load before every CTA has finished its items
+    const int nw = blockDim.x / 32;
+    const int n_heads = p.qkv.n_q + 2 * p.qkv.n_kv;
+    const int items = p.qkv.rows * n_heads;
+    const int gws = gridDim.x * nw;
+    for (int i0 = blockIdx.x * nw + warp; i0 < items; i0 += 4 * gws) {
+      float v[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int it = i0 + k * gws;
+        if (it < items) qkv_head_sum<128>(p.qkv, it / n_heads, it % n_heads, lane, v[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int it = i0 + k * gws;
+        if (it < items) qkv_head_finish<128>(p.qkv, it / n_heads, it % n_heads, lane, v[k]);
+      }
+    }
+    // q and the K/V rows are read by TMA (the async proxy) in every CTA
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) atomicAdd(&p.pro_cnt[0], 1);
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // base[b]: tiles of the requests before b (128-key tiles, split_keys = 128)
@@ -759,6 +792,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0 && fits) {
       int tc = 0, it = 0, q_issued = 0, nk = 0;
       bool ok = true;
+      if (p.qkv_on) {
+        const int total = static_cast<int>(gridDim.x);
+        const long long t0 = clock64();
+        const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
+        while (ld_acquire_gpu(&p.pro_cnt[0]) < total) {
+          if (clock64() - t0 > limit) {
+            ok = false;
+            break;
+          }
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        if (atomicAdd(&p.pro_cnt[1], 1) == total - 1) {
+          p.pro_cnt[0] = 0;
+          p.pro_cnt[1] = 0;
+        }
+      }
       TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
       TcSeg sg;
       for (; ok && tc_next(p, base, rg, sg); ++it) {
@@ -1388,9 +1437,16 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                              int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
-                             cudaEvent_t between) {
+                             cudaEvent_t between, const QkvReduceArgs* qkv, int32_t* pro_cnt) {
   if (s.batch > kMaxBatch) return cudaErrorInvalidValue;
   const Derived d = derive(s);
+  // the QKV reduction runs first: inside the tcgen05 kernel, else on its own
+  const bool fuse_qkv = qkv != nullptr && d.tc && pro_cnt != nullptr && qkv->head_dim == 128;
+  if (qkv != nullptr && !fuse_qkv) {
+    const cudaError_t e = launch_qkv_reduce(*qkv, stream);
+    if (e != cudaSuccess) return e;
+    if (launches) *launches += 1;
+  }
   const int G = s.n_q_heads / s.n_kv_heads;
   // Q as [rows][n_q][head_dim]: a 3-D box {64 dims, G heads, R rows} holds the
   // R*G query rows that share one KV head, row qi = r * G + h.
@@ -1426,6 +1482,12 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
   p.part_ml = reinterpret_cast<float2*>(p.part_o + static_cast<size_t>(d.max_items) * rows * s.head_dim);
   p.item_base = reinterpret_cast<int32_t*>(p.part_ml + static_cast<size_t>(d.max_items) * rows);
   p.status = status;
+  p.qkv_on = fuse_qkv ? 1 : 0;
+  if (fuse_qkv) {
+    if (qkv->splits < 1 || qkv->splits > 8) return cudaErrorInvalidValue;
+    p.qkv = *qkv;
+  }
+  p.pro_cnt = pro_cnt;
   static bool attr_set = false;
   if (!attr_set) {
     // dynamic + static shared memory of each CTA within its share of the SM

@@ -152,6 +152,8 @@ struct isd_ctx {
   void* acc_ws = nullptr;
   size_t acc_ws_bytes = 0;
   int32_t* prefill_lens = nullptr;  // [max_batch]
+  int32_t* pro_cnt = nullptr;       // [2] grid barrier of the GEMM prologue
+  std::map<std::tuple<int, int, int>, int> coresident;   // per GEMM kernel variant: CTAs at once
   int32_t* prefill_order = nullptr; // [max_batch] requests by descending prompt length
   int32_t* prefill_ptab = nullptr;  // [max_batch][max pages] page table rows in that order
 
@@ -253,10 +255,19 @@ struct AugSpec {
   int k2;
 };
 
+// The residual add + RMSNorm that produces a GEMM's input (c->hn) from the
+// previous projection's split-K slices: run as the GEMM's prologue when the
+// GEMM's grid fits on the device at once, else as its own kernel first.
+struct PendingNorm {
+  const float* part = nullptr;
+  int splits = 0;
+  const float* norm_w = nullptr;
+};
+
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
-         const AugSpec* aug = nullptr) {
+         const AugSpec* aug = nullptr, const PendingNorm* pn = nullptr) {
   if (epi == isd::kEpiF32 && out_elems > 0) {
     // large prefill chunks: no more splits than the partial buffer holds
     const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
@@ -281,9 +292,28 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
     if (rc) return rc;
     ga = isd::GemmAugment{aug->tw2, tx2, aug->k2};
   }
+  isd::GemmPrologue pro{};
+  if (pn) {
+    const isd_model_cfg& g = c->cfg;
+    auto key = std::make_tuple(plan.pair, plan.n_mma, static_cast<int>(plan.smem_bytes));
+    auto it = c->coresident.find(key);
+    if (it == c->coresident.end()) it = c->coresident.emplace(key, isd::gemm_coresident_ctas(plan)).first;
+    const int64_t ctas = plan.streamk ? static_cast<int64_t>(plan.units) * (plan.pair ? 2 : 1)
+                                      : static_cast<int64_t>(n / 128) * plan.n_chunks * plan.splits;
+    if (x == c->hn && k == g.hidden && !aug && ctas <= it->second) {
+      pro = isd::GemmPrologue{1, pn->part, pn->splits, static_cast<int64_t>(m) * g.hidden, c->x,
+                              pn->norm_w, g.rms_eps, c->hn, m, g.hidden, c->pro_cnt, it->second};
+    } else {
+      cudaEvent_t r0 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_residual_norm(pn->part, pn->splits, m, g.hidden, pn->norm_w, g.rms_eps,
+                                         c->x, c->hn, st));
+      prof_add(c, kPResNorm, r0, prof_mark(c, st));
+      c->launches += 1;
+    }
+  }
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, aug ? &ga : nullptr));
+                            c->sk_ws_bytes, aug ? &ga : nullptr, pro.on ? &pro : nullptr));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
@@ -369,9 +399,11 @@ int lora_xa(isd_ctx* c, const CUtensorMap& ta, const __nv_bfloat16* x, int M, in
 // the page table with each row repeated attn_sub times); attention is
 // read-only on the cache, so this is the same computation in query tiles the
 // attention kernel holds.
+// tail: the residual add + RMSNorm (final norm) after the last layer, left
+// for the next GEMM (the LM head) to run; null when no GEMM follows.
 int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, int32_t* status,
                    cudaStream_t st, bool use_lora = false, int attn_sub = 1,
-                   const int32_t* attn_table = nullptr) {
+                   const int32_t* attn_table = nullptr, PendingNorm* tail = nullptr) {
   const isd_model_cfg& g = c->cfg;
   const int M = batch * rows_per_req;
   const int H = g.hidden;
@@ -397,6 +429,8 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
   if (isd::attention_workspace_bytes(ash) > c->attn_ws_bytes)
     return fail(ISD_E_UNSUPPORTED, "attention workspace too small for this batch shape");
 
+  PendingNorm pending;            // layer l's input norm, from layer l - 1's down slices
+  bool have_pending = false;
   for (int l = 0; l < g.n_layers; ++l) {
     int s = 1;
     int rc = ISD_OK;
@@ -405,11 +439,21 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     // gated adapter on q/k/v: xa first, then B rides on the base GEMM's last split
     AugSpec aug_qkv{ll ? &ll->tb_qkv : nullptr, c->lora_xa, 3 * r};
     if (ll) {
+      if (have_pending) {
+        // the adapter's x A^T reads the normalised input first
+        cudaEvent_t r0 = prof_mark(c, st);
+        ISD_CUDA(isd::launch_residual_norm(pending.part, pending.splits, M, H, pending.norm_w,
+                                           g.rms_eps, c->x, c->hn, st));
+        prof_add(c, kPResNorm, r0, prof_mark(c, st));
+        c->launches += 1;
+        have_pending = false;
+      }
       rc = lora_xa(c, ll->ta_qkv, c->hn, M, H, 3 * r, status, st);
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmQkv, c->tm_qkv[l], c->hn, M, c->qkv_dim, H, isd::kEpiF32, c->part,
-              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr);
+              c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_qkv : nullptr,
+              have_pending ? &pending : nullptr);
     if (rc) return rc;
     isd::QkvReduceArgs qa;
     qa.part = c->part;
@@ -434,14 +478,12 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
     qa.status = status;
-    cudaEvent_t a0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_qkv_reduce(qa, st));
-    c->launches += 1;
+    // the QKV reduction runs as the attention kernel's prologue where it can
     cudaEvent_t a1 = prof_mark(c, st);
-    prof_add(c, kPQkvReduce, a0, a1);
     cudaEvent_t amid = prof_event(c);
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
-                                   c->attn, c->attn_ws, status, st, &c->launches, amid));
+                                   c->attn, c->attn_ws, status, st, &c->launches, amid, &qa,
+                                   c->pro_cnt + 64));
     cudaEvent_t a2 = prof_mark(c, st);
     prof_add(c, kPAttnSplit, a1, amid);
     prof_add(c, kPAttnCombine, amid, a2);
@@ -453,10 +495,14 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
               c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
     if (rc) return rc;
-    cudaEvent_t r0 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
-    prof_add(c, kPResNorm, r0, prof_mark(c, st));
-    c->launches += 1;
+    // the MLP's input norm: the gate/up GEMM's prologue (or its own kernel)
+    PendingNorm mlp_in{c->part, s, c->mlp_norm[l]};
+    if (ll) {
+      cudaEvent_t r0 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, c->mlp_norm[l], g.rms_eps, c->x, c->hn, st));
+      prof_add(c, kPResNorm, r0, prof_mark(c, st));
+      c->launches += 1;
+    }
     // gate/up with the fused SiLU epilogue; with the adapter, its (xa, B)
     // K-blocks follow each tile's base K-blocks (stream-K cuts unchanged)
     AugSpec aug_gu{ll ? &ll->tb_gu : nullptr, c->lora_xa, 2 * r};
@@ -465,7 +511,8 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
       if (rc) return rc;
     }
     rc = gemm(c, kPGemmGateUp, c->tm_gu[l], c->hn, M, 2 * g.intermediate, H, isd::kEpiSiluMul,
-              nullptr, 0, 1, c->act, nullptr, status, st, ll ? &aug_gu : nullptr);
+              nullptr, 0, 1, c->act, nullptr, status, st, ll ? &aug_gu : nullptr,
+              ll ? nullptr : &mlp_in);
     if (rc) return rc;
     AugSpec aug_d{ll ? &ll->tb_d : nullptr, c->lora_xa, r};
     if (ll) {
@@ -475,11 +522,23 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     rc = gemm(c, kPGemmDown, c->tm_down[l], c->act, M, H, g.intermediate, isd::kEpiF32, c->part,
               c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr);
     if (rc) return rc;
-    const float* next_norm = l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm;
-    cudaEvent_t r1 = prof_mark(c, st);
-    ISD_CUDA(isd::launch_residual_norm(c->part, s, M, H, next_norm, g.rms_eps, c->x, c->hn, st));
-    prof_add(c, kPResNorm, r1, prof_mark(c, st));
-    c->launches += 1;
+    // the next layer's input norm (the final norm after the last layer),
+    // left to the next GEMM's prologue
+    pending = PendingNorm{c->part, s, l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm};
+    have_pending = true;
+  }
+  if (have_pending) {
+    if (tail) {
+      *tail = pending;
+    } else {
+      cudaEvent_t r1 = prof_mark(c, st);
+      ISD_CUDA(isd::launch_residual_norm(pending.part, pending.splits, M, H, pending.norm_w,
+                                         g.rms_eps, c->x, c->hn, st));
+      prof_add(c, kPResNorm, r1, prof_mark(c, st));
+      c->launches += 1;
+    }
+  } else if (tail) {
+    tail->part = nullptr;
   }
   return ISD_OK;
 }
@@ -538,6 +597,7 @@ int alloc_workspace(isd_ctx* c) {
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
       static_cast<size_t>(g.max_batch) * 4,                                    // prefill order
+      512,                    // prologue barriers: [0, 64) GEMM, [64, 128) attention ints
       static_cast<size_t>(g.max_batch) * max_pages * 4,                        // prefill page rows
   };
   size_t total = 0;
@@ -569,9 +629,11 @@ int alloc_workspace(isd_ctx* c) {
   c->sk_ws = b + off[i++];
   c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
   c->prefill_order = reinterpret_cast<int32_t*>(b + off[i++]);
+  c->pro_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
   c->prefill_ptab = reinterpret_cast<int32_t*>(b + off[i++]);
-  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
-    return fail(ISD_E_CUDA, "stream-K workspace clear failed");
+  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
+      cudaMemset(c->pro_cnt, 0, 512) != cudaSuccess)
+    return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;
   std::vector<float2> tab(static_cast<size_t>(g.max_position) * half);
@@ -800,15 +862,18 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
                                      g.mask_token_id, meta, status_dev, st));
   prof_add(ctx, kPAssemble, e0, prof_mark(ctx, st));
   ctx->launches += 1;
-  rc = forward_layers(ctx, kv, B, R, status_dev, st, use_lora);
+  PendingNorm tail;
+  rc = forward_layers(ctx, kv, B, R, status_dev, st, use_lora, 1, nullptr, &tail);
   if (rc) return rc;
   const int M = B * R;
   if (!batch->logits_out_dev && static_cast<size_t>(M) > ctx->logit_rows)
     return fail(ISD_E_UNSUPPORTED, "more block rows than the logits workspace holds");
   float* logits = batch->logits_out_dev ? batch->logits_out_dev : ctx->logits;
-  // the LM head writes the logits themselves: never split-K
+  // the LM head writes the logits themselves: never split-K; its prologue
+  // applies the final norm
   rc = gemm(ctx, kPGemmLmHead, ctx->tm_lm, ctx->hn, M, g.vocab, g.hidden, isd::kEpiF32, logits,
-            static_cast<size_t>(M) * g.vocab, 1, nullptr, nullptr, status_dev, st);
+            static_cast<size_t>(M) * g.vocab, 1, nullptr, nullptr, status_dev, st, nullptr,
+            tail.part ? &tail : nullptr);
   if (rc) return rc;
   isd::AcceptArgs a;
   a.logits = logits;

@@ -64,6 +64,29 @@ struct GemmAugment {
   int32_t k;
 };
 
+// A prologue that produces the GEMM's own input before its mainloop: the
+// residual add and RMSNorm of the previous projection's split-K slices,
+// x[row] += sum_s part[s][row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w),
+// with hn the GEMM's X. The CTAs share the rows, arrive on cnt[0] and load
+// no token tile before every CTA has arrived, so the whole grid must be
+// resident at once (coresident: gemm_coresident_ctas of the plan). cnt[2]
+// starts at zero; each launch leaves it zero.
+struct GemmPrologue {
+  int32_t on;
+  const float* part;
+  int32_t splits;
+  int64_t split_stride;
+  float* x;
+  const float* norm_w;
+  float eps;
+  __nv_bfloat16* hn;
+  int32_t rows, hidden;
+  int32_t* cnt;
+  int32_t coresident;
+};
+// CTAs of this plan's kernel that can be resident on the device at once.
+int gemm_coresident_ctas(const GemmPlan& plan);
+
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
 // with W's rows interleaved in blocks of 16 (gate rows then up rows).
@@ -71,7 +94,8 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmAugment* augment = nullptr);
+                        const GemmAugment* augment = nullptr,
+                        const GemmPrologue* prologue = nullptr);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {
@@ -88,11 +112,17 @@ int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_
                     int seg_capacity, int* n_segments, int* max_parts);
 // k_map / v_map: tensor maps over the pools as [n_layers*num_pages*n_kv*page_size][head_dim]
 // with box_rows = page_size.
+// qkv (optional): this layer's QKV split-K reduction, which produces q and
+// the block's K/V rows; the tcgen05 kernel runs it as its prologue (pro_cnt:
+// two ints, zero before the first launch, left zero), otherwise it is
+// launched first on its own.
+struct QkvReduceArgs;
 cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map, const AttnShape& s,
                              int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
-                             cudaEvent_t between = nullptr);
+                             cudaEvent_t between = nullptr, const QkvReduceArgs* qkv = nullptr,
+                             int32_t* pro_cnt = nullptr);
 
 // ------------------------------------------------------------------ row ops
 struct RowMeta {

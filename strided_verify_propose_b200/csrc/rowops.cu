@@ -7,6 +7,7 @@
 // independent of what happens on MASK rows.
 #include "common.cuh"
 #include "kernels.h"
+#include "qkv_row.cuh"
 
 namespace isd {
 
@@ -190,75 +191,13 @@ constexpr int kQkvMaxSplits = 8;
 template <int HD>
 // (4 CTAs of 512 threads per SM: at most 32 registers per thread)
 __global__ void __launch_bounds__(kQkvWarps * 32, 4) qkv_reduce_kernel(const QkvReduceArgs a) {
-  constexpr int J = HD / 32;       // values per lane
-  constexpr int JH = J / 2;        // partner offset (d + HD/2)
   const int row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_heads = a.n_q + 2 * a.n_kv;
   const int hd = blockIdx.y * kQkvWarps + warp;
-  if (hd >= n_heads) return;
-  const int qkv_dim = n_heads * HD;
-  const int64_t split_stride = static_cast<int64_t>(a.rows) * qkv_dim;
-  const float* pr = a.part + static_cast<int64_t>(row) * qkv_dim + hd * HD + lane;
-  const int flags = a.meta.flags[row];
-  int pos = a.meta.pos[row];
-  const bool write_kv = (flags & kRowWriteKV) && pos >= 0;
-  if (pos >= a.max_position) {
-    if (lane == 0 && hd == 0) flag(a.status, ISD_DEV_BAD_STATE);
-    pos = a.max_position - 1;
-  }
-  const int rpos = pos < 0 ? 0 : pos;
-  float v[J];
-#pragma unroll
-  for (int j = 0; j < J; ++j) v[j] = 0.f;
-  // splits added in ascending order (bitwise reproducible)
-#pragma unroll
-  for (int sp = 0; sp < kQkvMaxSplits; ++sp) {
-    if (sp < a.splits) {
-#pragma unroll
-      for (int j = 0; j < J; ++j) v[j] += pr[sp * split_stride + 32 * j];
-    }
-  }
-  if (hd < a.n_q + a.n_kv) {
-    const float* nw = hd < a.n_q ? a.q_norm : a.k_norm;
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < J; ++j) ss += v[j] * v[j];
-    ss = warp_sum(ss);
-    const float rstd = rsqrtf(ss / HD + a.eps);
-#pragma unroll
-    for (int j = 0; j < J; ++j) v[j] *= rstd * nw[lane + 32 * j];
-    const float2* cs = a.rope + static_cast<int64_t>(rpos) * (HD / 2);
-#pragma unroll
-    for (int j = 0; j < JH; ++j) {
-      const float2 c = cs[lane + 32 * j];
-      const float x1 = v[j], x2 = v[j + JH];
-      v[j] = x1 * c.x - x2 * c.y;
-      v[j + JH] = x2 * c.x + x1 * c.y;
-    }
-  }
-  if (hd < a.n_q) {
-    __nv_bfloat16* qo = a.q_out + (static_cast<int64_t>(row) * a.n_q + hd) * HD;
-#pragma unroll
-    for (int j = 0; j < J; ++j) qo[lane + 32 * j] = __float2bfloat16_rn(v[j]);
-  } else if (write_kv) {
-    const int b = row / a.rows_per_req;
-    const int pidx = pos / a.page_size;
-    const int page = pidx < a.max_pages_per_req
-                         ? a.page_table[static_cast<int64_t>(b) * a.max_pages_per_req + pidx]
-                         : -1;
-    if (page < 0 || page >= a.num_pages) {
-      if (lane == 0) flag(a.status, ISD_DEV_BAD_PAGE);
-      return;
-    }
-    const int64_t slot_base = (static_cast<int64_t>(a.layer) * a.num_pages + page) * a.n_kv;
-    const bool is_k = hd < a.n_q + a.n_kv;
-    const int g = is_k ? hd - a.n_q : hd - a.n_q - a.n_kv;
-    __nv_bfloat16* dst = (is_k ? a.k_pool : a.v_pool) +
-                         (((slot_base + g) * a.page_size) + pos % a.page_size) * HD;
-#pragma unroll
-    for (int j = 0; j < J; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(v[j]);
-  }
+  if (hd >= a.n_q + 2 * a.n_kv) return;
+  float v[HD / 32];
+  qkv_head_sum<HD>(a, row, hd, lane, v);
+  qkv_head_finish<HD>(a, row, hd, lane, v);
 }
 
 }  // namespace
