@@ -64,11 +64,15 @@ WORKLOADS = {
     # R-ISD: Qwen3-8B shape + rank-128 gated LoRA on MASK rows, batch 32, N=4, prompts 2048
     "risd_8b_b32": dict(shape=synth.QWEN3_8B, batch=32, stride=4, len_lo=2048, len_hi=2048,
                         lora_rank=128),
+    # the headline configuration cut to two layers (same batch, prompts, pages): the
+    # per-layer kernels at the headline shapes in a few GB, for ncu captures
+    "qwen3_8b_b64_l2": dict(shape=synth.QWEN3_8B_2L, batch=64, stride=4, len_lo=512, len_hi=4096),
     # Qwen3-32B shape (64 layers, hidden 5120, 64/8 heads), batch 64, N=4, prompts U[1024, 8192]
     "qwen3_32b_b64": dict(shape=synth.QWEN3_32B, batch=64, stride=4, len_lo=1024, len_hi=8192),
 }
 ACCEPT_RATE = 0.9
 MODEL_NAMES = {synth.QWEN3_8B: "qwen3-8b-shape (random init)",
+               synth.QWEN3_8B_2L: "qwen3-8b-shape, 2 layers (random init)",
                synth.QWEN3_32B: "qwen3-32b-shape (random init)"}
 
 
@@ -527,11 +531,11 @@ def extra_configs(model, shape, args, seed):
     return out
 
 
-# DRAM bytes (read + write) per byte of K + V of the tcgen05 attention kernel,
-# from one ncu capture of the kernel at this workload shape (one layer, batch 64)
-# (603.6 MB for a launch over 580.4 MB of K + V at the same workload shape);
-# the roofline's `traffic` scales it to this run's launch.
-ATTN_DRAM_PER_KV_BYTE = 603.6 / 580.4
+# DRAM bytes (read + write) of the step's attention launch (the tcgen05
+# kernel with its QKV-reduction prologue) per algorithmic byte, from one ncu
+# capture of the same launch in the two-layer headline workload; the
+# roofline's `traffic` scales it to this run's launch. None until captured.
+ATTN_DRAM_PER_ALGO_BYTE = None
 
 
 def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
@@ -569,14 +573,22 @@ def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
     if top.startswith("attention"):
         # one layer's K+V, averaged over the profiled steps
         kv = float(np.mean([sum(int(L) + R for L in ls) for ls in lens_steps])) * shape.kv_dim * 2 * 2
-        achieved = kv / avg_s / 1e9
+        algo = kv
+        fused = (top == "attention" and shape.head_dim == 128 and shape.page_size == 64
+                 and R * (shape.n_q_heads // shape.n_kv_heads) <= 64)
+        if fused:
+            # the launch also finishes the layer's QKV projection: its fp32
+            # output read once, q and the block's K/V rows written in bf16
+            algo += M * shape.qkv_dim * 4 + M * (shape.q_dim + 2 * shape.kv_dim) * 2
+        achieved = algo / avg_s / 1e9
         peak = peaks["hbm"]
         traffic = None
-        if top == "attention" and shape.head_dim == 128 and shape.page_size == 64:
-            traffic = ATTN_DRAM_PER_KV_BYTE * kv   # bytes per launch (scaled ncu capture)
+        if fused and ATTN_DRAM_PER_ALGO_BYTE is not None:
+            traffic = ATTN_DRAM_PER_ALGO_BYTE * algo   # bytes per launch (scaled ncu capture)
         return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "traffic_note": "ncu dram read+write of one capture, scaled by K+V bytes",
+                "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": algo,
+                "traffic_note": "ncu dram read+write of one capture of the same launch, scaled "
+                                "by algorithmic bytes",
                 "peak_kind": f"{peaks['source']} HBM copy",
                 "avg_launch_ms": avg_s * 1e3, "launches": cnt}
     return {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s",

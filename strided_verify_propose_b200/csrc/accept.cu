@@ -13,7 +13,9 @@
 //
 // Kernels:
 //  1. accept_stats: one CTA per (row, 8192-token chunk): max, sum of
-//     exp(z - max) and the first argmax of the chunk.
+//     exp(z - max) and the first argmax of the chunk, from the logits, or
+//     (accept_slab_stats) from the statistics of 32-token slabs that the
+//     LM head's epilogue wrote beside the logits.
 //  2. accept_decide: one CTA per request: combines the chunk statistics,
 //     runs the sequential accept tests, draws the new token by inverse CDF
 //     (chunk totals first, then a block scan inside one chunk) and reads or
@@ -93,6 +95,48 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int j = 0; j < kVec; ++j)
       s += (expf(v4[j].x - m) + expf(v4[j].y - m)) + (expf(v4[j].z - m) + expf(v4[j].w - m));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float v2 = __shfl_xor_sync(0xffffffffu, av, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, ai, o);
+    merge_ms(m, s, m2, s2);
+    merge_arg(av, ai, v2, i2);
+  }
+  __shared__ ChunkStat part[kThreads / 32];
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) part[w] = ChunkStat{m, s, av, ai};
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    ChunkStat r = part[0];
+    for (int k = 1; k < kThreads / 32; ++k) {
+      merge_ms(r.m, r.s, part[k].m, part[k].s);
+      merge_arg(r.amax, r.idx, part[k].amax, part[k].idx);
+    }
+    stats[static_cast<int64_t>(row) * n_chunks + c] = r;
+  }
+}
+
+// The same chunk statistics from the LM head's per-(row, 32-token slab)
+// statistics: thread t merges slab c * 256 + t, then the warps and the
+// block merge as above (max and argmax are exact; the sums differ from the
+// logits pass only in the order of the additions).
+__global__ void __launch_bounds__(kThreads)
+    accept_slab_stats_kernel(const float4* slab, int32_t vocab, int32_t n_chunks, ChunkStat* stats) {
+  static_assert(kChunk == 32 * kThreads, "one slab per thread");
+  const int c = blockIdx.x, row = blockIdx.y;
+  const int n_slabs = vocab / 32;
+  const int sl = c * kThreads + threadIdx.x;
+  float m = -INFINITY, s = 0.f, av = -INFINITY;
+  int ai = INT_MAX;
+  if (sl < n_slabs) {
+    const float4 t = slab[static_cast<int64_t>(row) * n_slabs + sl];
+    m = t.x;
+    s = t.y;
+    av = t.z;
+    ai = __float_as_int(t.w);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -459,8 +503,14 @@ cudaError_t launch_accept(const AcceptArgs& a, void* workspace, cudaStream_t str
   const int R = 2 * a.stride_n - 1;
   const int n_chunks = (a.vocab + kChunk - 1) / kChunk;
   ChunkStat* stats = static_cast<ChunkStat*>(workspace);
-  accept_stats_kernel<<<dim3(n_chunks, a.batch * R), kThreads, 0, stream>>>(a.logits, a.vocab,
-                                                                           n_chunks, stats);
+  if (a.slab_stats != nullptr) {
+    if (a.vocab % 32 != 0) return cudaErrorInvalidValue;
+    accept_slab_stats_kernel<<<dim3(n_chunks, a.batch * R), kThreads, 0, stream>>>(
+        a.slab_stats, a.vocab, n_chunks, stats);
+  } else {
+    accept_stats_kernel<<<dim3(n_chunks, a.batch * R), kThreads, 0, stream>>>(a.logits, a.vocab,
+                                                                             n_chunks, stats);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;   // each kernel reads what the previous one wrote
   if (between0) cudaEventRecord(between0, stream);

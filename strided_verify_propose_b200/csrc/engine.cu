@@ -143,6 +143,7 @@ struct isd_ctx {
   __nv_bfloat16* attn = nullptr;    // [max_rows][q_dim]
   __nv_bfloat16* act = nullptr;     // [max_rows][intermediate]
   float* logits = nullptr;          // [logit_rows][vocab]
+  float4* slab_stats = nullptr;     // [logit_rows][vocab / 32] from the LM head's epilogue
   int32_t* meta_tok = nullptr;
   int32_t* meta_pos = nullptr;
   int32_t* meta_flags = nullptr;
@@ -152,8 +153,7 @@ struct isd_ctx {
   void* acc_ws = nullptr;
   size_t acc_ws_bytes = 0;
   int32_t* prefill_lens = nullptr;  // [max_batch]
-  int32_t* pro_cnt = nullptr;       // [2] grid barrier of the GEMM prologue
-  std::map<std::tuple<int, int, int>, int> coresident;   // per GEMM kernel variant: CTAs at once
+  int32_t* pro_cnt = nullptr;       // [2] grid-barrier words of the attention's prologue
   int32_t* prefill_order = nullptr; // [max_batch] requests by descending prompt length
   int32_t* prefill_ptab = nullptr;  // [max_batch][max pages] page table rows in that order
 
@@ -256,8 +256,9 @@ struct AugSpec {
 };
 
 // The residual add + RMSNorm that produces a GEMM's input (c->hn) from the
-// previous projection's split-K slices: run as the GEMM's prologue when the
-// GEMM's grid fits on the device at once, else as its own kernel first.
+// previous projection's split-K slices, launched right before that GEMM.
+// (Run as the GEMM's own prologue, behind a barrier over its grid, it cost
+// more per step than the separate launch.)
 struct PendingNorm {
   const float* part = nullptr;
   int splits = 0;
@@ -267,7 +268,8 @@ struct PendingNorm {
 int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int m, int n, int k,
          isd::GemmEpilogue epi, float* out, size_t out_elems, int max_splits,
          __nv_bfloat16* act, int* splits_used, int32_t* status, cudaStream_t st,
-         const AugSpec* aug = nullptr, const PendingNorm* pn = nullptr) {
+         const AugSpec* aug = nullptr, const PendingNorm* pn = nullptr,
+         float4* row_stats = nullptr) {
   if (epi == isd::kEpiF32 && out_elems > 0) {
     // large prefill chunks: no more splits than the partial buffer holds
     const size_t fit = out_elems / (static_cast<size_t>(m) * static_cast<size_t>(n));
@@ -292,28 +294,17 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
     if (rc) return rc;
     ga = isd::GemmAugment{aug->tw2, tx2, aug->k2};
   }
-  isd::GemmPrologue pro{};
   if (pn) {
     const isd_model_cfg& g = c->cfg;
-    auto key = std::make_tuple(plan.pair, plan.n_mma, static_cast<int>(plan.smem_bytes));
-    auto it = c->coresident.find(key);
-    if (it == c->coresident.end()) it = c->coresident.emplace(key, isd::gemm_coresident_ctas(plan)).first;
-    const int64_t ctas = plan.streamk ? static_cast<int64_t>(plan.units) * (plan.pair ? 2 : 1)
-                                      : static_cast<int64_t>(n / 128) * plan.n_chunks * plan.splits;
-    if (x == c->hn && k == g.hidden && !aug && ctas <= it->second) {
-      pro = isd::GemmPrologue{1, pn->part, pn->splits, static_cast<int64_t>(m) * g.hidden, c->x,
-                              pn->norm_w, g.rms_eps, c->hn, m, g.hidden, c->pro_cnt, it->second};
-    } else {
-      cudaEvent_t r0 = prof_mark(c, st);
-      ISD_CUDA(isd::launch_residual_norm(pn->part, pn->splits, m, g.hidden, pn->norm_w, g.rms_eps,
-                                         c->x, c->hn, st));
-      prof_add(c, kPResNorm, r0, prof_mark(c, st));
-      c->launches += 1;
-    }
+    cudaEvent_t r0 = prof_mark(c, st);
+    ISD_CUDA(isd::launch_residual_norm(pn->part, pn->splits, m, g.hidden, pn->norm_w, g.rms_eps,
+                                       c->x, c->hn, st));
+    prof_add(c, kPResNorm, r0, prof_mark(c, st));
+    c->launches += 1;
   }
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, aug ? &ga : nullptr, pro.on ? &pro : nullptr));
+                            c->sk_ws_bytes, aug ? &ga : nullptr, row_stats));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;
@@ -483,7 +474,8 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     cudaEvent_t amid = prof_event(c);
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid, &qa,
-                                   c->pro_cnt + 64));
+                                   c->pro_cnt, attn_sub == 1 && ash_table == kv->page_table_dev &&
+                                                        rows_per_req == ash.rows_per_req));
     cudaEvent_t a2 = prof_mark(c, st);
     prof_add(c, kPAttnSplit, a1, amid);
     prof_add(c, kPAttnCombine, amid, a2);
@@ -495,7 +487,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     rc = gemm(c, kPGemmO, c->tm_o[l], c->attn, M, H, c->q_dim, isd::kEpiF32, c->part, c->part_elems,
               c->max_splits, nullptr, &s, status, st, ll ? &aug_o : nullptr);
     if (rc) return rc;
-    // the MLP's input norm: the gate/up GEMM's prologue (or its own kernel)
+    // the MLP's input norm, launched before the gate/up GEMM
     PendingNorm mlp_in{c->part, s, c->mlp_norm[l]};
     if (ll) {
       cudaEvent_t r0 = prof_mark(c, st);
@@ -523,7 +515,7 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
               c->part_elems, c->max_splits, nullptr, &s, status, st, ll ? &aug_d : nullptr);
     if (rc) return rc;
     // the next layer's input norm (the final norm after the last layer),
-    // left to the next GEMM's prologue
+    // launched before the next GEMM
     pending = PendingNorm{c->part, s, l + 1 < g.n_layers ? c->attn_norm[l + 1] : c->final_norm};
     have_pending = true;
   }
@@ -597,8 +589,9 @@ int alloc_workspace(isd_ctx* c) {
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
       static_cast<size_t>(g.max_batch) * 4,                                    // prefill order
-      512,                    // prologue barriers: [0, 64) GEMM, [64, 128) attention ints
+      512,                    // grid-barrier words of the attention's prologue (2 used)
       static_cast<size_t>(g.max_batch) * max_pages * 4,                        // prefill page rows
+      step_rows * static_cast<size_t>(g.vocab / 32) * sizeof(float4),          // slab statistics
   };
   size_t total = 0;
   std::vector<size_t> off;
@@ -631,6 +624,7 @@ int alloc_workspace(isd_ctx* c) {
   c->prefill_order = reinterpret_cast<int32_t*>(b + off[i++]);
   c->pro_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
   c->prefill_ptab = reinterpret_cast<int32_t*>(b + off[i++]);
+  c->slab_stats = reinterpret_cast<float4*>(b + off[i++]);
   if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
       cudaMemset(c->pro_cnt, 0, 512) != cudaSuccess)
     return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
@@ -869,11 +863,14 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
   if (!batch->logits_out_dev && static_cast<size_t>(M) > ctx->logit_rows)
     return fail(ISD_E_UNSUPPORTED, "more block rows than the logits workspace holds");
   float* logits = batch->logits_out_dev ? batch->logits_out_dev : ctx->logits;
-  // the LM head writes the logits themselves: never split-K; its prologue
-  // applies the final norm
+  // the LM head writes the logits themselves: never split-K; the final norm
+  // is launched before it. Its epilogue also writes the max, sum of exp and
+  // first argmax of every 32 logits, which the accept step merges instead
+  // of reading the logits once more.
+  float4* slab = static_cast<size_t>(M) <= ctx->logit_rows ? ctx->slab_stats : nullptr;
   rc = gemm(ctx, kPGemmLmHead, ctx->tm_lm, ctx->hn, M, g.vocab, g.hidden, isd::kEpiF32, logits,
             static_cast<size_t>(M) * g.vocab, 1, nullptr, nullptr, status_dev, st, nullptr,
-            tail.part ? &tail : nullptr);
+            tail.part ? &tail : nullptr, slab);
   if (rc) return rc;
   isd::AcceptArgs a;
   a.logits = logits;
@@ -896,6 +893,7 @@ int isd_step(isd_ctx* ctx, const isd_batch* batch, const isd_kv* kv, int32_t* pe
   a.max_pages_per_req = kv->max_pages_per_req;
   a.free_count = kv->free_count;
   a.status = status_dev;
+  a.slab_stats = slab;
   cudaEvent_t c0 = prof_mark(ctx, st);
   cudaEvent_t c1 = prof_event(ctx), c2 = prof_event(ctx);
   ISD_CUDA(isd::launch_accept(a, ctx->acc_ws, st, &ctx->launches, c1, c2));

@@ -62,70 +62,54 @@ struct GemmParams {
   // continues over aug_kb K-blocks of a second operand pair (tmap_w2,
   // tmap_x2), accumulating into the same result
   int32_t aug_kb;
-  // prologue: the GEMM's own input X is produced first (see GemmPrologue)
-  GemmPrologue pro;
+  // kEpiF32 with one slice: per (token, 32-row slab) max, sum of exp(y - max)
+  // and first argmax of the finished result, [m][n_out / 32]
+  float4* row_stats;
 };
 
-// The residual add and RMSNorm of one row by the 256 epilogue threads: the
-// same arithmetic, in the same order, as residual_norm_kernel (x, then the
-// splits ascending; a warp sum, then the 8 warp sums in warp order).
-__device__ __forceinline__ void prologue_row(const GemmPrologue& a, int row, int tid, float* red) {
-  constexpr int kIt = 8;                 // hidden <= 256 threads x 4 x 8
-  float* xr = a.x + static_cast<int64_t>(row) * a.hidden;
-  const float* pr = a.part + static_cast<int64_t>(row) * a.hidden;
-  float4 v[kIt];
+// For each of the 32 values a lane holds (value j of every lane is token j;
+// lane L holds output row f0 + L): the max over the warp's 32 rows, the sum
+// of exp(y - max) over them and the first row reaching the max. A butterfly:
+// at offset o a lane keeps half of its 2o entries and merges the partner's
+// copy of that half into them (31 merges per lane), so that lane L ends with
+// token L's result. In a merge one of the two rescale factors is exp(0) = 1,
+// so each merge takes one exponential, of minus the gap between the maxima.
+__device__ __forceinline__ void slab_stats32(const float (&v)[32], int f, int lane, float& m_out,
+                                             float& s_out, int& i_out) {
+  float m[16], s[16];
+  int id[16];
+  {
+    const bool lo = (lane & 16) == 0;
+    const int fb = f ^ 16;
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    const int i = (it * 256 + tid) * 4;
-    v[it] = i < a.hidden ? *reinterpret_cast<const float4*>(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int sp = 0; sp < a.splits; ++sp) {
-#pragma unroll
-    for (int it = 0; it < kIt; ++it) {
-      const int i = (it * 256 + tid) * 4;
-      if (i < a.hidden) {
-        const float4 d = __ldcg(reinterpret_cast<const float4*>(pr + sp * a.split_stride + i));
-        v[it].x += d.x;
-        v[it].y += d.y;
-        v[it].z += d.z;
-        v[it].w += d.w;
-      }
+    for (int k = 0; k < 16; ++k) {
+      const float a = lo ? v[k] : v[k + 16];
+      const float b = __shfl_xor_sync(0xffffffffu, lo ? v[k + 16] : v[k], 16);
+      s[k] = 1.f + __expf(-fabsf(a - b));
+      m[k] = fmaxf(a, b);
+      id[k] = (b > a || (b == a && fb < f)) ? fb : f;
     }
   }
-  float ss = 0.f;
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    const int i = (it * 256 + tid) * 4;
-    if (i < a.hidden) {
-      *reinterpret_cast<float4*>(xr + i) = v[it];
-      ss += v[it].x * v[it].x + v[it].y * v[it].y + v[it].z * v[it].z + v[it].w * v[it].w;
+  for (int o = 8; o >= 1; o >>= 1) {
+    const bool lo = (lane & o) == 0;
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float am = lo ? m[k] : m[k + o], as = lo ? s[k] : s[k + o];
+      const int ai = lo ? id[k] : id[k + o];
+      const float bm = __shfl_xor_sync(0xffffffffu, lo ? m[k + o] : m[k], o);
+      const float bs = __shfl_xor_sync(0xffffffffu, lo ? s[k + o] : s[k], o);
+      const int bi = __shfl_xor_sync(0xffffffffu, lo ? id[k + o] : id[k], o);
+      const float gap = am - bm;
+      const float e = __expf(-fabsf(gap));
+      s[k] = gap >= 0.f ? fmaf(bs, e, as) : fmaf(as, e, bs);
+      m[k] = fmaxf(am, bm);
+      id[k] = (bm > am || (bm == am && bi < ai)) ? bi : ai;
     }
   }
-  ss = warp_sum(ss);
-  if ((tid & 31) == 0) red[tid >> 5] = ss;
-  named_bar_sync(1, 256);
-  float tot = 0.f;
-  if (tid < 32) {
-    tot = tid < 8 ? red[tid] : 0.f;
-    tot = warp_sum(tot);
-    if (tid == 0) red[8] = tot;
-  }
-  named_bar_sync(1, 256);
-  tot = red[8];
-  named_bar_sync(1, 256);
-  const float rstd = rsqrtf(tot / a.hidden + a.eps);
-  __nv_bfloat16* hr = a.hn + static_cast<int64_t>(row) * a.hidden;
-#pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    const int i = (it * 256 + tid) * 4;
-    if (i < a.hidden) {
-      const float4 w = *reinterpret_cast<const float4*>(a.norm_w + i);
-      __align__(8) __nv_bfloat16 o4[4] = {
-          __float2bfloat16_rn(v[it].x * rstd * w.x), __float2bfloat16_rn(v[it].y * rstd * w.y),
-          __float2bfloat16_rn(v[it].z * rstd * w.z), __float2bfloat16_rn(v[it].w * rstd * w.w)};
-      *reinterpret_cast<uint2*>(hr + i) = *reinterpret_cast<const uint2*>(o4);
-    }
-  }
+  m_out = m[0];
+  s_out = s[0];
+  i_out = id[0];
 }
 
 // One contiguous run of K-blocks of one tile, processed by one CTA (pair).
@@ -192,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ int epi_mode;
-  __shared__ float pro_red[9];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tok0 = blockIdx.y * p.n_pad;
@@ -252,33 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool ok = true;
     Segment sg;
-    if (p.pro.on) {
-      // the weights of the first stages head for L2 while the prologue runs;
-      // the token tiles are the prologue's output, so no load is issued
-      // before every CTA of the grid has written its rows
-      if (get_segment<kPair>(p, 0, sg)) {
-        const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
-        for (int i = 0; i < p.stages && sg.kb_lo + i < sg.kb_hi; ++i)
-          tma_prefetch_2d(&tmap_w, (sg.kb_lo + i) * kTileK, mt * kTileM);
-      }
-      const int total = static_cast<int>(gridDim.x * gridDim.y * gridDim.z);
-      const long long t0 = clock64();
-      const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
-      while (ld_acquire_gpu(&p.pro.cnt[0]) < total) {
-        if (clock64() - t0 > limit) {
-          flag(p.status, ISD_DEV_TIMEOUT);
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-      }
-      // the rows were written through the generic proxy; TMA reads them
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      if (atomicAdd(&p.pro.cnt[1], 1) == total - 1) {
-        p.pro.cnt[0] = 0;
-        p.pro.cnt[1] = 0;
-      }
-    }
     for (int idx = 0; ok && get_segment<kPair>(p, idx, sg); ++idx) {
       const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
       const int n_base = sg.kb_hi - sg.kb_lo;
@@ -399,18 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nchunk = (p.n_pad + 31) / 32;  // tmem_cols >= 32 * nchunk
     const uint32_t empty_addr = kPair ? map_to_rank(smem_u32(tmem_empty), 0) : 0u;
     const int split = p.streamk ? 0 : static_cast<int>(blockIdx.z);
-    if (p.pro.on) {
-      // this CTA's rows of the prologue (row = CTA, + CTAs, ...), then its
-      // arrival on the grid counter
-      const int cta = static_cast<int>(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-      const int ctas = static_cast<int>(gridDim.x * gridDim.y * gridDim.z);
-      for (int row = cta; row < p.pro.rows; row += ctas) prologue_row(p.pro, row, ew * 32 + lane, pro_red);
-      // the rows are read by TMA (the async proxy) in every CTA
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      __threadfence();
-      named_bar_sync(1, 32 * kEpiWarps);
-      if (ew == 0 && lane == 0) atomicAdd(&p.pro.cnt[0], 1);
-    }
     Segment sg;
     for (int idx = 0; get_segment<kPair>(p, idx, sg); ++idx) {
       // every epilogue warp takes the same branch (they share named barriers)
@@ -492,6 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c * 32 + j < p.n_pad && t0 + j < p.m) *rowp = v[j];
               rowp += p.n_out;
             }
+          }
+          if (p.row_stats != nullptr) {
+            // lane L: token t0 + L over this quadrant's 32 output rows
+            float sm, ss;
+            int si;
+            slab_stats32(v, f, lane, sm, ss, si);
+            if (c * 32 + lane < p.n_pad && t0 + lane < p.m)
+              p.row_stats[static_cast<int64_t>(t0 + lane) * (p.n_out / 32) + (f >> 5)] =
+                  make_float4(sm, ss, sm, __int_as_float(si));
           }
         } else {
           // Each quadrant's 32 TMEM lanes hold 16 gate rows then the 16 up
@@ -629,7 +582,11 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
       kStageA + static_cast<size_t>(best.n_boxes) * static_cast<size_t>(best.box_rows) * 128;
   const size_t extra = 1024 + 256;
   int stages = static_cast<int>((kMaxSmem - extra) / stage);
-  stages = std::min(stages, 8);
+  // few tokens (decode at small batch): a K-block is nearly all weights and
+  // the ring is what keeps HBM busy, so it takes all the shared memory, up to
+  // the 12 slots whose barriers fit the 256 bytes after the ring
+  // ((2 x 12 + 2) x 8 + 8 bytes)
+  stages = std::min(stages, 12);
   if (!best.streamk) stages = std::min(stages, std::max(best.kb_per_split, 2));
   best.stages = std::max(stages, 2);
   best.tmem_cols = pow2_at_least(static_cast<uint32_t>(best.n_pad));
@@ -654,43 +611,11 @@ size_t gemm_streamk_sync_bytes() { return kSkSyncBytes; }
 
 cudaError_t set_wait_limit_gemm(long long cycles) { return set_wait_limit_here(cycles); }
 
-int gemm_coresident_ctas(const GemmPlan& plan) {
-  auto kernel = plan.pair
-                    ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
-                    : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kMaxSmem)) != cudaSuccess)
-    return 0;
-  if (!plan.pair) {
-    int per_sm = 0, dev = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads,
-                                                      plan.smem_bytes) != cudaSuccess ||
-        cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return 0;
-    return per_sm * sms;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = plan.smem_bytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) return 0;
-  return 2 * clusters;
-}
-
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace, size_t sk_workspace_bytes,
-                        const GemmAugment* augment, const GemmPrologue* prologue) {
+                        const GemmAugment* augment, float4* row_stats) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -728,19 +653,9 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.sk_part = nullptr;
   p.sk_sync = nullptr;
   p.aug_kb = 0;
-  p.pro = GemmPrologue{};
-  if (prologue != nullptr && prologue->on) {
-    // every CTA of the grid waits for every other's rows: the whole grid must
-    // be resident at once
-    const int64_t ctas = plan.streamk ? static_cast<int64_t>(plan.units) * (plan.pair ? 2 : 1)
-                                      : static_cast<int64_t>(n_out / kTileM) * plan.n_chunks * plan.splits;
-    if (prologue->cnt == nullptr || prologue->x == nullptr || prologue->hn == nullptr ||
-        prologue->norm_w == nullptr || prologue->hidden % 4 || prologue->hidden > 8192 ||
-        prologue->splits < 0 || (prologue->splits > 0 && prologue->part == nullptr) ||
-        ctas > prologue->coresident)
-      return cudaErrorInvalidValue;
-    p.pro = *prologue;
-  }
+  p.row_stats = row_stats;
+  if (row_stats != nullptr && (epi != kEpiF32 || plan.splits != 1 || n_out % 32 != 0))
+    return cudaErrorInvalidValue;
   const CUtensorMap* tw2 = &tmap_w;
   const CUtensorMap* tx2 = &tmap_x;
   if (augment != nullptr && augment->k > 0) {
@@ -765,11 +680,9 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
     p.sk_part = reinterpret_cast<float*>(static_cast<uint8_t*>(sk_workspace) + kSkSyncBytes);
     grid = dim3(plan.units * per_unit, 1, 1);
   }
-  if (!plan.pair) {
-    kernel<<<grid, kThreads, plan.smem_bytes, stream>>>(tmap_w, tmap_x, *tw2, *tx2, p);
-    return cudaGetLastError();
-  }
-  if (grid.x % 2 != 0) return cudaErrorInvalidValue;
+  // cudaLaunchKernelEx returns this launch's own status (never an error
+  // left behind by an earlier call)
+  if (plan.pair && grid.x % 2 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -781,7 +694,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = plan.pair ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, tmap_w, tmap_x, *tw2, *tx2, p);
 }
 

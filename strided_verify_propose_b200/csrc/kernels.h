@@ -64,38 +64,16 @@ struct GemmAugment {
   int32_t k;
 };
 
-// A prologue that produces the GEMM's own input before its mainloop: the
-// residual add and RMSNorm of the previous projection's split-K slices,
-// x[row] += sum_s part[s][row]; hn[row] = bf16(RMSNorm(x[row]) * norm_w),
-// with hn the GEMM's X. The CTAs share the rows, arrive on cnt[0] and load
-// no token tile before every CTA has arrived, so the whole grid must be
-// resident at once (coresident: gemm_coresident_ctas of the plan). cnt[2]
-// starts at zero; each launch leaves it zero.
-struct GemmPrologue {
-  int32_t on;
-  const float* part;
-  int32_t splits;
-  int64_t split_stride;
-  float* x;
-  const float* norm_w;
-  float eps;
-  __nv_bfloat16* hn;
-  int32_t rows, hidden;
-  int32_t* cnt;
-  int32_t coresident;
-};
-// CTAs of this plan's kernel that can be resident on the device at once.
-int gemm_coresident_ctas(const GemmPlan& plan);
-
 // tmap_w: W with box_rows 128; tmap_x: X with rows = m and box_rows = plan.box_rows.
 // kEpiF32: out_f32[split][m][n_out]; kEpiSiluMul: out_act[m][n_out / 2] bf16
 // with W's rows interleaved in blocks of 16 (gate rows then up rows).
+// row_stats (kEpiF32, one slice): [m][n_out / 32] of {max, sum of
+// exp(y - max), max again, first argmax as int bits} over each 32 outputs.
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmAugment* augment = nullptr,
-                        const GemmPrologue* prologue = nullptr);
+                        const GemmAugment* augment = nullptr, float4* row_stats = nullptr);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {
@@ -122,7 +100,10 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
                              cudaEvent_t between = nullptr, const QkvReduceArgs* qkv = nullptr,
-                             int32_t* pro_cnt = nullptr);
+                             int32_t* pro_cnt = nullptr, bool prefix_early = false);
+// (prefix_early: each request's rows are one block at consecutive positions,
+// a decode step, so K/V tiles below a request's first row do not depend on
+// the prologue and may be loaded before its barrier.)
 
 // ------------------------------------------------------------------ row ops
 struct RowMeta {
@@ -198,6 +179,9 @@ struct AcceptArgs {
   int32_t* free_head;
   int32_t num_pages, max_pages_per_req, free_count;
   int32_t* status;
+  // per (row, 32-token slab) statistics of the logits from the LM head's
+  // epilogue (launch_gemm row_stats); null: computed from the logits
+  const float4* slab_stats = nullptr;
 };
 size_t accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab);
 // between[0] / between[1]: optional events recorded after the first and second kernel.

@@ -117,16 +117,18 @@ __global__ void __launch_bounds__(256)
 }
 
 // x[row] += sum_s part[s][row] (fixed order); hn[row] = bf16(RMSNorm(x[row]) * w).
-// Each thread holds up to kResIters float4 of the row, so every split's loads
-// are in flight together; the sum order (x, then splits ascending) is fixed.
+// Each thread holds up to kResIters float4 of the row and loads kBatch
+// splits of them at once (one memory round trip per kBatch splits, not per
+// split); the sum order (x, then splits ascending) is fixed. kIters float4
+// per thread cover hidden <= kIters * 1024; kMinCtas CTAs of 256 threads
+// share an SM, so a thread has 256 / kMinCtas registers: 4 CTAs when the
+// rows need them all for one wave, else 2 and a deeper batch.
 constexpr int kResThreads = 256;
 constexpr int kResIters = 8;        // hidden <= 8192
 constexpr int kResMaxSplits = 8;
 
-// (4 CTAs of 256 threads per SM: at most 64 registers per thread; kIters
-// float4 per thread cover hidden <= kIters * 1024)
-template <int kIters>
-__global__ void __launch_bounds__(kResThreads, 4)
+template <int kIters, int kBatch, int kMinCtas>
+__global__ void __launch_bounds__(kResThreads, kMinCtas)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
                          const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
   __shared__ float red[32];
@@ -140,17 +142,29 @@ __global__ void __launch_bounds__(kResThreads, 4)
     v[it] = i < hidden ? *reinterpret_cast<const float4*>(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
-  for (int s = 0; s < kResMaxSplits; ++s) {
-    if (s < splits) {
+  for (int s0 = 0; s0 < kResMaxSplits; s0 += kBatch) {
+    if (s0 < splits) {
+      float4 d[kBatch][kIters];
 #pragma unroll
-      for (int it = 0; it < kIters; ++it) {
-        const int i = (it * kResThreads + threadIdx.x) * 4;
-        if (i < hidden) {
-          const float4 d = *reinterpret_cast<const float4*>(pr + s * split_stride + i);
-          v[it].x += d.x;
-          v[it].y += d.y;
-          v[it].z += d.z;
-          v[it].w += d.w;
+      for (int u = 0; u < kBatch; ++u) {
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+          const int i = (it * kResThreads + threadIdx.x) * 4;
+          d[u][it] = s0 + u < splits && i < hidden
+                         ? *reinterpret_cast<const float4*>(pr + (s0 + u) * split_stride + i)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (s0 + u < splits) {
+#pragma unroll
+          for (int it = 0; it < kIters; ++it) {
+            v[it].x += d[u][it].x;
+            v[it].y += d[u][it].y;
+            v[it].z += d[u][it].z;
+            v[it].w += d[u][it].w;
+          }
         }
       }
     }
@@ -261,12 +275,32 @@ cudaError_t launch_residual_norm(const float* part, int32_t splits, int32_t rows
                                  cudaStream_t stream) {
   if (hidden % 4 || hidden > kResThreads * 4 * kResIters || splits < 0 || splits > kResMaxSplits)
     return cudaErrorInvalidValue;
-  if (hidden <= kResThreads * 4 * 4)
-    residual_norm_kernel<4><<<rows, kResThreads, 0, stream>>>(
-        part, splits, static_cast<int64_t>(rows) * hidden, hidden, norm_w, eps, x, hn);
-  else
-    residual_norm_kernel<kResIters><<<rows, kResThreads, 0, stream>>>(
-        part, splits, static_cast<int64_t>(rows) * hidden, hidden, norm_w, eps, x, hn);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool deep = rows <= 2 * sms;   // one wave at 2 CTAs per SM
+  const int64_t stride = static_cast<int64_t>(rows) * hidden;
+  if (hidden <= kResThreads * 4 * 4) {
+    if (deep)
+      residual_norm_kernel<4, 4, 2><<<rows, kResThreads, 0, stream>>>(part, splits, stride, hidden,
+                                                                      norm_w, eps, x, hn);
+    else
+      residual_norm_kernel<4, 2, 4><<<rows, kResThreads, 0, stream>>>(part, splits, stride, hidden,
+                                                                      norm_w, eps, x, hn);
+  } else if (hidden <= kResThreads * 4 * 5) {
+    if (deep)
+      residual_norm_kernel<5, 4, 2><<<rows, kResThreads, 0, stream>>>(part, splits, stride, hidden,
+                                                                      norm_w, eps, x, hn);
+    else
+      residual_norm_kernel<5, 1, 4><<<rows, kResThreads, 0, stream>>>(part, splits, stride, hidden,
+                                                                      norm_w, eps, x, hn);
+  } else {
+    if (deep)
+      residual_norm_kernel<kResIters, 2, 2><<<rows, kResThreads, 0, stream>>>(
+          part, splits, stride, hidden, norm_w, eps, x, hn);
+    else
+      residual_norm_kernel<kResIters, 1, 4><<<rows, kResThreads, 0, stream>>>(
+          part, splits, stride, hidden, norm_w, eps, x, hn);
+  }
   return cudaGetLastError();
 }
 
