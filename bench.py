@@ -531,11 +531,11 @@ def extra_configs(model, shape, args, seed):
     return out
 
 
-# DRAM bytes (read + write) of the step's attention launch (the tcgen05
-# kernel with its QKV-reduction prologue) per algorithmic byte, from one ncu
-# capture of the same launch in the two-layer headline workload; the
-# roofline's `traffic` scales it to this run's launch. None until captured.
-ATTN_DRAM_PER_ALGO_BYTE = None
+# DRAM bytes (read + write) of the tcgen05 attention kernel per byte of the
+# layer's K+V, from one ncu capture of the same launch in the two-layer
+# headline workload (549.9 MB for 527.9 MB of K+V; batch 64, prompts
+# U[512, 4096]); the roofline's `traffic` scales it to this run's launch.
+ATTN_DRAM_PER_KV_BYTE = 549.854 / 527.933
 
 
 def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
@@ -574,21 +574,23 @@ def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
         # one layer's K+V, averaged over the profiled steps
         kv = float(np.mean([sum(int(L) + R for L in ls) for ls in lens_steps])) * shape.kv_dim * 2 * 2
         algo = kv
-        fused = (top == "attention" and shape.head_dim == 128 and shape.page_size == 64
-                 and R * (shape.n_q_heads // shape.n_kv_heads) <= 64)
-        if fused:
-            # the launch also finishes the layer's QKV projection: its fp32
-            # output read once, q and the block's K/V rows written in bf16
+        tc = (top == "attention" and shape.head_dim == 128 and shape.page_size == 64
+              and R * (shape.n_q_heads // shape.n_kv_heads) <= 64)
+        if tc:
+            # the timed class also covers the layer's QKV reduction (the
+            # attention kernel's prologue at small batch, its own kernel just
+            # before it otherwise): the QKV projection's fp32 output read
+            # once, q and the block's K/V rows written in bf16
             algo += M * shape.qkv_dim * 4 + M * (shape.q_dim + 2 * shape.kv_dim) * 2
         achieved = algo / avg_s / 1e9
         peak = peaks["hbm"]
-        traffic = None
-        if fused and ATTN_DRAM_PER_ALGO_BYTE is not None:
-            traffic = ATTN_DRAM_PER_ALGO_BYTE * algo   # bytes per launch (scaled ncu capture)
+        traffic = ATTN_DRAM_PER_KV_BYTE * kv if tc else None
         return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": algo,
-                "traffic_note": "ncu dram read+write of one capture of the same launch, scaled "
-                                "by algorithmic bytes",
+                "kv_bytes": kv,
+                "traffic_note": "ncu dram read+write of the tcgen05 attention kernel in one "
+                                "capture of the same launch, scaled by this launch's K+V bytes "
+                                "(the QKV reduction's own traffic is not in it)",
                 "peak_kind": f"{peaks['source']} HBM copy",
                 "avg_launch_ms": avg_s * 1e3, "launches": cnt}
     return {"kernel": top, "bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s",

@@ -683,15 +683,20 @@ __host__ __device__ __forceinline__ bool tc_next(const AttnParams& p, const int*
 
 // Combine for the tcgen05 kernel's balanced ranges: (request b, KV head g)
 // has parts from CTAs c(first tile) .. c(last tile), in slots
-// (b * nkv + g) * max_parts + 0 .. parts - 1: per row the parts' softmax
-// masses give weights (once, in shared memory w), then each output is the
-// weighted sum of the parts in part order. NT threads (tid < NT) work; every
-// thread of the CTA calls it (it synchronises the CTA).
-template <int NP, int NT>
-__device__ __forceinline__ void combine_pair_tc(const AttnParams& p, const int* base, int C_grid,
-                                                int b, int g, float (*w)[kMaxSplits], int tid,
+// (b * nkv + g) * max_parts + 0 .. parts - 1. One CTA of 128 threads takes
+// kCombRows query rows q0 .. q0 + 7 of the pair: per row the parts' softmax
+// masses give weights (16 lanes per row, each over parts lane, lane + 16,
+// ...), then each output is the weighted sum of the parts in part order,
+// with kCombBatch parts' loads in flight per round trip.
+constexpr int kCombRows = 8;
+constexpr int kCombBatch = 4;
+template <int NP>
+__device__ __forceinline__ void combine_rows_tc(const AttnParams& p, const int* base, int C_grid,
+                                                int b, int g, int q0, float (*w)[kMaxSplits],
                                                 __nv_bfloat16* out) {
-  constexpr int HD = 128;
+  constexpr int HD = 128, NT = 128;
+  static_assert(NT == kCombRows * 16 && kMaxSplits == 16 * 4, "16 lanes x 4 parts per row");
+  const int tid = threadIdx.x;
   const int64_t U = tc_ubase(p, base, p.B);
   const int nt = base[b + 1] - base[b];
   int parts = 0;
@@ -705,47 +710,70 @@ __device__ __forceinline__ void combine_pair_tc(const AttnParams& p, const int* 
     parts = 0;
   }
   const int64_t slot0 = static_cast<int64_t>(b * p.nkv + g) * p.max_parts;
-  for (int qi = tid; qi < p.RG && tid < NT; qi += NT) {
-    float M = -INFINITY;
-    for (int s = 0; s < parts; ++s) M = fmaxf(M, __ldcg(&p.part_ml[(slot0 + s) * NP + qi]).x);
-    const float Rm = M == -INFINITY ? 0.f : M;
-    float L = 0.f;
-    for (int s = 0; s < parts; ++s) {
-      const float2 ml = __ldcg(&p.part_ml[(slot0 + s) * NP + qi]);
-      const float ws = ml.y * exp2f(ml.x - Rm);
-      w[qi][s] = ws;
-      L += ws;
+  {
+    const int r = tid >> 4, k = tid & 15;
+    const int qi = q0 + r;
+    float2 ml[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sp = k + 16 * u;
+      ml[u] = sp < parts && qi < p.RG ? __ldcg(&p.part_ml[(slot0 + sp) * NP + qi])
+                                      : make_float2(-INFINITY, 0.f);
     }
+    float M = fmaxf(fmaxf(ml[0].x, ml[1].x), fmaxf(ml[2].x, ml[3].x));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float Rm = M == -INFINITY ? 0.f : M;
+    float ws[4], L = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      ws[u] = k + 16 * u < parts ? ml[u].y * exp2f(ml[u].x - Rm) : 0.f;
+      L += ws[u];
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int s = 0; s < parts; ++s) w[qi][s] *= inv;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (k + 16 * u < parts) w[r][k + 16 * u] = ws[u] * inv;
   }
   __syncthreads();
-  // part-major: every load of one part is in flight at once (one L2 round
-  // trip per part); each output still sums its parts in part order
-  constexpr int kVec = NP * (HD / 4) / NT;   // float4 outputs per thread
+  constexpr int kVec = kCombRows * (HD / 4) / NT;   // float4 outputs per thread
   float4 acc[kVec];
 #pragma unroll
   for (int j = 0; j < kVec; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < parts; ++s) {
+  for (int s0 = 0; s0 < parts; s0 += kCombBatch) {
+    float4 v[kCombBatch][kVec];
 #pragma unroll
-    for (int j = 0; j < kVec; ++j) {
-      const int i = tid + j * NT;
-      if (tid < NT && i < p.RG * (HD / 4)) {
-        const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
-        const float ws = w[qi][s];
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((slot0 + s) * NP + qi) * HD + d));
-        acc[j].x += ws * v.x;
-        acc[j].y += ws * v.y;
-        acc[j].z += ws * v.z;
-        acc[j].w += ws * v.w;
+    for (int u = 0; u < kCombBatch; ++u) {
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) {
+        const int i = tid + j * NT;
+        const int qi = q0 + i / (HD / 4), d = (i % (HD / 4)) * 4;
+        v[u][j] = s0 + u < parts && qi < p.RG
+                      ? __ldcg(reinterpret_cast<const float4*>(p.part_o + ((slot0 + s0 + u) * NP + qi) * HD + d))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCombBatch; ++u) {
+      if (s0 + u < parts) {
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+          const float wsu = w[(tid + j * NT) / (HD / 4)][s0 + u];
+          acc[j].x += wsu * v[u][j].x;
+          acc[j].y += wsu * v[u][j].y;
+          acc[j].z += wsu * v[u][j].z;
+          acc[j].w += wsu * v[u][j].w;
+        }
       }
     }
   }
 #pragma unroll
   for (int j = 0; j < kVec; ++j) {
     const int i = tid + j * NT;
-    if (tid < NT && i < p.RG * (HD / 4)) {
-      const int qi = i / (HD / 4), d = (i % (HD / 4)) * 4;
+    const int qi = q0 + i / (HD / 4), d = (i % (HD / 4)) * 4;
+    if (qi < p.RG) {
       const int r = qi / p.G, h = qi % p.G;
       __align__(8) __nv_bfloat16 o4[4] = {__float2bfloat16_rn(acc[j].x), __float2bfloat16_rn(acc[j].y),
                                           __float2bfloat16_rn(acc[j].z), __float2bfloat16_rn(acc[j].w)};
@@ -753,7 +781,6 @@ __device__ __forceinline__ void combine_pair_tc(const AttnParams& p, const int* 
           *reinterpret_cast<const uint2*>(o4);
     }
   }
-  __syncthreads();   // w is rewritten by the next pair
 }
 
 template <int NP>
@@ -1327,15 +1354,15 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p, _
   }
 }
 
-// The tcgen05 kernel's (request, KV head) pairs, one CTA per pair. (Merging
-// them at the end of the attention kernel itself, after a barrier over its
-// grid, measured 0.19 ms per step slower: the 148 CTAs merge 512 pairs
-// where this kernel spreads them over 512 CTAs.)
+// The tcgen05 kernel's (request, KV head) pairs: grid (KV head, request,
+// groups of kCombRows query rows). (Merging them at the end of the
+// attention kernel itself, after a barrier over its grid, measured 0.19 ms
+// per step slower: 148 CTAs merged 512 pairs.)
 template <int NP>
 __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p, int C_grid,
                                                               __nv_bfloat16* out) {
-  __shared__ float w[NP][kMaxSplits];
-  combine_pair_tc<NP, 128>(p, p.item_base, C_grid, blockIdx.y, blockIdx.x, w, threadIdx.x, out);
+  __shared__ float w[kCombRows][kMaxSplits];
+  combine_rows_tc<NP>(p, p.item_base, C_grid, blockIdx.y, blockIdx.x, blockIdx.z * kCombRows, w, out);
 }
 
 struct Derived {
@@ -1581,10 +1608,11 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                                       : cudaLaunchKernelEx(&cfg, attn_tc_kernel<64>, k_map, v_map, qmap, p);
     if (le != cudaSuccess) return le;   // the combine reads what this kernel writes
     if (between) cudaEventRecord(between, stream);
+    const dim3 cgrid(s.n_kv_heads, s.batch, (d.RG + kCombRows - 1) / kCombRows);
     if (d.np == 32)
-      attn_combine_tc_kernel<32><<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
+      attn_combine_tc_kernel<32><<<cgrid, 128, 0, stream>>>(p, sms, out);
     else
-      attn_combine_tc_kernel<64><<<dim3(s.n_kv_heads, s.batch), 128, 0, stream>>>(p, sms, out);
+      attn_combine_tc_kernel<64><<<cgrid, 128, 0, stream>>>(p, sms, out);
     if (launches) *launches += 2;
     return cudaGetLastError();
   }

@@ -582,11 +582,9 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
       kStageA + static_cast<size_t>(best.n_boxes) * static_cast<size_t>(best.box_rows) * 128;
   const size_t extra = 1024 + 256;
   int stages = static_cast<int>((kMaxSmem - extra) / stage);
-  // few tokens (decode at small batch): a K-block is nearly all weights and
-  // the ring is what keeps HBM busy, so it takes all the shared memory, up to
-  // the 12 slots whose barriers fit the 256 bytes after the ring
-  // ((2 x 12 + 2) x 8 + 8 bytes)
-  stages = std::min(stages, 12);
+  // (12 slots for the few-token plans of batch-1 decode measured the same
+  // step time as 8)
+  stages = std::min(stages, 8);
   if (!best.streamk) stages = std::min(stages, std::max(best.kb_per_split, 2));
   best.stages = std::max(stages, 2);
   best.tmem_cols = pow2_at_least(static_cast<uint32_t>(best.n_pad));
