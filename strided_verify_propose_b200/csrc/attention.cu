@@ -1362,6 +1362,7 @@ template <int NP>
 __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const AttnParams p, int C_grid,
                                                               __nv_bfloat16* out) {
   __shared__ float w[kCombRows][kMaxSplits];
+  griddep_launch_dependents();   // the O projection may load its weights meanwhile
   combine_rows_tc<NP>(p, p.item_base, C_grid, blockIdx.y, blockIdx.x, blockIdx.z * kCombRows, w, out);
 }
 

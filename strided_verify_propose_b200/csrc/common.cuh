@@ -30,6 +30,18 @@ __device__ __forceinline__ void flag(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialisation may start before the kernel ahead of it in the stream has
+// finished; griddep_wait() returns once that kernel has completed and its
+// memory operations are visible, so every read of its output, and every
+// write to memory it may still read, comes after it. griddep_launch_dependents()
+// lets such a dependent kernel begin launching (without it, a CTA counts once
+// it exits); neither has an effect on kernels launched the ordinary way.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -129,6 +129,9 @@ struct isd_ctx {
   CUtensorMap tm_lm{};
   int32_t qkv_dim = 0, q_dim = 0;
   int32_t max_splits = 8;
+  // GEMMs launched with programmatic stream serialisation: each loads its
+  // first ring of weight tiles while the kernel ahead of it finishes
+  bool pdl = true;
 
   // workspace (the library's only allocation)
   void* ws = nullptr;
@@ -304,7 +307,7 @@ int gemm(isd_ctx* c, int cls, const CUtensorMap& tw, const __nv_bfloat16* x, int
   }
   cudaEvent_t e0 = prof_mark(c, st);
   ISD_CUDA(isd::launch_gemm(tw, *tx, plan, m, n, k, epi, out, act, status, st, c->sk_ws,
-                            c->sk_ws_bytes, aug ? &ga : nullptr, row_stats));
+                            c->sk_ws_bytes, aug ? &ga : nullptr, row_stats, c->pdl));
   prof_add(c, cls, e0, prof_mark(c, st));
   if (splits_used) *splits_used = plan.splits;
   c->launches += 1;

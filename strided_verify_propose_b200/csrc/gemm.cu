@@ -65,6 +65,9 @@ struct GemmParams {
   // kEpiF32 with one slice: per (token, 32-row slab) max, sum of exp(y - max)
   // and first argmax of the finished result, [m][n_out / 32]
   float4* row_stats;
+  // launched with programmatic stream serialisation: the producer loads the
+  // first ring of weight tiles, then waits for the kernel ahead of it
+  int32_t pdl;
 };
 
 // For each of the 32 values a lane holds (value j of every lane is token j;
@@ -235,11 +238,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     int issued = 0;
     bool ok = true;
     Segment sg;
+    // With programmatic launch, the weight tiles of the first p.stages
+    // iterations are loaded before the wait for the kernel ahead (they do
+    // not depend on it; the fresh ring needs no empty wait); the main pass
+    // then adds only their token tiles. `pre` counts those iterations.
+    int pre = 0;
+    if (p.pdl) {
+      int s0 = 0;
+      for (int idx = 0; pre < p.stages && get_segment<kPair>(p, idx, sg); ++idx) {
+        const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
+        const int n_base = sg.kb_hi - sg.kb_lo;
+        for (int i = 0; i < n_base + sg.aug && pre < p.stages; ++i, ++pre, ++s0) {
+          uint8_t* sa = smem + s0 * stage_bytes;
+          const bool aug = i >= n_base;
+          const int kc = (aug ? i - n_base : sg.kb_lo + i) * kTileK;
+          const CUtensorMap* mw = aug ? &tmap_w2 : &tmap_w;
+          if (kPair) {
+            const uint32_t bar = map_to_rank(smem_u32(&full[s0]), 0);
+            if (leader) mbar_arrive_expect_tx(&full[s0], tx);
+            tma_load_2d_pair(sa, mw, bar, kc, mt * kTileM, pol_w);
+          } else {
+            mbar_arrive_expect_tx(&full[s0], tx);
+            tma_load_2d_hint(sa, mw, &full[s0], kc, mt * kTileM, pol_w);
+          }
+        }
+      }
+      griddep_wait();
+    }
     for (int idx = 0; ok && get_segment<kPair>(p, idx, sg); ++idx) {
       const int mt = kPair ? sg.ut * 2 + static_cast<int>(rank) : sg.ut;
       const int n_base = sg.kb_hi - sg.kb_lo;
       for (int i = 0; i < n_base + sg.aug; ++i) {
-        if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
+        const bool w_done = issued < pre;   // weights already on their way
+        if (!w_done && (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag)) {
           flag(p.status, ISD_DEV_TIMEOUT);
           *abort_flag = 1;
           ok = false;
@@ -253,14 +284,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* mx = aug ? &tmap_x2 : &tmap_x;
         if (kPair) {
           const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d_pair(sa, mw, bar, kc, mt * kTileM, pol_w);
+          if (!w_done) {
+            if (leader) mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_2d_pair(sa, mw, bar, kc, mt * kTileM, pol_w);
+          }
           for (int bx = 0; bx < p.n_boxes; ++bx)
             tma_load_2d_pair(sb + bx * p.box_rows * 128, mx, bar, kc,
                              tok0 + bx * p.mma_n + static_cast<int>(rank) * p.box_rows, pol_x);
         } else {
-          mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d_hint(sa, mw, &full[s], kc, mt * kTileM, pol_w);
+          if (!w_done) {
+            mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_2d_hint(sa, mw, &full[s], kc, mt * kTileM, pol_w);
+          }
           for (int bx = 0; bx < p.n_boxes; ++bx)
             tma_load_2d_hint(sb + bx * p.box_rows * 128, mx, &full[s], kc,
                              tok0 + bx * p.box_rows, pol_x);
@@ -613,7 +648,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace, size_t sk_workspace_bytes,
-                        const GemmAugment* augment, float4* row_stats) {
+                        const GemmAugment* augment, float4* row_stats, bool pdl) {
   auto kernel = plan.pair
                     ? (plan.n_mma == 2 ? gemm_bf16_tcgen05<true, 2> : gemm_bf16_tcgen05<true, 1>)
                     : (plan.n_mma == 2 ? gemm_bf16_tcgen05<false, 2> : gemm_bf16_tcgen05<false, 1>);
@@ -652,6 +687,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   p.sk_sync = nullptr;
   p.aug_kb = 0;
   p.row_stats = row_stats;
+  p.pdl = pdl ? 1 : 0;
   if (row_stats != nullptr && (epi != kEpiF32 || plan.splits != 1 || n_out % 32 != 0))
     return cudaErrorInvalidValue;
   const CUtensorMap* tw2 = &tmap_w;
@@ -686,13 +722,22 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, co
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = plan.smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (plan.pair) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = plan.pair ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kernel, tmap_w, tmap_x, *tw2, *tx2, p);
 }
 

@@ -69,11 +69,14 @@ struct GemmAugment {
 // with W's rows interleaved in blocks of 16 (gate rows then up rows).
 // row_stats (kEpiF32, one slice): [m][n_out / 32] of {max, sum of
 // exp(y - max), max again, first argmax as int bits} over each 32 outputs.
+// pdl: launch with programmatic stream serialisation (the first ring of
+// weight tiles loads while the kernel ahead in the stream finishes).
 cudaError_t launch_gemm(const CUtensorMap& tmap_w, const CUtensorMap& tmap_x, const GemmPlan& plan,
                         int32_t m, int32_t n_out, int32_t k, GemmEpilogue epi, float* out_f32,
                         __nv_bfloat16* out_act, int32_t* status, cudaStream_t stream,
                         void* sk_workspace = nullptr, size_t sk_workspace_bytes = 0,
-                        const GemmAugment* augment = nullptr, float4* row_stats = nullptr);
+                        const GemmAugment* augment = nullptr, float4* row_stats = nullptr,
+                        bool pdl = false);
 
 // ----------------------------------------------------------------- attention
 struct AttnShape {

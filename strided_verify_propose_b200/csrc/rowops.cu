@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(256)
     embed_norm_kernel(const __nv_bfloat16* embed, const float* norm_w, RowMeta meta, int32_t hidden,
                       int32_t vocab, float eps, float* x, __nv_bfloat16* hn, int32_t* status) {
   __shared__ float red[32];
+  griddep_launch_dependents();   // the next GEMM may load its weights meanwhile
   const int row = blockIdx.x;
   int tok = meta.tok[row];
   if (tok < 0 || tok >= vocab) {
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(kResThreads, kMinCtas)
     residual_norm_kernel(const float* part, int32_t splits, int64_t split_stride, int32_t hidden,
                          const float* norm_w, float eps, float* x, __nv_bfloat16* hn) {
   __shared__ float red[32];
+  griddep_launch_dependents();   // the next GEMM may load its weights meanwhile
   const int row = blockIdx.x;
   float* xr = x + static_cast<int64_t>(row) * hidden;
   const float* pr = part + static_cast<int64_t>(row) * hidden;
