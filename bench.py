@@ -291,18 +291,21 @@ def run_cuda(args, ws, rank, local):
         raise RuntimeError(f"step status {int(st.status.item())}")
 
     # ---- the same number of steps launched one by one
-    eager_ms, eager_committed = None, 0
+    eager_ms, eager_committed, step_ms = None, 0, None
     if not args.no_graph:
-        h_start, h_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # an event between consecutive steps: the per-step spread
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        h_start, h_stop = marks[0], marks[-1]
         eager_hist = torch.zeros(args.steps, B, device="cuda", dtype=torch.int32)
         torch.cuda.synchronize()
         h_start.record(stream)
         for i in range(args.steps):
             one(unif_d[step_i]); step_i += 1
             eager_hist[i].copy_(st.accepted)
-        h_stop.record(stream)
+            marks[i + 1].record(stream)
         torch.cuda.synchronize()
         eager_ms = h_start.elapsed_time(h_stop)
+        step_ms = np.array([marks[i].elapsed_time(marks[i + 1]) for i in range(args.steps)])
         eager_committed = int((eager_hist.long() + 1).sum().item())
 
     lens_after_timed = st.seq_len.cpu().numpy().copy()   # (after the eager steps too)
@@ -422,7 +425,9 @@ def run_cuda(args, ws, rank, local):
             "eager": None if eager_ms is None else {
                 "value": eager_committed / (eager_ms_all * 1e-3), "unit": "tokens/s",
                 "ms_per_step": eager_ms_all / args.steps,
-                "note": "the same number of steps launched one by one"},
+                "step_ms_p10_median_p90": [round(float(np.percentile(step_ms, q)), 4)
+                                           for q in (10, 50, 90)],
+                "note": "the same number of steps launched one by one (per-step spread on rank 0)"},
             "prefill_s": t_prefill, "setup_s": t_setup,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,

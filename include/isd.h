@@ -298,9 +298,10 @@ int isd_accept_propose(const float *logits_dev, const isd_batch *batch, const is
  * its own). The paper has no counterpart: this is a deployment variant.
  * Scratch comes from a 4 MiB array compiled into the library, present on
  * every GPU that loads it until the process exits; a call needs
- * batch * (2N-1) * ceil(vocab/8192) * 16 bytes of it (at most 4 MiB, e.g.
- * batch <= 1024 at N = 4 and vocab 151936) and returns ISD_E_UNSUPPORTED
- * above that. The first call on each device looks up the array's device
+ * isd_accept_workspace_bytes(batch, N, vocab) bytes of it (the chunk
+ * statistics, batch * (2N-1) * ceil(vocab/8192) * 16 bytes, then 4 bytes
+ * per request; at most 4 MiB, e.g. batch <= 1024 at N = 4 and vocab 151936)
+ * and returns ISD_E_UNSUPPORTED above that. The first call on each device looks up the array's device
  * address with that device current. Under CUDA's lazy module loading (the
  * default) that lookup is also what loads this part of the library onto the
  * device and places the array there, so the first call on a device does

@@ -19,7 +19,8 @@
 //  2. accept_decide: one CTA per request: combines the chunk statistics,
 //     runs the sequential accept tests, draws the new token by inverse CDF
 //     (chunk totals first, then a block scan inside one chunk) and reads or
-//     samples the proposals.
+//     samples the proposals; in SAMPLE mode write_q_rows then stores the
+//     proposals' q rows with one CTA per 8192-token chunk.
 //  3. bookkeep: one CTA: lengths += 1 + A; pages for the next block from
 //     the free list by an exclusive prefix sum in request order.
 #include <float.h>
@@ -161,6 +162,30 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// One row's max, sum of exp(z - max) and first argmax from its chunk
+// statistics, by one warp (lane-strided, then a butterfly); every caller
+// merges in this order, so all of them get the same bits.
+__device__ __forceinline__ void row_stats(const ChunkStat* st, int n_chunks, int lane, float& m,
+                                          float& s, int& ai) {
+  m = -INFINITY;
+  s = 0.f;
+  float av = -INFINITY;
+  ai = INT_MAX;
+  for (int c = lane; c < n_chunks; c += 32) {
+    merge_ms(m, s, st[c].m, st[c].s);
+    merge_arg(av, ai, st[c].amax, st[c].idx);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float v2 = __shfl_xor_sync(0xffffffffu, av, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, ai, o);
+    merge_ms(m, s, m2, s2);
+    merge_arg(av, ai, v2, i2);
+  }
+}
+
 // Block-wide inclusive scan of one float per thread (kThreads threads).
 __device__ float block_incl_scan(float v, float* warp_tot) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -278,7 +303,7 @@ __device__ int sample_row(const Weights& wf, int vocab, int n_chunks, float u, D
 
 __global__ void __launch_bounds__(kThreads) accept_decide_kernel(const AcceptArgs a,
                                                                  const ChunkStat* stats,
-                                                                 int32_t n_chunks) {
+                                                                 int32_t n_chunks, int32_t* qsrc) {
   __shared__ DecideShared sh;
   const int b = blockIdx.x;
   const int N = a.stride_n, R = 2 * N - 1;
@@ -294,22 +319,9 @@ __global__ void __launch_bounds__(kThreads) accept_decide_kernel(const AcceptArg
   {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int r = w; r < R; r += kThreads / 32) {
-      const ChunkStat* st = stats + (static_cast<int64_t>(b) * R + r) * n_chunks;
-      float m = -INFINITY, s = 0.f, av = -INFINITY;
-      int ai = INT_MAX;
-      for (int c = lane; c < n_chunks; c += 32) {
-        merge_ms(m, s, st[c].m, st[c].s);
-        merge_arg(av, ai, st[c].amax, st[c].idx);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        const float v2 = __shfl_xor_sync(0xffffffffu, av, o);
-        const int i2 = __shfl_xor_sync(0xffffffffu, ai, o);
-        merge_ms(m, s, m2, s2);
-        merge_arg(av, ai, v2, i2);
-      }
+      float m, s;
+      int ai;
+      row_stats(stats + (static_cast<int64_t>(b) * R + r) * n_chunks, n_chunks, lane, m, s, ai);
       if (lane == 0) {
         sh.M[r] = m;
         sh.S[r] = s;
@@ -407,11 +419,11 @@ __global__ void __launch_bounds__(kThreads) accept_decide_kernel(const AcceptArg
       if (!propose_sample) {
         if (threadIdx.x == 0) sh.props[i] = sh.amax[r];
       } else {
+        // (the q row itself is written by write_q_rows_kernel, over the
+        // whole device, once this kernel has read the previous q rows)
         const int row = b * R + r;
         const float* z = a.logits + static_cast<int64_t>(row) * V;
         const float M = sh.M[r], inv_S = 1.f / sh.S[r];
-        float* qo = a.q_cache + (static_cast<int64_t>(b) * (N - 1) + i - 1) * V;
-        for (int t = threadIdx.x; t < V; t += kThreads) qo[t] = expf(z[t] - M) * inv_S;
         const ChunkStat* st = stats + static_cast<int64_t>(row) * n_chunks;
         if (threadIdx.x < n_chunks) sh.W[threadIdx.x] = st[threadIdx.x].s * expf(st[threadIdx.x].m - M);
         __syncthreads();
@@ -425,6 +437,7 @@ __global__ void __launch_bounds__(kThreads) accept_decide_kernel(const AcceptArg
   __syncthreads();
 
   if (threadIdx.x == 0) {
+    if (propose_sample) qsrc[b] = A == n ? n : -1;
     a.accepted[b] = A;
     if (a.committed) {
       int32_t* cm = a.committed + static_cast<int64_t>(b) * N;
@@ -434,6 +447,51 @@ __global__ void __launch_bounds__(kThreads) accept_decide_kernel(const AcceptArg
     pw[0] = new_tok;
     for (int i = 1; i < N; ++i) pw[i] = (A == n) ? sh.props[i] : -1;
     a.n_draft[b] = (A == n) ? N - 1 : 0;
+  }
+}
+
+// SAMPLE mode: the proposal rows' q' = softmax(z), one CTA per (8192-token
+// chunk, request, proposal i), for the requests whose proposals stand
+// (qsrc[b] = n >= 0: rows n + 1 .. n + N - 1). q = exp(z - M) * (1 / S)
+// with the row's M and S merged exactly as the decide kernel merges them.
+// Every load of a thread is issued before its arithmetic.
+__global__ void __launch_bounds__(kThreads)
+    write_q_rows_kernel(const AcceptArgs a, const ChunkStat* stats, int32_t n_chunks,
+                        const int32_t* qsrc) {
+  constexpr int kVec = kChunk / (kThreads * 4);
+  __shared__ float ms[2];
+  const int c = blockIdx.x, b = blockIdx.y, i = blockIdx.z + 1;
+  const int N = a.stride_n, R = 2 * N - 1, V = a.vocab;
+  const int n = qsrc[b];
+  if (n < 0) return;
+  const int row = b * R + n + i;
+  if (threadIdx.x < 32) {
+    float m, s;
+    int ai;
+    row_stats(stats + static_cast<int64_t>(row) * n_chunks, n_chunks, threadIdx.x, m, s, ai);
+    if (threadIdx.x == 0) {
+      ms[0] = m;
+      ms[1] = s;
+    }
+  }
+  __syncthreads();
+  const float M = ms[0], inv_S = 1.f / ms[1];
+  const float* z = a.logits + static_cast<int64_t>(row) * V;
+  float* qo = a.q_cache + (static_cast<int64_t>(b) * (N - 1) + i - 1) * V;
+  const int lo = c * kChunk, hi = min(V, lo + kChunk);
+  float4 v4[kVec];
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int t = lo + (j * kThreads + threadIdx.x) * 4;
+    v4[j] = t < hi ? *reinterpret_cast<const float4*>(z + t) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < kVec; ++j) {
+    const int t = lo + (j * kThreads + threadIdx.x) * 4;
+    if (t < hi)
+      *reinterpret_cast<float4*>(qo + t) =
+          make_float4(expf(v4[j].x - M) * inv_S, expf(v4[j].y - M) * inv_S,
+                      expf(v4[j].z - M) * inv_S, expf(v4[j].w - M) * inv_S);
   }
 }
 
@@ -493,9 +551,15 @@ __global__ void __launch_bounds__(1024) bookkeep_kernel(const AcceptArgs a) {
 
 }  // namespace
 
-size_t accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab) {
+// Workspace: the chunk statistics, then (256-byte aligned) qsrc[batch].
+static size_t stats_bytes(int32_t batch, int32_t stride_n, int32_t vocab) {
   const int n_chunks = (vocab + kChunk - 1) / kChunk;
-  return static_cast<size_t>(batch) * (2 * stride_n - 1) * n_chunks * sizeof(ChunkStat) + 256;
+  const size_t b = static_cast<size_t>(batch) * (2 * stride_n - 1) * n_chunks * sizeof(ChunkStat);
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+
+size_t accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab) {
+  return stats_bytes(batch, stride_n, vocab) + static_cast<size_t>(batch) * sizeof(int32_t) + 256;
 }
 
 cudaError_t launch_accept(const AcceptArgs& a, void* workspace, cudaStream_t stream, int* launches,
@@ -514,12 +578,21 @@ cudaError_t launch_accept(const AcceptArgs& a, void* workspace, cudaStream_t str
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;   // each kernel reads what the previous one wrote
   if (between0) cudaEventRecord(between0, stream);
-  accept_decide_kernel<<<a.batch, kThreads, 0, stream>>>(a, stats, n_chunks);
+  int32_t* qsrc = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                             stats_bytes(a.batch, a.stride_n, a.vocab));
+  accept_decide_kernel<<<a.batch, kThreads, 0, stream>>>(a, stats, n_chunks, qsrc);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  const bool q_rows = (a.flags & ISD_PROPOSE_SAMPLE) && a.q_cache != nullptr && a.stride_n > 1;
+  if (q_rows) {
+    write_q_rows_kernel<<<dim3(n_chunks, a.batch, a.stride_n - 1), kThreads, 0, stream>>>(
+        a, stats, n_chunks, qsrc);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (between1) cudaEventRecord(between1, stream);
   bookkeep_kernel<<<1, 1024, 0, stream>>>(a);
-  if (launches) *launches += 3;
+  if (launches) *launches += q_rows ? 4 : 3;
   return cudaGetLastError();
 }
 

@@ -83,7 +83,8 @@ extern "C" int isd_accept_propose_noalloc(const float* logits_dev, const isd_bat
     const std::string msg = "isd_accept_propose_noalloc: this batch needs " + std::to_string(need) +
                             " bytes of scratch but the fixed array holds " +
                             std::to_string(kScratchBytes) +
-                            " (batch * (2N-1) * ceil(vocab/8192) * 16 bytes); use isd_accept_propose";
+                            " (batch * (2N-1) * ceil(vocab/8192) * 16 bytes of chunk statistics"
+                            " and 4 bytes per request); use isd_accept_propose";
     return isd::set_error(ISD_E_UNSUPPORTED, msg.c_str());
   }
   void* scratch = nullptr;

@@ -59,8 +59,13 @@ struct AttnParams {
   int32_t* pro_cnt;            // [2] arrivals / departures (zero between launches)
   // rows of a request hold one block at consecutive positions (a decode
   // step): K/V tiles of keys below its first row are not written by the
-  // prologue and may be loaded before the barrier
+  // QKV reduction and may be loaded before waiting for it
   int32_t prefix_early;
+  // launched with programmatic stream serialisation right after the kernel
+  // that writes q and the block's K/V rows (the QKV reduction, or the QKV
+  // projection when the reduction is the prologue): nothing it writes is
+  // read before griddep_wait()
+  int32_t pdl;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -859,6 +864,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
   }
   build_items(p, kend, base);     // ends with __syncthreads
+  if (p.pdl && p.qkv_on) griddep_wait();   // the prologue reads the QKV projection
   if (p.qkv_on) {
     // this layer's QKV reduction, (row, head) items spread over every warp of
     // the grid, four per warp at a time with all their loads in flight; the
@@ -939,10 +945,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       TcRange rg = tc_range(p, base, gridDim.x, blockIdx.x);
       TcSeg sg;
       bool have = tc_next(p, base, rg, sg);
-      int pre = 0;   // tiles of the first segment loaded before the prologue's barrier
-      if (p.qkv_on) {
+      int pre = 0;   // tiles of the first segment loaded before the wait for q and K/V
+      if (p.qkv_on || p.pdl) {
         if (have && p.prefix_early) {
-          // prefix keys only: the block's own rows are the prologue's output
+          // prefix keys only: the block's own rows are the QKV reduction's output
           const int k_lo = sg.t0 * kTcKeys;
           const int k_hi = min(kend[sg.b], k_lo + sg.len * kTcKeys);
           const int prefix_end = kend[sg.b] - p.R;
@@ -952,19 +958,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ++pre;
           }
         }
-        const int total = static_cast<int>(gridDim.x);
-        const long long t0 = clock64();
-        const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
-        while (ok && ld_acquire_gpu(&p.pro_cnt[0]) < total) {
-          if (clock64() - t0 > limit) {
-            ok = false;
-            break;
+        if (p.qkv_on) {
+          const int total = static_cast<int>(gridDim.x);
+          const long long t0 = clock64();
+          const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
+          while (ok && ld_acquire_gpu(&p.pro_cnt[0]) < total) {
+            if (clock64() - t0 > limit) {
+              ok = false;
+              break;
+            }
           }
-        }
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        if (atomicAdd(&p.pro_cnt[1], 1) == total - 1) {
-          p.pro_cnt[0] = 0;
-          p.pro_cnt[1] = 0;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          if (atomicAdd(&p.pro_cnt[1], 1) == total - 1) {
+            p.pro_cnt[0] = 0;
+            p.pro_cnt[1] = 0;
+          }
+        } else {
+          griddep_wait();   // the QKV reduction ahead in the stream has finished
         }
       }
       for (; ok && have; have = tc_next(p, base, rg, sg), ++it) {
@@ -1500,7 +1510,7 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
                              cudaEvent_t between, const QkvReduceArgs* qkv, int32_t* pro_cnt,
-                             bool prefix_early) {
+                             bool prefix_early, bool pdl) {
   if (s.batch > kMaxBatch) return cudaErrorInvalidValue;
   const Derived d = derive(s);
   int sms = 148;
@@ -1564,6 +1574,9 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
   }
   p.pro_cnt = pro_cnt;
   p.prefix_early = prefix_early ? 1 : 0;
+  // programmatic launch only after a kernel that writes q and K/V: the QKV
+  // reduction launched just above, or (fused) the QKV projection
+  p.pdl = pdl && qkv != nullptr && d.tc ? 1 : 0;
   static bool attr_set = false;
   if (!attr_set) {
     // dynamic + static shared memory of each CTA within its share of the SM
@@ -1605,6 +1618,11 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = d.smem;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.pdl ? 1 : 0;
     const cudaError_t le = d.np == 32 ? cudaLaunchKernelEx(&cfg, attn_tc_kernel<32>, k_map, v_map, qmap, p)
                                       : cudaLaunchKernelEx(&cfg, attn_tc_kernel<64>, k_map, v_map, qmap, p);
     if (le != cudaSuccess) return le;   // the combine reads what this kernel writes

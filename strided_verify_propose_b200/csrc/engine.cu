@@ -129,8 +129,9 @@ struct isd_ctx {
   CUtensorMap tm_lm{};
   int32_t qkv_dim = 0, q_dim = 0;
   int32_t max_splits = 8;
-  // GEMMs launched with programmatic stream serialisation: each loads its
-  // first ring of weight tiles while the kernel ahead of it finishes
+  // GEMMs (and the tcgen05 attention) launched with programmatic stream
+  // serialisation: each loads what does not depend on the kernel ahead of
+  // it (weight tiles; K/V tiles of earlier steps) while that kernel finishes
   bool pdl = true;
 
   // workspace (the library's only allocation)
@@ -478,7 +479,8 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid, &qa,
                                    c->pro_cnt, attn_sub == 1 && ash_table == kv->page_table_dev &&
-                                                        rows_per_req == ash.rows_per_req));
+                                                        rows_per_req == ash.rows_per_req,
+                                   c->pdl));
     cudaEvent_t a2 = prof_mark(c, st);
     prof_add(c, kPAttnSplit, a1, amid);
     prof_add(c, kPAttnCombine, amid, a2);

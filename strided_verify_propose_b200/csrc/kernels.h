@@ -103,10 +103,14 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
                              cudaEvent_t between = nullptr, const QkvReduceArgs* qkv = nullptr,
-                             int32_t* pro_cnt = nullptr, bool prefix_early = false);
+                             int32_t* pro_cnt = nullptr, bool prefix_early = false,
+                             bool pdl = false);
 // (prefix_early: each request's rows are one block at consecutive positions,
 // a decode step, so K/V tiles below a request's first row do not depend on
-// the prologue and may be loaded before its barrier.)
+// the QKV reduction and may be loaded before waiting for it. pdl: the
+// tcgen05 kernel is launched with programmatic stream serialisation, which
+// is correct only when the kernel ahead of it in the stream is the QKV
+// reduction this call launches or the QKV projection feeding its prologue.)
 
 // ------------------------------------------------------------------ row ops
 struct RowMeta {

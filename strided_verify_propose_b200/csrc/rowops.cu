@@ -207,6 +207,7 @@ constexpr int kQkvMaxSplits = 8;
 template <int HD>
 // (4 CTAs of 512 threads per SM: at most 32 registers per thread)
 __global__ void __launch_bounds__(kQkvWarps * 32, 4) qkv_reduce_kernel(const QkvReduceArgs a) {
+  griddep_launch_dependents();   // the attention may load earlier steps' K/V meanwhile
   const int row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hd = blockIdx.y * kQkvWarps + warp;
