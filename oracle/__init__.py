@@ -27,7 +27,9 @@ implementation (HF transformers) on tiny shapes; the accept / resample rule by
 exact enumeration; the ISD layout by the pages' TPF formula, the TPF and
 efficiency values the pages print, and brute-force trajectory distributions;
 the gated LoRA by bitwise base-only verify rows and by a merged-weight model
-on the MASK rows; page bookkeeping by brute-force invariants. Parity
-unpinned: which MASK row proposes which draft position (reading R4 of
-isd.py), which no distribution-level test can see.
+on the MASK rows; page bookkeeping by brute-force invariants; which MASK
+row proposes which draft position (reading R4 of isd.py), which no
+distribution-level test can see, by a predictor that is perfect for a token
+sequence: every draft accepted, tokens per forward N as the pages' formula
+gives at acceptance 1.
 """

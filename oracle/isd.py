@@ -33,10 +33,11 @@ R3 the one new final token comes from row A (A = number of accepted drafts):
 R4 proposals: rows n+1..n+N-1 (the MASK rows after the bonus slot) give the
    next drafts, valid only when no draft was rejected; after a rejection the
    next step is a restart step (n = 0) whose padding rows are ignored.
-   Which MASK row proposes which position is parity unpinned: the acceptance
-   rule keeps the AR distribution for any proposal, so no distribution-level
-   pin can see the choice (the GPU parity tests compare it with this
-   reading, which is not the same as a pin to the pages).
+   The acceptance rule keeps the AR distribution for any proposal, so no
+   distribution-level pin can see which MASK row proposes which position;
+   it is pinned instead by a predictor that is perfect for a token sequence:
+   every proposal must then be the sequence's next token and be accepted,
+   giving N tokens per forward, the pages' formula at acceptance 1.
 R5 commit: seq_len += 1 + A (x* and the accepted drafts); committed tokens
    this step = accepted drafts + the new token.
 R6 sampling: inverse CDF in ascending token order: the smallest i whose

@@ -318,3 +318,69 @@ def test_isd_trajectory_distribution_equals_ar(N, propose, K):
     keys = set(isd) | set(ar)
     err = max(abs(isd.get(k, 0.0) - ar.get(k, 0.0)) for k in keys)
     assert err < 1e-12
+
+
+def _perfect_predictor_run(monkeypatch, N, shift=0, steps=12, seed=3):
+    """Whole oracle steps (greedy verification, argmax proposals) with the
+    block logits replaced by those of a predictor that is perfect for a fixed
+    token sequence: the row at position t scores seq[t + 1] (the logit shift).
+    shift != 0 plants a mistake: the proposals are read from the MASK rows
+    `shift` places off. Returns the accepted counts and the committed tokens."""
+    shape = synth.TINY
+    dec = om.Decoder(shape, synth.decoder_weights(shape, seed=seed))
+    rng = np.random.default_rng(seed)
+    seq = rng.integers(0, shape.mask_token_id, 64 + steps * (2 * N + 2))
+    real_logits, real_decide = oi.step_logits, oi.decide
+
+    def logits_fn(m, st, n_stride, lora=False):
+        logits, bk, bv = real_logits(m, st, n_stride, lora)
+        R = 2 * n_stride - 1
+        z = np.zeros_like(logits)
+        z[np.arange(R), seq[st.seq_len + 1 + np.arange(R)]] = 10.0
+        return z, bk, bv
+
+    def decide_fn(logits, drafts, q_rows, n_stride, u, propose=oi.ARGMAX, verify=oi.STOCHASTIC):
+        d = real_decide(logits, drafts, q_rows, n_stride, u, propose, verify)
+        if shift and d.proposals:
+            n = len(drafts)
+            d.proposals = [oi.argmax_lowest(logits[n + i + shift]) for i in range(1, n_stride)]
+        return d
+
+    monkeypatch.setattr(oi, "step_logits", logits_fn)
+    monkeypatch.setattr(oi, "decide", decide_fn)
+    prompt = seq[:20]
+    st = oi.start_state(dec, prompt)  # x* = seq[19] at position L = 19 (KV not yet written)
+    assert st.seq_len == 19 and st.x_star == int(seq[19])
+    accepted, committed = [], []
+    for s in range(steps):
+        res = oi.isd_step(dec, st, N, np.zeros(2 * N - 1), oi.ARGMAX, oi.GREEDY)
+        accepted.append(res.accepted)
+        committed.extend(res.committed)
+    return accepted, committed, seq
+
+
+@pytest.mark.parametrize("N", [2, 3, 4])
+def test_a_perfect_predictor_accepts_every_draft(monkeypatch, N):
+    """Pins R4 (which MASK row proposes which draft position): with a
+    predictor that is perfect for a token sequence, every draft it proposed
+    is the sequence's next token, so after the first (restart) step every
+    full step accepts all N - 1 drafts and commits N tokens: tokens per
+    forward N, the pages' formula at acceptance 1 (tpf_formula(1, N) = N,
+    [wiki] Method). The committed stream is the sequence itself."""
+    accepted, committed, seq = _perfect_predictor_run(monkeypatch, N)
+    assert oi.tpf_formula(1.0, N) == pytest.approx(N)
+    assert accepted[0] == 0                          # restart step: nothing pending
+    assert all(a == N - 1 for a in accepted[1:])
+    assert list(committed) == [int(t) for t in seq[20:20 + len(committed)]]
+
+
+@pytest.mark.parametrize("shift", [-1, 1])
+def test_proposals_read_from_the_wrong_mask_row_are_rejected(monkeypatch, shift):
+    """The planted mistake the pin above must catch: proposals read one MASK
+    row early or late are not the sequence's next tokens, so full steps
+    reject drafts (the committed stream stays the sequence: greedy ISD is
+    lossless whatever the proposals)."""
+    N = 4
+    accepted, committed, seq = _perfect_predictor_run(monkeypatch, N, shift=shift)
+    assert any(a < N - 1 for a in accepted[1:])
+    assert list(committed) == [int(t) for t in seq[20:20 + len(committed)]]
