@@ -538,9 +538,9 @@ def extra_configs(model, shape, args, seed):
 
 # DRAM bytes (read + write) of the tcgen05 attention kernel per byte of the
 # layer's K+V, from one ncu capture of the same launch in the two-layer
-# headline workload (549.9 MB for 527.9 MB of K+V; batch 64, prompts
+# headline workload (549.6 MB for 527.9 MB of K+V; batch 64, prompts
 # U[512, 4096]); the roofline's `traffic` scales it to this run's launch.
-ATTN_DRAM_PER_KV_BYTE = 549.854 / 527.933
+ATTN_DRAM_PER_KV_BYTE = 549.625 / 527.933
 
 
 def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
