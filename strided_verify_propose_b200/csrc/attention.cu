@@ -605,15 +605,14 @@ __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo_by
 }
 
 // Work of the tcgen05 kernel: the (request, KV head) pairs in one sequence,
-// request-major, then head. Pair (b, g) occupies nt_b + kTcSegCost units: the
-// first kTcSegCost stand for the fixed cost of starting and finishing a
-// segment (row state, partial-output write, the pipeline drain at its end),
+// request-major, then head. Pair (b, g) occupies nt_b + tc_seg_cost(p) units:
+// the first tc_seg_cost(p) stand for the fixed cost of starting and finishing
+// a segment (row state, partial-output write, the pipeline drain at its end),
 // then one unit per 128-key tile. CTA c of the C working CTAs takes units
 // [c U / C, (c+1) U / C), so a CTA whose range crosses many short pairs gets
 // fewer tiles. A maximal run of one pair's tiles inside a CTA's range is a
 // segment; it leaves its partial output in slot (b * nkv + g) * max_parts +
 // (c - the CTA of the pair's first tile).
-constexpr int kTcSegCost = 2;
 
 struct TcSeg {
   int b, g, t0, len, slot;
@@ -633,9 +632,15 @@ __host__ __device__ __forceinline__ int tc_cta_of(int64_t x, int64_t U, int C) {
   return static_cast<int>(((x + 1) * C - 1) / U);
 }
 
+// A segment's fixed cost in tile units: 3 at 32 query rows, 5 at 64 (the
+// row state and the partial write double; measured best at each size:
+// attention 4.44 vs 4.54 ms per step at 2 and 4.52 at 5 for Qwen3-8B widths,
+// batch 64; 16.46 vs 17.12 ms at 3 for Qwen3-32B widths).
+__host__ __device__ __forceinline__ int tc_seg_cost(const AttnParams& p) { return p.RG > 32 ? 5 : 3; }
+
 // First unit of request b (base[b] = 128-key tiles of the requests before b).
 __host__ __device__ __forceinline__ int64_t tc_ubase(const AttnParams& p, const int* base, int b) {
-  return static_cast<int64_t>(p.nkv) * (base[b] + static_cast<int64_t>(kTcSegCost) * b);
+  return static_cast<int64_t>(p.nkv) * (base[b] + static_cast<int64_t>(tc_seg_cost(p)) * b);
 }
 
 // Working CTAs: each takes at least min_tiles units.
@@ -665,18 +670,19 @@ __host__ __device__ __forceinline__ bool tc_next(const AttnParams& p, const int*
     }
     const int b = lo;
     const int nt = base[b + 1] - base[b];
-    const int w = nt + kTcSegCost;
+    const int sc = tc_seg_cost(p);
+    const int w = nt + sc;
     const int64_t x0b = tc_ubase(p, base, b);
     const int rem = static_cast<int>(r.x - x0b);
     const int g = rem / w, off = rem % w;
-    const int64_t first = x0b + static_cast<int64_t>(g) * w + kTcSegCost;   // the pair's first tile
-    if (off < kTcSegCost) {
+    const int64_t first = x0b + static_cast<int64_t>(g) * w + sc;   // the pair's first tile
+    if (off < sc) {
       r.x = first;   // start of the pair's tiles (of the next pair when nt = 0)
       continue;
     }
     sg.b = b;
     sg.g = g;
-    sg.t0 = off - kTcSegCost;
+    sg.t0 = off - sc;
     sg.len = static_cast<int>(i64min(r.hi - r.x, nt - sg.t0));
     const int part = r.c - tc_cta_of(first, r.U, r.C);
     sg.slot = part < p.max_parts ? (b * p.nkv + sg.g) * p.max_parts + part : -1;
@@ -707,7 +713,8 @@ __device__ __forceinline__ void combine_rows_tc(const AttnParams& p, const int* 
   int parts = 0;
   if (nt > 0) {
     const int C = tc_ctas(p, U, C_grid);
-    const int64_t first = tc_ubase(p, base, b) + static_cast<int64_t>(g) * (nt + kTcSegCost) + kTcSegCost;
+    const int sc = tc_seg_cost(p);
+    const int64_t first = tc_ubase(p, base, b) + static_cast<int64_t>(g) * (nt + sc) + sc;
     parts = tc_cta_of(first + nt - 1, U, C) - tc_cta_of(first, U, C) + 1;
   }
   if (parts > p.max_parts || parts > kMaxSplits) {

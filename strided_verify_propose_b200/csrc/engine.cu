@@ -116,7 +116,7 @@ bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
 using isd::GemmPlan;
 
 // K-splits allowed for the adapter's thin x A^T products
-constexpr int kLoraSplits = 32;
+constexpr int kLoraSplits = 16;
 
 struct isd_ctx {
   isd_model_cfg cfg{};

@@ -94,9 +94,10 @@ int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_
 // k_map / v_map: tensor maps over the pools as [n_layers*num_pages*n_kv*page_size][head_dim]
 // with box_rows = page_size.
 // qkv (optional): this layer's QKV split-K reduction, which produces q and
-// the block's K/V rows; the tcgen05 kernel runs it as its prologue (pro_cnt:
-// two ints, zero before the first launch, left zero), otherwise it is
-// launched first on its own.
+// the block's K/V rows; the tcgen05 kernel runs it as its prologue when its
+// (row, head) items fit one pass of the kernel's warps (pro_cnt: two ints,
+// zero before the first launch, left zero), otherwise it is launched first
+// on its own.
 struct QkvReduceArgs;
 cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map, const AttnShape& s,
                              int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,

@@ -14,8 +14,13 @@ import pytest
 import synth
 from strided_verify_propose_b200 import binding as B
 
-SEG_COST = 2          # tiles one segment counts for in the split
 TILE_KEYS = 128
+
+
+def seg_cost(R, nq, nkv):
+    """Tiles one segment counts for in the split: 3 for tiles of 32 query
+    rows per KV head, 5 for 64."""
+    return 5 if R * (nq // nkv) > 32 else 3
 
 
 def _check(batch, R, nq, nkv, maxp, page, kend, sms):
@@ -60,7 +65,8 @@ def _check(batch, R, nq, nkv, maxp, page, kend, sms):
                 assert s == (b * nkv + g) * max_parts + (c - c0)
     # balance: a CTA's tiles plus the overhead of the segments it starts fit
     # in its share of the units
-    units = nkv * (int(nt.sum()) + SEG_COST * batch)
+    sc = seg_cost(R, nq, nkv)
+    units = nkv * (int(nt.sum()) + sc * batch)
     used = sorted(set(int(c) for c in seg[:, 0]))
     share = -(-units // len(used))
     per_cta = {}
@@ -68,7 +74,7 @@ def _check(batch, R, nq, nkv, maxp, page, kend, sms):
         tiles, segs = per_cta.get(c, (0, 0))
         per_cta[c] = (tiles + ln, segs + 1)
     for c, (tiles, segs) in per_cta.items():
-        assert tiles + SEG_COST * (segs - 1) <= share, (c, tiles, segs, share)
+        assert tiles + sc * (segs - 1) <= share, (c, tiles, segs, share)
     return seg, max_parts
 
 
