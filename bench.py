@@ -405,7 +405,7 @@ def run_cuda(args, ws, rank, local):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (random-init weights, uniform random prompts, seeded)",
-            "config": {"workload": args.workload, "model": MODEL_NAMES.get(shape, "tiny"),
+            "config": {"workload": args.workload, "shape": MODEL_NAMES.get(shape, "tiny"),
                        "batch_per_gpu": B,
                        "global_batch": B * ws, "stride_n": N, "rows_per_step": B * R,
                        "prompt_len": [wl["len_lo"], wl["len_hi"]], "page_size": P,
