@@ -2,7 +2,8 @@
 
 The headline workload in the launch configuration bench.py times: Qwen3-8B
 shape with all 36 layers (random weights drawn on the device), batch 64,
-stride 4 (448 block rows), prompts U[512, 4096], pages randomly permuted.
+stride 4 (448 block rows), prompts U[512, 4096], pages randomly permuted;
+and the Qwen3-32B shape (64 layers) at batch 64 with prompts U[1024, 8192].
 The oracle cannot run this model, so each step is checked by what holds at
 any size:
 
@@ -24,14 +25,18 @@ from oracle import pages as op
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
-SHAPE = synth.QWEN3_8B
 BN, N, STEPS, SEED = 64, 4, 3, 1000
 
 
-def test_full_size_steps_hold_their_invariants():
+@pytest.mark.parametrize("shape_name,len_lo,len_hi", [
+    ("QWEN3_8B", 512, 4096),       # the headline workload
+    ("QWEN3_32B", 1024, 8192),     # Qwen3-32B shape, 64 layers, 56 query rows per KV head
+])
+def test_full_size_steps_hold_their_invariants(shape_name, len_lo, len_hi):
     from strided_verify_propose_b200 import binding as B
+    SHAPE = getattr(synth, shape_name)
     R, P, V = 2 * N - 1, SHAPE.page_size, SHAPE.vocab
-    lens = synth.prompt_lengths(BN, 512, 4096, SEED)
+    lens = synth.prompt_lengths(BN, len_lo, len_hi, SEED)
     prompts = synth.prompts(SHAPE, lens, SEED)
     maxp = op.pages_covering(int(lens.max()) + (STEPS + 1) * N + R + 1, P) + 1
     need = [op.pages_covering(int(L) - 1 + R, P) for L in lens]
