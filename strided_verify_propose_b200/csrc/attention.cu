@@ -22,7 +22,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "qkv_row.cuh"
 
 namespace isd {
 
@@ -52,18 +51,12 @@ struct AttnParams {
   int32_t min_tiles;           // fewest tiles per CTA (fewer CTAs for small work)
   int32_t kstages, vstages;    // K and V ring slots
   int32_t* status;
-  // tcgen05 kernel prologue: this layer's QKV reduction (QK-norm, RoPE, q and
-  // the block's K/V page writes) done by every CTA before any load
-  int32_t qkv_on;
-  QkvReduceArgs qkv;
-  int32_t* pro_cnt;            // [2] arrivals / departures (zero between launches)
   // rows of a request hold one block at consecutive positions (a decode
   // step): K/V tiles of keys below its first row are not written by the
   // QKV reduction and may be loaded before waiting for it
   int32_t prefix_early;
-  // launched with programmatic stream serialisation right after the kernel
-  // that writes q and the block's K/V rows (the QKV reduction, or the QKV
-  // projection when the reduction is the prologue): nothing it writes is
+  // launched with programmatic stream serialisation right after the QKV
+  // reduction that writes q and the block's K/V rows: nothing it writes is
   // read before griddep_wait()
   int32_t pdl;
 };
@@ -871,34 +864,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
   }
   build_items(p, kend, base);     // ends with __syncthreads
-  if (p.pdl && p.qkv_on) griddep_wait();   // the prologue reads the QKV projection
-  if (p.qkv_on) {
-    // this layer's QKV reduction, (row, head) items spread over every warp of
-    // the grid, four per warp at a time with all their loads in flight; the
-    // producer issues no load before every CTA has finished its items
-    const int nw = blockDim.x / 32;
-    const int n_heads = p.qkv.n_q + 2 * p.qkv.n_kv;
-    const int items = p.qkv.rows * n_heads;
-    const int gws = gridDim.x * nw;
-    for (int i0 = blockIdx.x * nw + warp; i0 < items; i0 += 4 * gws) {
-      float v[4][4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int it = i0 + k * gws;
-        if (it < items) qkv_head_sum<128>(p.qkv, it / n_heads, it % n_heads, lane, v[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int it = i0 + k * gws;
-        if (it < items) qkv_head_finish<128>(p.qkv, it / n_heads, it % n_heads, lane, v[k]);
-      }
-    }
-    // q and the K/V rows are read by TMA (the async proxy) in every CTA
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) atomicAdd(&p.pro_cnt[0], 1);
-  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // base[b]: tiles of the requests before b (128-key tiles, split_keys = 128)
@@ -953,7 +918,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       TcSeg sg;
       bool have = tc_next(p, base, rg, sg);
       int pre = 0;   // tiles of the first segment loaded before the wait for q and K/V
-      if (p.qkv_on || p.pdl) {
+      if (p.pdl) {
         if (have && p.prefix_early) {
           // prefix keys only: the block's own rows are the QKV reduction's output
           const int k_lo = sg.t0 * kTcKeys;
@@ -965,24 +930,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ++pre;
           }
         }
-        if (p.qkv_on) {
-          const int total = static_cast<int>(gridDim.x);
-          const long long t0 = clock64();
-          const long long limit = *const_cast<volatile long long*>(&g_wait_limit);
-          while (ok && ld_acquire_gpu(&p.pro_cnt[0]) < total) {
-            if (clock64() - t0 > limit) {
-              ok = false;
-              break;
-            }
-          }
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-          if (atomicAdd(&p.pro_cnt[1], 1) == total - 1) {
-            p.pro_cnt[0] = 0;
-            p.pro_cnt[1] = 0;
-          }
-        } else {
-          griddep_wait();   // the QKV reduction ahead in the stream has finished
-        }
+        griddep_wait();   // the QKV reduction ahead in the stream has finished
       }
       for (; ok && have; have = tc_next(p, base, rg, sg), ++it) {
         const int b = sg.b, g = sg.g;
@@ -1516,8 +1464,8 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
                              int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
-                             cudaEvent_t between, const QkvReduceArgs* qkv, int32_t* pro_cnt,
-                             bool prefix_early, bool pdl) {
+                             cudaEvent_t between, const QkvReduceArgs* qkv, bool prefix_early,
+                             bool pdl) {
   if (s.batch > kMaxBatch) return cudaErrorInvalidValue;
   const Derived d = derive(s);
   int sms = 148;
@@ -1526,15 +1474,13 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
     if (cudaGetDevice(&dev) == cudaSuccess)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  // The QKV reduction runs first: inside the tcgen05 kernel when its (row,
-  // head) items need one pass of the kernel's warps (decode at small batch,
-  // where the saved launch is the gain), else as its own kernel, which
-  // spreads many items over a full device of warps (measured: fused costs
-  // 0.38 ms per step at 448 rows, saves 0.1 ms at 7).
-  const bool fuse_qkv = qkv != nullptr && d.tc && pro_cnt != nullptr && qkv->head_dim == 128 &&
-                        static_cast<int64_t>(qkv->rows) * (qkv->n_q + 2 * qkv->n_kv) <=
-                            static_cast<int64_t>(sms) * (kTcThreads / 32);
-  if (qkv != nullptr && !fuse_qkv) {
+  // The layer's QKV reduction (QK-norm, RoPE, q and the block's K/V rows)
+  // runs first, as its own kernel. (Run instead as this kernel's prologue,
+  // every warp taking (row, head) items before a barrier over the grid, it
+  // measured 0.38 ms per step slower at 448 rows and, once the kernel loaded
+  // earlier steps' K/V before waiting for the reduction, 0.08 ms slower at
+  // 7 rows too.)
+  if (qkv != nullptr) {
     const cudaError_t e = launch_qkv_reduce(*qkv, stream);
     if (e != cudaSuccess) return e;
     if (launches) *launches += 1;
@@ -1574,15 +1520,8 @@ cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map,
   p.part_ml = reinterpret_cast<float2*>(p.part_o + static_cast<size_t>(d.max_items) * rows * s.head_dim);
   p.item_base = reinterpret_cast<int32_t*>(p.part_ml + static_cast<size_t>(d.max_items) * rows);
   p.status = status;
-  p.qkv_on = fuse_qkv ? 1 : 0;
-  if (fuse_qkv) {
-    if (qkv->splits < 1 || qkv->splits > 8) return cudaErrorInvalidValue;
-    p.qkv = *qkv;
-  }
-  p.pro_cnt = pro_cnt;
   p.prefix_early = prefix_early ? 1 : 0;
-  // programmatic launch only after a kernel that writes q and K/V: the QKV
-  // reduction launched just above, or (fused) the QKV projection
+  // programmatic launch only right after the QKV reduction launched above
   p.pdl = pdl && qkv != nullptr && d.tc ? 1 : 0;
   static bool attr_set = false;
   if (!attr_set) {

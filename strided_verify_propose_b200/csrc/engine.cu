@@ -157,7 +157,6 @@ struct isd_ctx {
   void* acc_ws = nullptr;
   size_t acc_ws_bytes = 0;
   int32_t* prefill_lens = nullptr;  // [max_batch]
-  int32_t* pro_cnt = nullptr;       // [2] grid-barrier words of the attention's prologue
   int32_t* prefill_order = nullptr; // [max_batch] requests by descending prompt length
   int32_t* prefill_ptab = nullptr;  // [max_batch][max pages] page table rows in that order
 
@@ -473,12 +472,12 @@ int forward_layers(isd_ctx* c, const isd_kv* kv, int batch, int rows_per_req, in
     qa.v_pool = static_cast<__nv_bfloat16*>(kv->v_pool_dev);
     qa.q_out = c->qbuf;
     qa.status = status;
-    // the QKV reduction runs as the attention kernel's prologue where it can
+    // the QKV reduction, then the attention (both in launch_attention)
     cudaEvent_t a1 = prof_mark(c, st);
     cudaEvent_t amid = prof_event(c);
     ISD_CUDA(isd::launch_attention(kmap, vmap, ash, l, c->qbuf, c->meta_pos, ash_table,
                                    c->attn, c->attn_ws, status, st, &c->launches, amid, &qa,
-                                   c->pro_cnt, attn_sub == 1 && ash_table == kv->page_table_dev &&
+                                   attn_sub == 1 && ash_table == kv->page_table_dev &&
                                                         rows_per_req == ash.rows_per_req,
                                    c->pdl));
     cudaEvent_t a2 = prof_mark(c, st);
@@ -594,7 +593,6 @@ int alloc_workspace(isd_ctx* c) {
       c->sk_ws_bytes,
       static_cast<size_t>(g.max_batch) * c->prefill_sub_max * max_pages * 4,   // prefill table
       static_cast<size_t>(g.max_batch) * 4,                                    // prefill order
-      512,                    // grid-barrier words of the attention's prologue (2 used)
       static_cast<size_t>(g.max_batch) * max_pages * 4,                        // prefill page rows
       step_rows * static_cast<size_t>(g.vocab / 32) * sizeof(float4),          // slab statistics
   };
@@ -627,11 +625,9 @@ int alloc_workspace(isd_ctx* c) {
   c->sk_ws = b + off[i++];
   c->prefill_table = reinterpret_cast<int32_t*>(b + off[i++]);
   c->prefill_order = reinterpret_cast<int32_t*>(b + off[i++]);
-  c->pro_cnt = reinterpret_cast<int32_t*>(b + off[i++]);
   c->prefill_ptab = reinterpret_cast<int32_t*>(b + off[i++]);
   c->slab_stats = reinterpret_cast<float4*>(b + off[i++]);
-  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess ||
-      cudaMemset(c->pro_cnt, 0, 512) != cudaSuccess)
+  if (cudaMemset(c->sk_ws, 0, isd::gemm_streamk_sync_bytes()) != cudaSuccess)
     return fail(ISD_E_CUDA, "GEMM synchronisation words clear failed");
   // RoPE table in double precision: angle = pos * theta^(-2i/d)
   const int half = g.head_dim / 2;

@@ -94,24 +94,19 @@ int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_
 // k_map / v_map: tensor maps over the pools as [n_layers*num_pages*n_kv*page_size][head_dim]
 // with box_rows = page_size.
 // qkv (optional): this layer's QKV split-K reduction, which produces q and
-// the block's K/V rows; the tcgen05 kernel runs it as its prologue when its
-// (row, head) items fit one pass of the kernel's warps (pro_cnt: two ints,
-// zero before the first launch, left zero), otherwise it is launched first
-// on its own.
+// the block's K/V rows; it is launched first, as its own kernel.
 struct QkvReduceArgs;
 cudaError_t launch_attention(const CUtensorMap& k_map, const CUtensorMap& v_map, const AttnShape& s,
                              int32_t layer, const __nv_bfloat16* q, const int32_t* row_pos,
                              const int32_t* page_table, __nv_bfloat16* out, void* workspace,
                              int32_t* status, cudaStream_t stream, int* launches,
                              cudaEvent_t between = nullptr, const QkvReduceArgs* qkv = nullptr,
-                             int32_t* pro_cnt = nullptr, bool prefix_early = false,
-                             bool pdl = false);
+                             bool prefix_early = false, bool pdl = false);
 // (prefix_early: each request's rows are one block at consecutive positions,
 // a decode step, so K/V tiles below a request's first row do not depend on
 // the QKV reduction and may be loaded before waiting for it. pdl: the
-// tcgen05 kernel is launched with programmatic stream serialisation, which
-// is correct only when the kernel ahead of it in the stream is the QKV
-// reduction this call launches or the QKV projection feeding its prologue.)
+// tcgen05 kernel is launched with programmatic stream serialisation right
+// after the QKV reduction this call launches.)
 
 // ------------------------------------------------------------------ row ops
 struct RowMeta {

@@ -1,6 +1,5 @@
-// One (row, head) of the QKV projection's split-K reduction, shared by the
-// standalone reduction kernel and the attention kernel's prologue so that
-// both give the same bits: the splits summed in ascending order; for q and
+// One (row, head) of the QKV projection's split-K reduction (one warp per
+// item in qkv_reduce_kernel): the splits summed in ascending order; for q and
 // k heads RMSNorm over head_dim and NeoX rotary embedding (pairs (i, i +
 // d/2)) at the row's absolute position; q to the attention input, k and v
 // into the row's page slot. Lane l holds elements l + 32 j of the head.
