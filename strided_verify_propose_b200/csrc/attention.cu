@@ -1420,6 +1420,7 @@ int attention_split(const AttnShape& s, const int32_t* kend, int num_sms, int32_
   AttnParams p{};
   p.B = s.batch;
   p.nkv = s.n_kv_heads;
+  p.RG = d.RG;                  // the tile height sets the segment cost
   p.min_tiles = d.min_tiles;
   p.max_parts = d.max_splits;
   // 128-key tile prefix, as the kernel builds it from the row positions

@@ -107,6 +107,34 @@ def test_random_shapes(seed):
     _check(batch, R, nkv * G, nkv, maxp, page, kend, sms)
 
 
+def test_benchmark_shape_qwen3_32b():
+    """Qwen3-32B widths, batch 64, 7 rows per request (56 query rows per KV
+    head: tiles of 64 rows, 5 tiles per segment), prompts U[1024, 8192]."""
+    lens = synth.prompt_lengths(64, 1024, 8192, 7)
+    seg, _ = _check(64, 7, 64, 8, 130, 64, lens + 7, 148)
+    assert len(set(seg[:, 0].tolist())) == 148
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_random_shapes_64_rows(seed):
+    """33..64 query rows per KV head (the 64-row tile and its segment cost)."""
+    rng = np.random.default_rng(1000 + seed)
+    batch = int(rng.integers(1, 120))
+    nkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    R = int(rng.integers(32 // G + 1, 64 // G + 1))
+    page = 64
+    maxp = int(rng.integers(1, 80))
+    kend = rng.integers(0, maxp * page + 200, batch)
+    if seed % 5 == 0:
+        kend[:] = rng.integers(0, 3, batch)
+    if kend.max() <= 0:
+        kend[0] = 1
+    sms = int(rng.choice([1, 7, 148]))
+    assert R * G > 32
+    _check(batch, R, nkv * G, nkv, maxp, page, kend, sms)
+
+
 def test_shapes_not_on_tensor_cores():
     # head_dim 64, 32-key pages and more than 64 query rows per KV head go to
     # the other kernel; 33..64 rows (Qwen3-32B's 8 heads x 7 rows) stay
