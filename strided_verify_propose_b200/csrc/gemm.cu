@@ -594,7 +594,10 @@ GemmPlan plan_gemm(int32_t m, int32_t n_out, int32_t k, int32_t force_splits, in
   // 2-SM pairs need an even number of 128-row tiles; mma_n is a multiple of
   // 16 (n_pad is padded to 16, or to 32 when split over two MMAs), so each
   // CTA's half of an MMA's tokens is a whole number of 8-row swizzle atoms.
-  best.pair = (m_tiles % 2 == 0 && best.mma_n % 16 == 0) ? 1 : 0;
+  // With at most 32 token columns a pair shares almost nothing (a few KB of
+  // tokens per K-block) and its cluster set-up and barriers are pure cost:
+  // single CTAs there (batch 1: 4.40 -> 4.28 ms per step).
+  best.pair = (m_tiles % 2 == 0 && best.mma_n % 16 == 0 && best.n_pad > 32) ? 1 : 0;
   if (best.pair) {
     best.box_rows = best.mma_n / 2;
     best.n_boxes = best.n_mma;

@@ -33,7 +33,7 @@ def _bf16(a):
 # ------------------------------------------------------------------- GEMM ---
 
 @pytest.mark.parametrize("m,n,k,split", [
-    (7, 256, 256, 1),          # decode b1 rows, one 2-SM pair of tiles
+    (7, 256, 256, 1),          # decode b1 rows (single CTAs: no pairs at <= 32 token columns)
     (7, 384, 256, 1),          # odd tile count: single-CTA MMAs
     (28, 512, 1024, 3),        # ragged split-K
     (300, 384, 640, 1),        # ragged token count, n_pad not a multiple of 32
