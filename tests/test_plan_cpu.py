@@ -41,6 +41,7 @@ def test_plans_satisfy_the_kernel_invariants(single):
         if p["pair"]:
             assert tiles % 2 == 0 and p["box_rows"] * 2 == p["mma_n"]
             assert p["n_boxes"] == p["n_mma"]
+            assert p["n_pad"] > 32          # few tokens: single CTAs
         else:
             assert p["box_rows"] * p["n_boxes"] == p["n_pad"]
         # shared memory: stages of 16 KB weights + this CTA's token rows
@@ -68,6 +69,17 @@ def test_the_step_shapes_plan_as_measured():
     assert (gate_up["pair"], gate_up["streamk"], gate_up["units"]) == (1, 1, 74)
     lm_head = B.gemm_plan(448, 151936, 4096, single=True)
     assert (lm_head["pair"], lm_head["streamk"], lm_head["units"]) == (0, 1, 148)   # 1187 tiles: odd
+
+
+def test_the_batch1_shapes_plan_as_measured():
+    """Qwen3-8B at batch 1, stride 4 (7 rows): single CTAs (a pair would share
+    only a 2 KB token tile per K-block), one wave of K-splits or stream-K."""
+    qkv = B.gemm_plan(7, 6144, 4096)
+    assert (qkv["pair"], qkv["n_pad"], qkv["splits"]) == (0, 16, 3)
+    o = B.gemm_plan(7, 4096, 4096)
+    assert (o["pair"], o["splits"]) == (0, 4)
+    gate_up = B.gemm_plan(7, 24576, 4096, single=True)
+    assert (gate_up["pair"], gate_up["streamk"], gate_up["units"]) == (0, 1, 148)
 
 
 def test_invalid_shapes_are_refused():
