@@ -6,15 +6,24 @@
 // the block's own K/V are written to their page slots before this kernel
 // runs, so one causal mask over positions covers both parts).
 //
-// Work unit = (request b, KV head g, key split s). The R rows x G query heads
-// that share KV head g form one query tile of R*G rows (28 at stride 4 with
-// Qwen3-8B's 4:1 grouping), so each K/V byte is read once per request. A
-// producer warp streams 64-key tiles of K and V page by page with TMA
-// (128-byte swizzled boxes of one page x 64 dims, zero-filled past the
-// request's end) into a ring of stages; four consumer warps run QK^T and PV
-// on mma.sync bf16 tensor cores with an fp32 online softmax. Warps split the
-// query rows into 16-row tiles and the 64 keys of a tile into key groups;
-// key groups are merged through shared memory, splits by a second kernel.
+// The R rows x G query heads that share KV head g form one query tile of
+// R*G rows (28 at stride 4 with Qwen3-8B's 4:1 grouping, 56 with
+// Qwen3-32B's 8:1), so each K/V byte is read once per request. Two kernels:
+//
+// * attn_tc_kernel (head_dim 128, 64-key pages, up to 64 query rows): the
+//   decode path. tcgen05 MMAs with TMEM accumulators: S^T = K Q^T and
+//   O_t^T = V^T P^T, K and V streamed by TMA through separate rings, one warp
+//   issuing the S MMAs and one the PV MMAs, eight softmax warps. One CTA per
+//   SM takes a contiguous range of the (request, KV head, 128-key tile)
+//   sequence, balanced by tiles plus a fixed cost per segment; the pairs cut
+//   between CTAs are merged by attn_combine_tc_kernel. Launched right after
+//   the QKV reduction with programmatic stream serialisation, so its first
+//   tiles of earlier steps' K/V load before it waits for that reduction.
+// * attn_persistent_kernel (the other shapes): work unit = (request, KV
+//   head, key split); a producer warp streams 64-key tiles with TMA into a
+//   ring; four consumer warps run QK^T and PV on mma.sync bf16 tensor cores
+//   with an fp32 online softmax; key groups are merged through shared
+//   memory, splits by attn_combine_kernel.
 #include <algorithm>
 #include <cstdlib>
 #include <string>

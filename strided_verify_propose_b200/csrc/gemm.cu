@@ -25,6 +25,13 @@
 //   Two addends commute exactly, so results do not depend on which part
 //   finishes first, and no CTA ever waits for one that has not started.
 // Both are bitwise reproducible run to run.
+//
+// Plans with more than 32 token columns run even tile counts as 2-SM pairs
+// (tcgen05 cta_group::2, M = 256). Launched with programmatic stream
+// serialisation, the producer loads the first ring of weight tiles before
+// it waits for the kernel ahead. The fp32 epilogue can also write, per 32
+// output rows, the max, the sum of exp and the first argmax of each token's
+// results (the LM head's accept statistics).
 #include <algorithm>
 #include <cmath>
 #include <cstring>
