@@ -139,3 +139,38 @@ def test_component_calls_refuse_unsupported_shapes():
     assert lib.isd_paged_attention(*args, 4, 9, 64, 8, 128, 64, 10, 4, 1, 0, 1, 1, 1 << 20, None,
                                    None) == binding.ISD_E_UNSUPPORTED
     assert lib.isd_set_wait_limit(10) == binding.ISD_E_INVALID
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """The product path has no fallback: without libisd.so the binding raises."""
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libisd.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        binding.lib()
+
+
+def _sources(top, exts):
+    for d, _, files in os.walk(os.path.join(ROOT, top)):
+        for f in files:
+            if f.endswith(exts):
+                yield os.path.join(d, f)
+
+
+def test_oracle_and_product_share_no_code():
+    """Neither side imports, includes or loads the other, and the input
+    generators import neither."""
+    imp = re.compile(r"^\s*(from|import)\s+([A-Za-z_][\w.]*)", re.M)
+    inc = re.compile(r'^\s*#\s*include\s*[<"]([^>"]+)[>"]', re.M)
+    for path in _sources("strided_verify_propose_b200", (".py",)):
+        mods = [m.group(2) for m in imp.finditer(open(path).read())]
+        assert not [m for m in mods if m.split(".")[0] == "oracle"], path
+    for path in list(_sources("strided_verify_propose_b200", (".cu", ".cuh", ".h"))) + \
+            list(_sources("include", (".h",))):
+        assert not [h for h in inc.findall(open(path).read()) if "oracle" in h], path
+    for path in _sources("oracle", (".py", ".c", ".h")):
+        src = open(path).read()
+        mods = [m.group(2).split(".")[0] for m in imp.finditer(src)]
+        assert "strided_verify_propose_b200" not in mods and "libisd" not in src, path
+    for path in _sources("synth", (".py",)):
+        mods = [m.group(2).split(".")[0] for m in imp.finditer(open(path).read())]
+        assert "oracle" not in mods and "strided_verify_propose_b200" not in mods, path
