@@ -113,6 +113,23 @@ def test_rms_norm_closed_form():
     assert np.allclose(y, [[3 / rms, 8 / rms]], rtol=1e-15)
 
 
+def test_rms_norm_matches_the_library_norm_at_large_eps():
+    """eps sits inside the root: against the Qwen3 RMSNorm of HF transformers
+    (an independent implementation) at an eps large enough to show where it
+    is added."""
+    torch = pytest.importorskip("torch")
+    tr = pytest.importorskip("transformers.models.qwen3.modeling_qwen3")
+    x = np.asarray(synth.normal((6, 10), 4, 1), dtype=np.float64) * 0.3
+    g = 1.0 + np.asarray(synth.normal((10,), 4, 2), dtype=np.float64) * 0.3
+    for eps in (0.0, 0.05, 0.5):
+        norm = tr.Qwen3RMSNorm(10, eps=eps).double()
+        with torch.no_grad():
+            norm.weight.copy_(torch.tensor(g))
+            ref = norm(torch.tensor(x)).numpy()
+        # the library normalises in float32
+        assert np.allclose(om.rms_norm(x, g, eps), ref, rtol=2e-6, atol=0)
+
+
 def test_block_rows_are_causal():
     shape = SMALL
     dec = om.Decoder(shape, _weights(shape, seed=5))

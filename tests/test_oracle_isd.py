@@ -89,11 +89,60 @@ def test_accept_resample_reproduces_p_exactly(propose, seed):
     assert np.abs(total - p).max() < 1e-12
 
 
+@pytest.mark.parametrize("propose", [oi.ARGMAX, oi.SAMPLE])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_second_draft_reproduces_its_row_exactly(propose, seed):
+    """N = 3, first draft accepted: P(the token committed after it = x) ==
+    p_1(x), row 1's distribution, integrating decide() over the second
+    draft's accept test and the resampling uniform. The two drafts differ,
+    so the residual must remove the second draft's proposal mass, not the
+    first's."""
+    V, N = 7, 3
+    z = np.stack([synth.normal((V,), seed, 10 + r, std=1.5) for r in range(2 * N - 1)]).astype(np.float64)
+    zq = [synth.normal((V,), seed, 20 + r, std=1.5).astype(np.float64) for r in range(2)]
+    p1 = oi.softmax(z[1])
+    if propose == oi.ARGMAX:
+        d2 = int(np.argmax(zq[1]))
+        cases = [((d2 + 1) % V, d2, 1.0, None)]
+    else:
+        q = [oi.softmax(r) for r in zq]
+        cases = [(int(np.argmax(zq[0])), d2, q[1][d2], q) for d2 in range(V)]
+    total = np.zeros(V)
+    for d1, d2, qd, qrows in cases:
+        assert d1 != d2 or propose == oi.SAMPLE
+
+        def run(u1, u2):
+            return oi.decide(z, [d1, d2], qrows, N, [0.0, u1, u2, 0.5, 0.5], propose=propose)
+        assert run(0.0, 0.5).accepted >= 1                  # u = 0 accepts the first draft
+        t_acc = _threshold(lambda u1: run(u1, 0.5).accepted == 2)
+        total[d2] += qd * t_acc
+        if t_acc < 1.0:
+            u_rej = min(1.0 - 1e-12, t_acc + 0.5 * (1.0 - t_acc))
+            assert run(u_rej, 0.5).accepted == 1
+            total += qd * (1.0 - t_acc) * _sampler_intervals(lambda u2: run(u_rej, u2).new_token, V)
+    assert np.abs(total - p1).max() < 1e-12
+
+
 def test_residual_with_identical_p_q_falls_back_to_p():
     p = oi.softmax(np.array([0.3, -1.0, 2.0]))
     assert np.array_equal(oi.residual(p, p), p)
     r = oi.residual(p, np.array([1.0, 0.0, 0.0]))
     assert r[0] == 0.0 and np.array_equal(r[1:], p[1:])
+
+
+def test_a_draft_of_probability_zero_is_never_accepted():
+    """min(1, p/q) = 0 when p(d) = 0: the draft is rejected for every u in
+    [0, 1), u = 0 included, whatever its proposal probability."""
+    V, N = 5, 2
+    rows = np.array([[0.0, 1.0, -1000.0, 0.5, 0.2],     # p(2) underflows to exactly 0
+                     [0.3, 0.1, 0.0, -0.2, 0.4],
+                     [0.0, 0.0, 0.0, 0.0, 0.0]])
+    assert oi.softmax(rows[0])[2] == 0.0
+    q = np.full(V, 0.2)
+    for u0 in (0.0, 0.5, 1.0 - 2.0**-53):
+        u = [u0, 0.3, 0.6]
+        assert oi.decide(rows, [2], None, N, u, propose=oi.ARGMAX).accepted == 0
+        assert oi.decide(rows, [2], [q], N, u, propose=oi.SAMPLE).accepted == 0
 
 
 def test_inverse_cdf_rules():
@@ -306,7 +355,8 @@ def _exact_ar_distribution(m, prompt, K):
     return dist
 
 
-@pytest.mark.parametrize("N,propose,K", [(2, oi.SAMPLE, 3), (3, oi.SAMPLE, 3), (2, oi.ARGMAX, 3)])
+@pytest.mark.parametrize("N,propose,K", [(2, oi.SAMPLE, 3), (3, oi.SAMPLE, 3), (2, oi.ARGMAX, 3),
+                                         (3, oi.ARGMAX, 3)])
 def test_isd_trajectory_distribution_equals_ar(N, propose, K):
     shape = synth.ModelShape(n_layers=1, hidden=8, n_q_heads=2, n_kv_heads=1, head_dim=4,
                              intermediate=8, vocab=3, page_size=16)
