@@ -257,7 +257,8 @@ int isd_paged_attention(const void *q_dev, const int32_t *row_pos_dev, const voi
  * 128, 64-key pages, at most 64 query rows per KV head): no GPU work. The
  * kernel runs one CTA per SM over the (request, KV head, 128-key tile)
  * sequence; each CTA takes a contiguous range in which every (request, KV
- * head) segment counts as 2 tiles besides its own tiles, and a pair cut
+ * head) pair costs a fixed 3 tiles besides its own tiles (5 above 32 query
+ * rows per KV head: starting and finishing a pair), and a pair cut
  * between CTAs leaves one partial per CTA, merged in CTA order (paged
  * attention on tensor cores, a block's queries against its request's paged
  * prefix; Bud's Wiki "Introspective Diffusion Language Models", Method).
