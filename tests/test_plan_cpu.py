@@ -16,9 +16,11 @@ MAX_SMEM = 231424 + 1280   # dynamic shared memory the kernel is given, plus ali
 
 
 def _shapes():
+    # Qwen3-8B and Qwen3-32B widths (hidden 4096 / 5120, QKV 6144 / 10240,
+    # gate/up 24576 / 51200, down K 12288 / 25600), the adapter's rank 128
     ms = [1, 7, 28, 96, 224, 300, 448, 449, 512, 960, 1024, 4096]
-    ns = [128, 256, 384, 1024, 4096, 6144, 19072, 24576, 151936]
-    ks = [64, 256, 4096, 12288]
+    ns = [128, 256, 384, 1024, 4096, 5120, 6144, 10240, 19072, 24576, 51200, 151936]
+    ks = [64, 128, 256, 4096, 5120, 8192, 12288, 25600]
     return list(itertools.product(ms, ns, ks))
 
 
