@@ -188,6 +188,29 @@ def step_bytes_flops(shape, lens_now, B, N):
 
 # ---------------------------------------------------------------- CUDA arm ---
 
+def metric_name(workload: str) -> str:
+    """The JSON line's `metric` (both arms print the same one)."""
+    if workload == "qwen3_8b_b64":
+        return "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
+    return f"committed tokens/s ({workload})"
+
+
+def workload_config(workload: str, ws: int) -> dict:
+    """The JSON line's `config` (both arms print the same one): the workload
+    with its sizes, and how it spreads over ws ranks."""
+    wl = WORKLOADS[workload]
+    shape, B, N = wl["shape"], wl["batch"], wl["stride"]
+    wbytes = 2 * step_w_params(shape)
+    return {"workload": workload, "shape": MODEL_NAMES.get(shape, "tiny"), "batch_per_gpu": B,
+            "global_batch": B * ws, "stride_n": N, "rows_per_step": B * (2 * N - 1),
+            "prompt_len": [wl["len_lo"], wl["len_hi"]], "page_size": shape.page_size,
+            "parallelism": f"replicas x{ws} (request-sharded, no collective)",
+            "uniforms": f"acceptance-controlled a={ACCEPT_RATE}",
+            "l2": (f"inputs larger than L2 (weights {wbytes / 1e9:.0f} GB + KV > 126 MB)"
+                   if wbytes > 126e6 else
+                   f"inputs smaller than L2 (weights {wbytes / 1e6:.1f} MB): a test workload")}
+
+
 def run_cuda(args, ws, rank, local):
     import torch
     import torch.distributed as dist
@@ -394,8 +417,7 @@ def run_cuda(args, ws, rank, local):
         ceiling = (step_bytes / (peaks["hbm"] * 1e9)) / t_floor
         roof = roofline_entry(prof, shape, B, N, lens_prof, args.steps, peaks)
         result = {
-            "metric": "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
-            if args.workload == "qwen3_8b_b64" else f"committed tokens/s ({args.workload})",
+            "metric": metric_name(args.workload),
             "value": committed / (ms * 1e-3),
             "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -405,14 +427,7 @@ def run_cuda(args, ws, rank, local):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (random-init weights, uniform random prompts, seeded)",
-            "config": {"workload": args.workload, "shape": MODEL_NAMES.get(shape, "tiny"),
-                       "batch_per_gpu": B,
-                       "global_batch": B * ws, "stride_n": N, "rows_per_step": B * R,
-                       "prompt_len": [wl["len_lo"], wl["len_hi"]], "page_size": P,
-                       "parallelism": f"replicas x{ws} (request-sharded, no collective)",
-                       "uniforms": f"acceptance-controlled a={ACCEPT_RATE}",
-                       "l2": f"inputs larger than L2 (weights {2 * step_w_params(shape) / 1e9:.0f} GB "
-                             "+ KV > 126 MB)"},
+            "config": workload_config(args.workload, ws),
             "tokens_per_forward": committed / (args.steps * B * ws),
             "hbm_roofline_fraction_step": hbm_frac_step,
             "hbm_roofline_ceiling_step": ceiling,
@@ -671,14 +686,11 @@ def run_reference(args, ws, rank):
         oracle_sample(args, 1, args.workload)
     t0 = time.time()
     value, threads, sample, per_step = oracle_sample(args, reps, args.workload)
-    wl = WORKLOADS[args.workload]
-    return {"metric": "committed tokens/s (ISD step, Qwen3-8B shape, batch 64, N=4)"
-            if args.workload == "qwen3_8b_b64" else f"committed tokens/s ({args.workload})",
+    return {"metric": metric_name(args.workload),
             "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "batch_per_gpu": wl["batch"],
-                                             "stride_n": wl["stride"]},
+            "data": "synthetic", "config": workload_config(args.workload, ws),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": sample, "wall_s": time.time() - t0,
                              "cpu_model": cpu_model(), "host_cpus": os.cpu_count()},

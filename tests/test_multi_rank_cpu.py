@@ -63,3 +63,24 @@ def test_reference_arm_runs_on_rank_zero_only():
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_prints_the_gpu_arms_metric_and_config():
+    """Both arms describe the same workload: the reference line's metric,
+    unit, direction and config are the ones the GPU arm prints."""
+    sys.path.insert(0, ROOT)
+    import bench
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.metric_name("tiny")
+    assert line["config"] == bench.workload_config("tiny", 1)
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
+    head = bench.workload_config("qwen3_8b_b64", 1)
+    assert head["global_batch"] == 64 and head["rows_per_step"] == 448
+    assert head["l2"].startswith("inputs larger than L2")
