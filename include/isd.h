@@ -105,7 +105,7 @@ typedef struct {
  * pointers. A_t: [rank][in_t] bf16, B_t: [out_t][rank] bf16 (the two
  * nn.Linear weights); delta = scale * (x A_t^T) B_t^T on MASK rows only. */
 typedef struct {
-  int32_t rank;     /* multiple of 64, at most 256 */
+  int32_t rank;     /* 128, the rank the pages give (others: ISD_E_UNSUPPORTED) */
   float scale;
   const void *const *A[7];
   const void *const *B[7];

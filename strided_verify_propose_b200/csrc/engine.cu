@@ -728,7 +728,7 @@ int isd_load_gated_lora(isd_ctx* ctx, const isd_lora* lora) {
   if (!ctx || !lora) return fail(ISD_E_INVALID, "ctx and lora are required");
   const isd_model_cfg& g = ctx->cfg;
   const int r = lora->rank, L = g.n_layers;
-  if (r != 128 && r != 256) return fail(ISD_E_UNSUPPORTED, "gated LoRA rank must be 128 or 256");
+  if (r != 128) return fail(ISD_E_UNSUPPORTED, "gated LoRA rank must be 128");
   if (L < 1) return fail(ISD_E_INVALID, "the model has no layers");
   for (int t = 0; t < 7; ++t) {
     if (!lora->A[t] || !lora->B[t]) return fail(ISD_E_INVALID, "missing LoRA pointer array");
