@@ -88,14 +88,34 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def load_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(path):
+FALLBACK_PEAKS = dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0)
+
+
+def load_peaks(path=None):
+    """Roofline denominators: the measured copy bandwidth (GB/s) and bf16
+    GEMM rates (TFLOP/s, burst and sustained) from MEASURED_PEAKS.json when
+    it is there, each figure that is missing or not a plain positive number
+    taken from the fallback; `source` says which."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    keys = dict(hbm="hbm_gbs", bf16="bf16_tflops", bf16_sus="bf16_tflops_sustained")
+    try:
         with open(path) as f:
             p = json.load(f)
-        return dict(hbm=p.get("hbm_gbs", 6650.0), bf16=p.get("bf16_tflops", 1590.0),
-                    bf16_sus=p.get("bf16_tflops_sustained", 1400.0), source="measured")
-    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+    except (OSError, ValueError):
+        p = None
+    if not isinstance(p, dict):
+        return dict(FALLBACK_PEAKS, source="fallback")
+    out, used = {}, []
+    for k, name in keys.items():
+        v = p.get(name)
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            out[k] = float(v)
+            used.append(k)
+        else:
+            out[k] = FALLBACK_PEAKS[k]
+    out["source"] = ("measured" if len(used) == len(keys) else
+                     "fallback" if not used else "measured " + ", ".join(used) + "; fallback for the rest")
+    return out
 
 
 class ClockSampler:

@@ -77,3 +77,21 @@ def test_step_bytes_count_weights_kv_and_logits_once():
     assert kv == (100 + R + 300 + R) * shape.kv_bytes_per_token()
     assert logits == B * R * shape.vocab * 4
     assert flops == pytest.approx(2.0 * B * R * params)
+
+
+def test_peaks_file_figures_and_fallbacks(tmp_path):
+    """The measured peaks are used when the driver's file holds them as plain
+    numbers; anything else falls back figure by figure, and `source` says so."""
+    f = tmp_path / "peaks.json"
+    assert bench.load_peaks(str(tmp_path / "absent.json"))["source"] == "fallback"
+    f.write_text('{"hbm_gbs": 6531.3, "bf16_tflops": 1636.3, "bf16_tflops_sustained": 1396.6}')
+    p = bench.load_peaks(str(f))
+    assert (p["hbm"], p["bf16"], p["bf16_sus"], p["source"]) == (6531.3, 1636.3, 1396.6, "measured")
+    f.write_text('{"hbm_gbs": {"burst": 6531.3}, "bf16_tflops": 1636.3, "notes": "x"}')
+    p = bench.load_peaks(str(f))
+    assert p["hbm"] == bench.FALLBACK_PEAKS["hbm"] and p["bf16"] == 1636.3
+    assert p["bf16_sus"] == bench.FALLBACK_PEAKS["bf16_sus"] and "fallback" in p["source"]
+    for bad in ("not json", "[1, 2]", '{"hbm_gbs": true}', '{"hbm_gbs": -1}'):
+        f.write_text(bad)
+        p = bench.load_peaks(str(f))
+        assert p["hbm"] == bench.FALLBACK_PEAKS["hbm"] and p["source"].endswith("fallback")
