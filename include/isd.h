@@ -228,7 +228,9 @@ size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k);
  * n_pad (token columns per CTA), token chunks, splits, K-blocks per split,
  * MMAs per k-step, MMA N, TMA box rows, boxes, pipeline stages, 2-SM pair
  * (0/1), stream-K (0/1), stream-K units, TMEM columns, dynamic shared
- * memory bytes. Returns ISD_E_UNSUPPORTED when no plan exists. */
+ * memory bytes. Returns ISD_E_UNSUPPORTED when no plan exists (n not a
+ * multiple of 128, k not of 64), ISD_E_INVALID for m, max_splits or num_sms
+ * below 1 or a null out. */
 #define ISD_GEMM_PLAN_FIELDS 14
 int isd_gemm_plan(int32_t m, int32_t n, int32_t k, int32_t single, int32_t max_splits,
                   int32_t num_sms, int32_t *out);

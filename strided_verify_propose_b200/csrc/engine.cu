@@ -1033,8 +1033,10 @@ int isd_gemm_bf16(const void* w_dev, const void* x_dev, float* y_dev, int32_t m,
 int isd_gemm_plan(int32_t m, int32_t n, int32_t k, int32_t single, int32_t max_splits,
                   int32_t num_sms_hint, int32_t* out) {
   if (!out) return fail(ISD_E_INVALID, "null argument");
-  if (m < 1 || n < 128 || n % 128 || k < 64 || k % 64 || max_splits < 1 || num_sms_hint < 1)
-    return fail(ISD_E_INVALID, "need m >= 1, n % 128 == 0, k % 64 == 0, max_splits >= 1, sms >= 1");
+  if (m < 1 || max_splits < 1 || num_sms_hint < 1)
+    return fail(ISD_E_INVALID, "need m >= 1, max_splits >= 1, sms >= 1");
+  if (n < 128 || n % 128 || k < 64 || k % 64)
+    return fail(ISD_E_UNSUPPORTED, "need n % 128 == 0 and k % 64 == 0");
   const GemmPlan p = single ? isd::plan_gemm(m, n, k, 0, 1, num_sms_hint, true)
                             : isd::plan_gemm(m, n, k, 0, max_splits, num_sms_hint);
   const int32_t v[ISD_GEMM_PLAN_FIELDS] = {p.n_pad,  p.n_chunks, p.splits,  p.kb_per_split,

@@ -139,6 +139,12 @@ def test_component_calls_refuse_unsupported_shapes():
     assert lib.isd_paged_attention(*args, 4, 9, 64, 8, 128, 64, 10, 4, 1, 0, 1, 1, 1 << 20, None,
                                    None) == binding.ISD_E_UNSUPPORTED
     assert lib.isd_set_wait_limit(10) == binding.ISD_E_INVALID
+    # the plan query: an unaligned shape has no plan, a count below 1 is invalid
+    out = (ctypes.c_int32 * len(binding.GEMM_PLAN_FIELDS))()
+    assert lib.isd_gemm_plan(448, 100, 4096, 0, 8, 148, out) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_gemm_plan(448, 128, 96, 0, 8, 148, out) == binding.ISD_E_UNSUPPORTED
+    assert lib.isd_gemm_plan(0, 128, 64, 0, 8, 148, out) == binding.ISD_E_INVALID
+    assert lib.isd_gemm_plan(448, 128, 64, 0, 0, 148, out) == binding.ISD_E_INVALID
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
@@ -174,3 +180,31 @@ def test_oracle_and_product_share_no_code():
     for path in _sources("synth", (".py",)):
         mods = [m.group(2).split(".")[0] for m in imp.finditer(open(path).read())]
         assert "oracle" not in mods and "strided_verify_propose_b200" not in mods, path
+
+
+def test_a_c99_program_calls_the_library(tmp_path):
+    """The header is plain C: a C99 program (tests/c/host_calls.c) compiles
+    against it with -Wall -Wextra -pedantic -Werror, links libisd.so and,
+    without a GPU, gets the same plan and work split as the Python binding."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.dirname(binding.LIB_PATH)
+    exe = str(tmp_path / "host_calls")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "host_calls.c"),
+                    "-L", pkg, "-lisd", f"-Wl,-rpath,{pkg}", "-o", exe], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+    vals = {}
+    for line in filter(None, out):
+        name, v = line.split()
+        vals.setdefault(name, []).append(int(v))
+    assert vals["plan_rc"] == [binding.ISD_OK] and vals["split_rc"] == [binding.ISD_OK]
+    assert vals["refused_rc"] == [binding.ISD_E_UNSUPPORTED]
+    plan = binding.gemm_plan(448, 6144, 4096)
+    assert vals["plan"] == [plan[f] for f in binding.GEMM_PLAN_FIELDS]
+    segs, max_parts = binding.attention_split(3, 7, 32, 8, 128, 64, 64, [100, 1500, 4096], num_sms=16)
+    assert vals["segments"] == [len(segs)] and vals["max_parts"] == [max_parts]
+    assert vals["seg"] == np.asarray(segs).reshape(-1).tolist()
