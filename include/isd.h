@@ -142,7 +142,11 @@ typedef struct isd_ctx isd_ctx;
 int isd_init(const isd_model_cfg *cfg, const isd_weights *w, isd_ctx **out);
 
 /* Attach a gated LoRA (copies the pointer arrays; the tensors stay
- * caller-owned). Steps use it when flags has ISD_USE_LORA. */
+ * caller-owned). Steps use it when flags has ISD_USE_LORA. The library packs
+ * the adapters into fused matrices it owns (freed by isd_destroy).
+ * Errors: ISD_E_UNSUPPORTED for a rank other than 128; ISD_E_INVALID for a
+ * null ctx or lora or a missing pointer; ISD_E_NOMEM when the packed
+ * matrices cannot be allocated; ISD_E_CUDA when packing fails. */
 int isd_load_gated_lora(isd_ctx *ctx, const isd_lora *lora);
 
 /* One ISD step for the whole batch (enqueue only; CUDA-graph capturable).
@@ -156,7 +160,16 @@ int isd_load_gated_lora(isd_ctx *ctx, const isd_lora *lora);
  *  out_committed_dev [B][N] int32: the A_b accepted drafts then the new
  *                final token (A_b + 1 valid entries), or NULL.
  *  status_dev    [1] int32 device status word (bits OR-ed in).
- *  stream        cudaStream_t. */
+ *  stream        cudaStream_t.
+ * Errors (nothing is enqueued): ISD_E_INVALID for a null argument, a batch
+ * outside [1, min(1024, cfg.max_batch)], N outside [1, 8], unknown flag
+ * bits, ISD_USE_LORA without an adapter, SAMPLE proposals without q_cache,
+ * batch * (2N-1) above cfg.max_rows, or an inconsistent isd_kv;
+ * ISD_E_UNSUPPORTED when (2N-1) * n_q_heads / n_kv_heads exceeds 64, the
+ * KV pool holds 2^31 or more rows (layers x pages x KV heads x page_size)
+ * or the block rows exceed the logits workspace (pass logits_out_dev);
+ * ISD_E_CUDA
+ * when a launch fails (the work enqueued before it stays enqueued). */
 int isd_step(isd_ctx *ctx, const isd_batch *batch, const isd_kv *kv, int32_t *pending_dev,
              float *q_cache_dev, const float *uniforms_dev, int32_t *out_accepted_dev,
              int32_t *out_committed_dev, int32_t *status_dev, void *stream);
@@ -166,7 +179,11 @@ int isd_step(isd_ctx *ctx, const isd_batch *batch, const isd_kv *kv, int32_t *pe
  * last prompt token, n_draft = 0 (so the first step is a restart step).
  *  tokens_dev [B][max_len] int32; lens_host [B] host int32, 1 <= len <= max_len.
  * Pages for positions [0, len_b - 1 + 2N - 1) must already be in the page
- * table. Rows are processed in chunks through the same kernels as a step. */
+ * table. Rows are processed in chunks through the same kernels as a step.
+ * Errors: ISD_E_INVALID for a null argument, batch outside [1,
+ * cfg.max_batch], stride_n outside [1, 8], a length outside [1, max_len] or
+ * an inconsistent isd_kv (nothing enqueued); ISD_E_UNSUPPORTED for a KV
+ * pool of 2^31 or more rows; ISD_E_CUDA when a launch fails. */
 int isd_prefill(isd_ctx *ctx, const isd_kv *kv, const int32_t *tokens_dev, int32_t max_len,
                 const int32_t *lens_host, int32_t batch, int32_t stride_n,
                 int32_t *seq_len_dev, int32_t *n_draft_dev, int32_t *pending_dev,
@@ -179,13 +196,21 @@ int isd_last_launch_count(const isd_ctx *ctx);
  * the step's stream (for measurement; off by default, not for use inside a
  * CUDA graph capture). isd_profile_read synchronises on the last recorded
  * event, writes the summed milliseconds and launch counts of each class
- * (ISD_PROF_CLASSES entries) and clears the record. */
+ * (ISD_PROF_CLASSES entries, host arrays) and clears the record.
+ * isd_profile_class_name gives a class's name ("" outside the range).
+ * Errors: ISD_E_INVALID for a null argument; ISD_E_CUDA when an event
+ * query fails. */
 #define ISD_PROF_CLASSES 16
 int isd_profile_enable(isd_ctx *ctx, int enable);
 int isd_profile_read(isd_ctx *ctx, double *total_ms, int32_t *counts);
 const char *isd_profile_class_name(int cls);
 
+/* Text of the calling thread's last error (owned by the library, valid
+ * until that thread's next failing call). */
 const char *isd_last_error(void);
+/* Free the context, its workspace and any packed adapter (NULL is a no-op).
+ * The caller first makes sure no work it enqueued with the context is still
+ * running. Caller-owned buffers are untouched. */
 void isd_destroy(isd_ctx *ctx);
 
 /* Cycle limit of every bounded device wait (an mbarrier phase, a stream-K
