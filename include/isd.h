@@ -230,7 +230,11 @@ int isd_set_wait_limit(long long cycles);
  *  w_dev [n][k] bf16 (nn.Linear layout), x_dev [m][k] bf16,
  *  y_dev [split_k][m][n] fp32: split s holds the partial sum over its share
  *  of k (the caller adds the splits). n % 128 == 0, k % 64 == 0,
- *  1 <= m <= 4096, 1 <= split_k <= 16. */
+ *  1 <= m <= 4096, 1 <= split_k <= 16.
+ * Errors: ISD_E_INVALID for a null operand or a pointer TMA cannot address
+ * (16-byte alignment); ISD_E_UNSUPPORTED outside the limits above or when
+ * split_k leaves a split without K-blocks; ISD_E_CUDA when the launch
+ * fails. */
 int isd_gemm_bf16(const void *w_dev, const void *x_dev, float *y_dev, int32_t m, int32_t n,
                   int32_t k, int32_t split_k, int32_t *status_dev, void *stream);
 
@@ -243,7 +247,10 @@ int isd_gemm_bf16(const void *w_dev, const void *x_dev, float *y_dev, int32_t m,
  *  workspace_dev: isd_gemm_workspace_bytes(m, n, k) bytes (0: none needed,
  *  may be NULL). Its first 4096 bytes must be zero before the first call;
  *  each call leaves them zero, so a workspace serves any number of calls
- *  in stream order (not two calls running at once). */
+ *  in stream order (not two calls running at once).
+ * isd_gemm_workspace_bytes returns 0 for shapes outside the limits too.
+ * Errors of isd_gemm_bf16_single: as isd_gemm_bf16, and ISD_E_INVALID for a
+ * missing or short workspace. */
 size_t isd_gemm_workspace_bytes(int32_t m, int32_t n, int32_t k);
 
 /* The tile plan the library would use for Y = X W^T with m rows, n outputs
@@ -268,7 +275,14 @@ int isd_gemm_bf16_single(const void *w_dev, const void *x_dev, float *y_dev, int
  *  row_pos_dev [B*R] int32: position of each row; a row sees keys t <= pos
  *  (pos < 0: no keys, output 0). Keys live in the pools at layer `layer`.
  *  out_dev [B*R][n_q_heads*head_dim] bf16.
- *  workspace_dev: isd_attention_workspace_bytes(...) bytes of device memory. */
+ *  workspace_dev: isd_attention_workspace_bytes(...) bytes of device memory.
+ * Errors: ISD_E_INVALID for a null argument, head counts that do not
+ * divide, sizes or layer out of range, or a short workspace;
+ * ISD_E_UNSUPPORTED for head_dim other than 64 / 128, a group size other
+ * than 1, 2, 4, 8, rows_per_req * group above 64, a page size other than
+ * 16, 32, 64, or a pool of 2^31 or more rows; ISD_E_CUDA when a launch
+ * fails. A page id outside [0, num_pages) read on the device sets
+ * ISD_DEV_BAD_PAGE and reads zeros. */
 size_t isd_attention_workspace_bytes(int32_t batch, int32_t rows_per_req, int32_t n_q_heads,
                                      int32_t n_kv_heads, int32_t head_dim,
                                      int32_t max_pages_per_req, int32_t page_size);
@@ -310,7 +324,11 @@ int isd_attention_split(int32_t batch, int32_t rows_per_req, int32_t n_q_heads,
  * page bookkeeping: the tail of isd_step without the forward.
  *  logits_dev [B*(2N-1)][vocab] fp32; other arguments as in isd_step (kv
  *  supplies page_table / free list / num_pages / max_pages_per_req / page_size).
- *  workspace_dev: isd_accept_workspace_bytes(B, N, vocab) bytes. */
+ *  workspace_dev: isd_accept_workspace_bytes(B, N, vocab) bytes.
+ * Errors: ISD_E_INVALID for a null argument, batch outside [1, 1024], N
+ * outside [1, 8], page_size below 1, SAMPLE proposals without q_cache, or a
+ * short workspace; ISD_E_UNSUPPORTED for a vocab that is not a multiple of
+ * 4 in [4, 524288]; ISD_E_CUDA when a launch fails. */
 size_t isd_accept_workspace_bytes(int32_t batch, int32_t stride_n, int32_t vocab);
 int isd_accept_propose(const float *logits_dev, const isd_batch *batch, const isd_kv *kv,
                        int32_t page_size, int32_t vocab, int32_t *pending_dev,
