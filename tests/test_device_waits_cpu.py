@@ -41,3 +41,20 @@ def test_no_kernel_traps_or_asserts():
             assert "__trap" not in code and not re.search(r"\btrap;", code), f"{name}:{i + 1}"
             assert not re.search(r"\bassert\s*\(", code), f"{name}:{i + 1}"
             assert "__brkpt" not in code, f"{name}:{i + 1}"
+
+
+def test_no_bulk_copy_uses_cluster_multicast():
+    """Every TMA / bulk copy reads or writes this CTA's (or its pair's) own
+    tile: none carries a multicast qualifier. The only multicast in the
+    kernels is the tcgen05 commit's mbarrier arrive inside a 2-SM pair."""
+    qualifier = "multi" + "cast"
+    copies = 0
+    for name, lines in _sources():
+        for i, line in enumerate(lines):
+            code = line.split("//")[0]
+            if "cp.async.bulk" in code:
+                copies += 1
+                assert qualifier not in code, f"{name}:{i + 1}"
+            elif qualifier + "::" in code:
+                assert "tcgen05.commit" in code, f"{name}:{i + 1}"
+    assert copies >= 3
