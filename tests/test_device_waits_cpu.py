@@ -1,5 +1,5 @@
-"""Static checks of the kernel sources: every device wait is bounded, and no
-kernel traps.
+"""Static checks of the kernel sources: every device wait is bounded, no
+kernel traps, and no bulk copy multicasts across a cluster.
 
 A loop that polls memory another agent writes (an mbarrier phase, a
 stream-K partner's flag) must give up after the library's cycle limit, so a
