@@ -88,6 +88,7 @@ PAGE_PINS = [
     ("covers and never shares",
      lambda: [TP.test_bookkeep_covers_and_never_shares(s) for s in range(5)]),
     ("exhausted pool", TP.test_bookkeep_exhausted_pool_assigns_nothing),
+    ("table row too short", TP.test_bookkeep_table_row_too_short_assigns_nothing),
 ]
 
 # (module, function, expression, its mutant, pins)
@@ -172,6 +173,7 @@ MUTANTS = {
                           PAGE_PINS),
     "exact fit refused": (op, "bookkeep", "free_head + total <= len(free_list)", "free_head + total < len(free_list)",
                           PAGE_PINS),
+    "row width never checked": (op, "bookkeep", " and bool(np.all(want <= table.shape[1]))", "", PAGE_PINS),
     "pages rounded down": (op, "pages_covering", "-(-int(length) // int(page_size))",
                            "int(length) // int(page_size)", PAGE_PINS),
 }

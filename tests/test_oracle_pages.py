@@ -61,6 +61,29 @@ def test_bookkeep_exhausted_pool_assigns_nothing():
     assert [table3[b, need[b]] for b in range(3)] == [99, 98, 97]
 
 
+def test_bookkeep_table_row_too_short_assigns_nothing():
+    """A request whose next block would need more pages than its page-table
+    row holds: no page is handed out to anyone, the free-list head stays,
+    lengths still advance and the step reports failure."""
+    N, P = 4, 16
+    R = 2 * N - 1
+    lens = np.array([3 * P - R, P - R])                 # request 0 fills its 3-page row exactly
+    need = [op.pages_covering(L + R, P) for L in lens]
+    table, _ = synth.page_layout(need, int(sum(need)), 3, 5)
+    free = np.arange(40, 50, dtype=np.int32)            # plenty of free pages
+    A = np.array([N - 1, 0])
+    new_len, table2, head2, ok = op.bookkeep(lens, A, table, free, 0, N, P)
+    assert not ok and head2 == 0 and np.array_equal(table2, table)
+    assert np.array_equal(new_len, lens + 1 + A)
+    # the same step with a 4-page row goes through: request 0 takes its
+    # fourth page and request 1 (length 9 + 1, block of 7) its second, in
+    # request order
+    table4 = np.full((2, 4), -1, np.int64)
+    table4[:, :3] = table
+    _, table5, head5, ok = op.bookkeep(lens, A, table4, free, 0, N, P)
+    assert ok and head5 == 2 and table5[0, 3] == 40 and table5[1, 1] == 41
+
+
 def test_page_layout_is_a_permutation():
     need = [3, 1, 4, 1, 5]
     table, free = synth.page_layout(need, 30, 8, 3)
