@@ -75,13 +75,6 @@ class DenseKV:
     def length(self) -> int:
         return self.n
 
-    def keep(self, n: int) -> None:
-        """Truncate every layer's history to its first n positions."""
-        for l in range(len(self.k)):
-            self.k[l] = self.k[l][:n]
-            self.v[l] = self.v[l][:n]
-        self.n = min(self.n, n)
-
     def copy(self) -> "DenseKV":
         c = DenseKV.__new__(DenseKV)
         c.k = [a.copy() for a in self.k]

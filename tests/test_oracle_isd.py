@@ -145,6 +145,19 @@ def test_a_draft_of_probability_zero_is_never_accepted():
         assert oi.decide(rows, [2], [q], N, u, propose=oi.SAMPLE).accepted == 0
 
 
+def test_layout_rejects_draft_and_uniform_counts_outside_it():
+    """The block holds 0 or N - 1 pending drafts and a step takes 2N - 1
+    uniforms; anything else is refused, not silently padded."""
+    m = _decoder(MICRO, seed=2)
+    st = oi.start_state(m, [1, 2, 3])
+    st.drafts = [4]                                   # 1 draft at N = 3
+    with pytest.raises(ValueError):
+        oi.block_tokens(st, 3, MICRO.mask_token_id)
+    z = np.zeros((5, MICRO.vocab))
+    with pytest.raises(ValueError):
+        oi.decide(z, [], None, 3, [0.5] * 4)          # 4 uniforms at N = 3
+
+
 def test_inverse_cdf_rules():
     w = np.array([0.0, 0.25, 0.0, 0.5, 0.25])
     assert oi.inverse_cdf(w, 0.0)[0] == 1
