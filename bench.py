@@ -89,6 +89,7 @@ def cpu_model() -> str:
 
 
 FALLBACK_PEAKS = dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0)
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e nominal, beside the measured copy peak
 
 
 def load_peaks(path=None):
@@ -450,6 +451,7 @@ def run_cuda(args, ws, rank, local):
             "config": workload_config(args.workload, ws),
             "tokens_per_forward": committed / (args.steps * B * ws),
             "hbm_roofline_fraction_step": hbm_frac_step,
+            "hbm_fraction_step_of_nominal": (step_bytes / (ms_step * 1e-3)) / (NOMINAL_HBM_GBS * 1e9),
             "hbm_roofline_ceiling_step": ceiling,
             "step_algorithmic_bytes": step_bytes,
             "risd_overhead_alpha": (ms / base_ms) if base_ms else None,
@@ -602,6 +604,7 @@ def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
             peak = peaks["hbm"]
             return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak,
                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                    "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                     "peak_kind": f"{peaks['source']} HBM copy (weight streaming, {M} rows)",
                     "avg_launch_ms": avg_s * 1e3, "launches": cnt}
         achieved = gemm_flops[top] / avg_s / 1e12
@@ -617,17 +620,17 @@ def roofline_entry(prof, shape, B, N, lens_steps, steps, peaks):
         tc = (top == "attention" and shape.head_dim == 128 and shape.page_size == 64
               and R * (shape.n_q_heads // shape.n_kv_heads) <= 64)
         if tc:
-            # the timed class also covers the layer's QKV reduction (the
-            # attention kernel's prologue at small batch, its own kernel just
-            # before it otherwise): the QKV projection's fp32 output read
-            # once, q and the block's K/V rows written in bf16
+            # the timed class also covers the layer's QKV reduction (its own
+            # kernel, launched just before the attention): the QKV
+            # projection's fp32 output read once, q and the block's K/V rows
+            # written in bf16
             algo += M * shape.qkv_dim * 4 + M * (shape.q_dim + 2 * shape.kv_dim) * 2
         achieved = algo / avg_s / 1e9
         peak = peaks["hbm"]
         traffic = ATTN_DRAM_PER_KV_BYTE * kv if tc else None
         return {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "algorithmic_bytes": algo,
-                "kv_bytes": kv,
+                "kv_bytes": kv, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                 "traffic_note": "ncu dram read+write of the tcgen05 attention kernel in one "
                                 "capture of the same launch, scaled by this launch's K+V bytes "
                                 "(the QKV reduction's own traffic is not in it)",

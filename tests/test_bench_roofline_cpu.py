@@ -40,6 +40,7 @@ def test_attention_roofline_from_known_times():
     achieved = (kv + qkv) / (per_launch_ms * 1e-3) / 1e9
     assert roof["achieved"] == pytest.approx(achieved)
     assert roof["frac"] == pytest.approx(achieved / PEAKS["hbm"])
+    assert roof["frac_of_nominal"] == pytest.approx(achieved / 8000.0)
     assert roof["traffic"] == pytest.approx(bench.ATTN_DRAM_PER_KV_BYTE * kv)
     assert roof["launches"] == launches and roof["avg_launch_ms"] == pytest.approx(per_launch_ms)
 
