@@ -1,0 +1,74 @@
+"""Undefined names in the Python that only a GPU runs.
+
+bench.py's CUDA arm, the binding's device classes and __graft_entry__.smoke()
+cannot execute on a machine without a GPU, so a misspelt or removed name in
+them would first show on the GPU machine. This walks every function and method
+of those files and checks that each name it reads is a parameter, assigned
+or imported in the function (or an enclosing one), a module-level name, or a
+builtin.
+"""
+import ast
+import builtins
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FILES = ["bench.py", "__graft_entry__.py", os.path.join("strided_verify_propose_b200", "binding.py"),
+         os.path.join("strided_verify_propose_b200", "build.py")]
+
+
+def _bound(node):
+    """Names a function binds anywhere in its body (nested scopes included)."""
+    names = set()
+    for n in ast.walk(node):
+        if isinstance(n, ast.Name) and isinstance(n.ctx, (ast.Store, ast.Del)):
+            names.add(n.id)
+        elif isinstance(n, (ast.Import, ast.ImportFrom)):
+            names.update((a.asname or a.name).split(".")[0] for a in n.names)
+        elif isinstance(n, (ast.FunctionDef, ast.AsyncFunctionDef, ast.Lambda)):
+            if not isinstance(n, ast.Lambda):
+                names.add(n.name)
+            a = n.args
+            names.update(x.arg for x in a.posonlyargs + a.args + a.kwonlyargs)
+            names.update(x.arg for x in (a.vararg, a.kwarg) if x is not None)
+        elif isinstance(n, ast.ClassDef):
+            names.add(n.name)
+        elif isinstance(n, ast.ExceptHandler) and n.name:
+            names.add(n.name)
+        elif isinstance(n, (ast.Global, ast.Nonlocal)):
+            names.update(n.names)
+    return names
+
+
+def _module_names(tree):
+    names = set(dir(builtins)) | {"__file__", "__name__"}
+    for node in tree.body:
+        if isinstance(node, (ast.FunctionDef, ast.AsyncFunctionDef, ast.ClassDef)):
+            names.add(node.name)
+        elif isinstance(node, (ast.Import, ast.ImportFrom)):
+            names.update((a.asname or a.name).split(".")[0] for a in node.names)
+        else:
+            for n in ast.walk(node):
+                if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Store):
+                    names.add(n.id)
+                elif isinstance(n, (ast.Import, ast.ImportFrom)):
+                    names.update((a.asname or a.name).split(".")[0] for a in n.names)
+    return names
+
+
+@pytest.mark.parametrize("rel", FILES)
+def test_no_undefined_names(rel):
+    tree = ast.parse(open(os.path.join(ROOT, rel)).read(), rel)
+    module = _module_names(tree)
+    functions = [n for n in tree.body if isinstance(n, (ast.FunctionDef, ast.AsyncFunctionDef))]
+    for cls in (n for n in tree.body if isinstance(n, ast.ClassDef)):
+        functions += [n for n in cls.body if isinstance(n, (ast.FunctionDef, ast.AsyncFunctionDef))]
+    assert functions
+    missing = []
+    for fn in functions:
+        bound = _bound(fn)
+        for n in ast.walk(fn):
+            if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in bound | module:
+                missing.append(f"{rel}:{n.lineno} {fn.name}: {n.id}")
+    assert not missing, missing
