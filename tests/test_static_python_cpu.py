@@ -1,11 +1,11 @@
 """Undefined names in the Python that only a GPU runs.
 
-bench.py's CUDA arm, the binding's device classes and __graft_entry__.smoke()
-cannot execute on a machine without a GPU, so a misspelt or removed name in
-them would first show on the GPU machine. This walks every function and method
-of those files and checks that each name it reads is a parameter, assigned
-or imported in the function (or an enclosing one), a module-level name, or a
-builtin.
+bench.py's CUDA arm, the binding's device classes, __graft_entry__.smoke()
+and the GPU tests cannot execute on a machine without a GPU, so a misspelt
+or removed name in them would first show on the GPU machine. This walks every
+function and method of those files and checks that each name it reads is a
+parameter, assigned or imported in the function (or an enclosing one), a
+module-level name, or a builtin.
 """
 import ast
 import builtins
@@ -15,7 +15,9 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 FILES = ["bench.py", "__graft_entry__.py", os.path.join("strided_verify_propose_b200", "binding.py"),
-         os.path.join("strided_verify_propose_b200", "build.py")]
+         os.path.join("strided_verify_propose_b200", "build.py"), os.path.join("tests", "_parity.py")] + \
+    sorted(os.path.join("tests", f) for f in os.listdir(os.path.join(ROOT, "tests"))
+           if f.startswith(("test_gpu_", "test_zz_")) and f.endswith(".py"))
 
 
 def _bound(node):
