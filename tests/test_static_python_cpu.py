@@ -1,11 +1,13 @@
-"""Undefined names in the Python that only a GPU runs.
+"""Undefined names and attributes in the Python that only a GPU runs.
 
 bench.py's CUDA arm, the binding's device classes, __graft_entry__.smoke()
 and the GPU tests cannot execute on a machine without a GPU, so a misspelt
 or removed name in them would first show on the GPU machine. This walks every
 function and method of those files and checks that each name it reads is a
 parameter, assigned or imported in the function (or an enclosing one), a
-module-level name, or a builtin.
+module-level name, or a builtin; and that every attribute read from one of
+this repository's modules (the binding, synth, the oracle, the parity
+rules) names something that module defines.
 """
 import ast
 import builtins
@@ -73,4 +75,44 @@ def test_no_undefined_names(rel):
         for n in ast.walk(fn):
             if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in bound | module:
                 missing.append(f"{rel}:{n.lineno} {fn.name}: {n.id}")
+    assert not missing, missing
+
+
+OWN_MODULES = ("strided_verify_propose_b200.binding", "synth", "oracle.isd", "oracle.model",
+               "oracle.pages", "tests._parity", "bench")
+
+
+def _aliases(tree):
+    """local name -> module, for every import of one of this repository's
+    modules anywhere in the file."""
+    out = {}
+    for n in ast.walk(tree):
+        if isinstance(n, ast.ImportFrom) and n.module:
+            for a in n.names:
+                full = f"{n.module}.{a.name}"
+                if full in OWN_MODULES:
+                    out[a.asname or a.name] = full
+        elif isinstance(n, ast.Import):
+            for a in n.names:
+                if a.name in OWN_MODULES:
+                    out[a.asname or a.name.split(".")[0]] = a.name
+    return out
+
+
+@pytest.mark.parametrize("rel", FILES)
+def test_module_attributes_exist(rel):
+    """Every `alias.name` read from one of this repository's modules names
+    something that module defines."""
+    import importlib
+    import sys
+    sys.path.insert(0, ROOT)
+    tree = ast.parse(open(os.path.join(ROOT, rel)).read(), rel)
+    aliases = _aliases(tree)
+    missing = []
+    for n in ast.walk(tree):
+        if (isinstance(n, ast.Attribute) and isinstance(n.value, ast.Name) and n.value.id in aliases
+                and isinstance(n.ctx, ast.Load)):
+            mod = importlib.import_module(aliases[n.value.id])
+            if not hasattr(mod, n.attr):
+                missing.append(f"{rel}:{n.lineno} {n.value.id}.{n.attr}")
     assert not missing, missing
