@@ -5,9 +5,11 @@ and the GPU tests cannot execute on a machine without a GPU, so a misspelt
 or removed name in them would first show on the GPU machine. This walks every
 function and method of those files and checks that each name it reads is a
 parameter, assigned or imported in the function (or an enclosing one), a
-module-level name, or a builtin; and that every attribute read from one of
+module-level name, or a builtin; that every attribute read from one of
 this repository's modules (the binding, synth, the oracle, the parity
-rules) names something that module defines.
+rules) names something that module defines; and that every attribute read
+from an object a function makes with one of the binding's classes is one
+that class defines.
 """
 import ast
 import builtins
@@ -115,4 +117,58 @@ def test_module_attributes_exist(rel):
             mod = importlib.import_module(aliases[n.value.id])
             if not hasattr(mod, n.attr):
                 missing.append(f"{rel}:{n.lineno} {n.value.id}.{n.attr}")
+    assert not missing, missing
+
+
+def _class_members(rel, classes):
+    """Per class of the file: its methods, class-level names and every
+    attribute its methods store on self."""
+    tree = ast.parse(open(os.path.join(ROOT, rel)).read(), rel)
+    out = {}
+    for cls in (n for n in tree.body if isinstance(n, ast.ClassDef) and n.name in classes):
+        names = set()
+        for item in cls.body:
+            if isinstance(item, (ast.FunctionDef, ast.AsyncFunctionDef)):
+                names.add(item.name)
+            elif isinstance(item, ast.Assign):
+                names.update(t.id for t in item.targets if isinstance(t, ast.Name))
+        for n in ast.walk(cls):
+            if (isinstance(n, ast.Attribute) and isinstance(n.ctx, ast.Store)
+                    and isinstance(n.value, ast.Name) and n.value.id == "self"):
+                names.add(n.attr)
+        out[cls.name] = names
+    return out
+
+
+BINDING_CLASSES = ("Model", "KVCache", "StepState", "StepGraph")
+
+
+@pytest.mark.parametrize("rel", FILES)
+def test_binding_object_attributes_exist(rel):
+    """Where a function holds an object made by one of the binding's classes
+    (`st = B.StepState(...)`), every attribute it reads from it is one that
+    class defines."""
+    members = _class_members(os.path.join("strided_verify_propose_b200", "binding.py"), BINDING_CLASSES)
+    assert set(members) == set(BINDING_CLASSES)
+    tree = ast.parse(open(os.path.join(ROOT, rel)).read(), rel)
+    aliases = {k for k, v in _aliases(tree).items() if v == "strided_verify_propose_b200.binding"}
+    in_binding = rel.endswith("binding.py")
+    missing = []
+    for fn in (n for n in ast.walk(tree) if isinstance(n, (ast.FunctionDef, ast.AsyncFunctionDef))):
+        held = {}
+        for n in ast.walk(fn):
+            if (isinstance(n, ast.Assign) and len(n.targets) == 1 and isinstance(n.targets[0], ast.Name)
+                    and isinstance(n.value, ast.Call)):
+                f = n.value.func
+                cls = None
+                if isinstance(f, ast.Attribute) and isinstance(f.value, ast.Name) and f.value.id in aliases:
+                    cls = f.attr
+                elif in_binding and isinstance(f, ast.Name):
+                    cls = f.id
+                if cls in BINDING_CLASSES:
+                    held[n.targets[0].id] = cls
+        for n in ast.walk(fn):
+            if (isinstance(n, ast.Attribute) and isinstance(n.value, ast.Name) and n.value.id in held
+                    and n.attr not in members[held[n.value.id]]):
+                missing.append(f"{rel}:{n.lineno} {n.value.id}.{n.attr} ({held[n.value.id]})")
     assert not missing, missing
