@@ -208,3 +208,51 @@ def test_a_c99_program_calls_the_library(tmp_path):
     segs, max_parts = binding.attention_split(3, 7, 32, 8, 128, 64, 64, [100, 1500, 4096], num_sms=16)
     assert vals["segments"] == [len(segs)] and vals["max_parts"] == [max_parts]
     assert vals["seg"] == np.asarray(segs).reshape(-1).tolist()
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) from include/isd.h."""
+    src = open(os.path.join(ROOT, "include", "isd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"#[^\n]*", "", src)
+    out = {}
+    for ret, name, params in re.findall(r"([A-Za-z_][\w\s\*]*?)\b(isd_\w+)\s*\(([^)]*)\)\s*;", src):
+        ps = [p.strip() for p in params.split(",")] if params.strip() not in ("", "void") else []
+        # drop the parameter name, keep its type
+        types = [re.sub(r"\b\w+$", "", p).strip() if not p.endswith("*") else p for p in ps]
+        out[name] = (ret.strip(), types)
+    return out
+
+
+def _kind_of_c(t):
+    t = t.replace("const", "").strip()
+    if "*" in t:
+        return "ptr"
+    return {"int32_t": "i32", "int": "i32", "size_t": "size", "long long": "i64", "void": "void"}[
+        " ".join(t.split())]
+
+
+def _kind_of_ctypes(t):
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(t, ctypes._Pointer):
+        return "ptr"
+    if t in (ctypes.c_int32, ctypes.c_int):       # both 32-bit on this ABI
+        return "i32"
+    return {ctypes.c_size_t: "size", ctypes.c_longlong: "i64"}[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype's parameters and return type, by kind (pointer, 32-bit
+    int, size_t, long long, void), equal the binding's ctypes declaration."""
+    lib = binding.lib()
+    protos = _prototypes()
+    assert set(protos) == set(_declared_functions())
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        want = [_kind_of_c(p) for p in params]
+        if params:
+            assert fn.argtypes is not None, f"{name}: no argtypes"
+            got = [_kind_of_ctypes(t) for t in fn.argtypes]
+            assert got == want, (name, got, want)
+        assert _kind_of_ctypes(fn.restype) == _kind_of_c(ret), (name, fn.restype, ret)
