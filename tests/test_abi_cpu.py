@@ -256,3 +256,55 @@ def test_binding_signatures_match_the_header():
             got = [_kind_of_ctypes(t) for t in fn.argtypes]
             assert got == want, (name, got, want)
         assert _kind_of_ctypes(fn.restype) == _kind_of_c(ret), (name, fn.restype, ret)
+
+
+def _header_structs():
+    """struct name -> field names in declaration order, from include/isd.h."""
+    src = open(os.path.join(ROOT, "include", "isd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for body, name in re.findall(r"typedef struct\s*\{(.*?)\}\s*(\w+)\s*;", src, flags=re.S):
+        fields = []
+        for decl in filter(None, (d.strip() for d in body.split(";"))):
+            # the type ends where the first declarator's name begins
+            m = re.match(r"^(.*?[\s\*])(\w+\s*(\[\d+\])?\s*(,\s*\**\s*\w+\s*(\[\d+\])?\s*)*)$", decl, flags=re.S)
+            assert m, decl
+            fields += [re.sub(r"[\s\*]|\[\d+\]", "", d) for d in m.group(2).split(",")]
+        out[name] = fields
+    return out
+
+
+def test_struct_field_offsets_match_the_c_compiler(tmp_path):
+    """Each ctypes mirror's fields sit at the offsets, and have the sizes, gcc
+    gives the header's struct, field by field; the struct sizes agree."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    structs = _header_structs()
+    mirrors = {"isd_model_cfg": binding.ModelCfg, "isd_weights": binding.Weights,
+               "isd_batch": binding.Batch, "isd_kv": binding.KV, "isd_lora": binding.Lora}
+    assert set(structs) == set(mirrors)
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "isd.h"', "int main(void) {"]
+    for s, fields in structs.items():
+        lines.append(f'  printf("{s} sizeof %zu\\n", sizeof({s}));')
+        for f in fields:
+            lines.append(f'  printf("{s} {f} %zu %zu\\n", offsetof({s}, {f}), sizeof((({s} *)0)->{f}));')
+    lines += ["  return 0;", "}"]
+    c = tmp_path / "offsets.c"
+    c.write_text("\n".join(lines) + "\n")
+    exe = str(tmp_path / "offsets")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(c),
+                    "-o", exe], check=True)
+    got = {}
+    for line in subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n"):
+        if line:
+            s, f, *v = line.split()
+            got.setdefault(s, []).append((f, tuple(int(x) for x in v)))
+    for s, mirror in mirrors.items():
+        size = dict(got[s])["sizeof"][0]
+        fields = [v for f, v in got[s] if f != "sizeof"]
+        assert ctypes.sizeof(mirror) == size, s
+        mine = [(getattr(mirror, name).offset, getattr(mirror, name).size) for name, *_ in mirror._fields_]
+        assert mine == fields, (s, mine, fields)
