@@ -308,3 +308,17 @@ def test_struct_field_offsets_match_the_c_compiler(tmp_path):
         assert ctypes.sizeof(mirror) == size, s
         mine = [(getattr(mirror, name).offset, getattr(mirror, name).size) for name, *_ in mirror._fields_]
         assert mine == fields, (s, mine, fields)
+
+
+def test_accept_workspace_is_the_size_the_header_states():
+    """batch * (2N-1) * ceil(vocab / 8192) chunk statistics of 16 bytes, then
+    4 bytes per request, plus at most alignment padding; the headline shape
+    fits the fixed 4 MiB array of the no-allocation entry point."""
+    lib = binding.lib()
+    rng = np.random.default_rng(4)
+    for _ in range(200):
+        B, N, V = int(rng.integers(1, 1025)), int(rng.integers(1, 9)), int(rng.integers(1, 131073)) * 4
+        want = B * (2 * N - 1) * (-(-V // 8192)) * 16 + 4 * B
+        got = lib.isd_accept_workspace_bytes(B, N, V)
+        assert want <= got <= want + 512, (B, N, V, got, want)
+    assert lib.isd_accept_workspace_bytes(1024, 4, 151936) <= 4 << 20
